@@ -1,0 +1,170 @@
+"""CPU oracle for the paged-KV decode path (TEST INFRASTRUCTURE).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg (``bench.py --impl reference`` and the ``cpu_baseline`` field) may import
+this package.  The product path never does: the CUDA library fails loudly
+when it is missing instead of falling back to anything here.
+
+Contents
+--------
+- ``pa_oracle.c`` (compiled to ``liboracle.so`` by :func:`build`): write,
+  copy-on-write block copy and decode attention in plain C, fp64.
+- :func:`slot_of` / :func:`slot_mapping` / :func:`blocks_for` /
+  :func:`tail_waste`: the slot, block-count and waste formulas, in Python.
+- ``oracle.pool``: a pure-Python model of the block pool (free list,
+  reference counts, append with copy-on-write, fork, release).
+
+How each piece is pinned to something other than itself (the tests under
+``tests/test_oracle_*.py`` and ``tests/test_pool*.py``):
+- write / copy: worked examples, the fancy-index definition of the copy,
+  negative-slot skipping, byte-exact NaN payload preservation;
+- decode: the contiguous special case against ``torch``'s scaled dot-product
+  attention in float64, closed forms (all-equal keys give the mean of V; one
+  dominant key gives its V row; a single token gives V_0 exactly), invariance
+  under any permutation of physical blocks and any block size, brute force on
+  tiny inputs, NaN poison in unused storage;
+- slot / block / waste formulas: the worked examples printed on the pages
+  (slot 30,608 for request r7; cdiv(4097, 16) = 257; tail waste 15/1/0/15;
+  the simulator's 4 blocks, 2 slots of slack, 50 slots of contiguous waste);
+- pool: the pages' invariants, their CPU-allocator trace, and refcounts under
+  sharing and copy-on-write.
+No oracle function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile pa_oracle.c into liboracle.so (plain gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                               "-o", _LIB_PATH, _SRC, "-lm"])
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        lib.oracle_write_kv.argtypes = [P, P, P, i64, i64, i64, P, P]
+        lib.oracle_write_kv.restype = ctypes.c_int
+        lib.oracle_copy_blocks.argtypes = [P, i64, i64, i64, P, P]
+        lib.oracle_copy_blocks.restype = ctypes.c_int
+        lib.oracle_decode.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
+                                      ctypes.c_double, P, i64, P]
+        lib.oracle_decode.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _req(a, dtype):
+    a = np.asarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    assert a.flags.c_contiguous
+    return a
+
+
+# ----------------------------------------------------------------------------
+# Formulas of the paging scheme
+# ----------------------------------------------------------------------------
+
+
+def blocks_for(n: int, block_size: int) -> int:
+    """ceil(n / B): blocks a sequence of n tokens occupies ("Memory
+    management", Maths)."""
+    return -(-n // block_size)
+
+
+def tail_waste(n: int, block_size: int) -> int:
+    """B*ceil(n/B) - n unused slots in the last block ("Memory management",
+    Maths; "PagedAttention: fragmentation, blocks, block tables", Tail waste
+    has a distribution)."""
+    return block_size * blocks_for(n, block_size) - n
+
+
+def slot_of(table_row, pos: int, block_size: int) -> int:
+    """slot = table[pos // B] * B + pos % B ("PagedAttention: fragmentation,
+    blocks, block tables", section 3 "The slot mapping")."""
+    return int(table_row[pos // block_size]) * block_size + pos % block_size
+
+
+def slot_mapping(table_rows, positions, block_size: int) -> np.ndarray:
+    """One int64 slot per (row, position) pair; position -1 marks padding and
+    maps to -1 (any negative value means "skip")."""
+    out = np.empty(len(positions), dtype=np.int64)
+    for i, (row, pos) in enumerate(zip(table_rows, positions)):
+        out[i] = -1 if pos < 0 else slot_of(row, pos, block_size)
+    return out
+
+
+# ----------------------------------------------------------------------------
+# Device operations, on host arrays
+# ----------------------------------------------------------------------------
+
+
+def write_kv(k, v, slots, k_cache, v_cache) -> None:
+    """In place: k_cache.reshape(-1, H_kv*D)[slots[i]] = k[i] (same for V);
+    negative slots skipped."""
+    k = _req(k, np.uint16); v = _req(v, np.uint16); slots = _req(slots, np.int64)
+    k_cache = _req(k_cache, np.uint16); v_cache = _req(v_cache, np.uint16)
+    row = int(np.prod(k.shape[1:])) if k.ndim > 1 else 1
+    num_slots = k_cache.size // row
+    rc = _load().oracle_write_kv(_ptr(k), _ptr(v), _ptr(slots), len(slots), row, num_slots,
+                                 _ptr(k_cache), _ptr(v_cache))
+    if rc:
+        raise ValueError("slot out of range")
+
+
+def copy_blocks(pairs, k_cache, v_cache) -> None:
+    """In place: cache[dst] = cache[src] for each (src, dst) pair, all sources
+    read before any destination is written."""
+    pairs = _req(np.ascontiguousarray(pairs, dtype=np.int64).reshape(-1, 2), np.int64)
+    k_cache = _req(k_cache, np.uint16); v_cache = _req(v_cache, np.uint16)
+    nb = k_cache.shape[0]
+    rc = _load().oracle_copy_blocks(_ptr(pairs), len(pairs), k_cache.size // nb, nb,
+                                    _ptr(k_cache), _ptr(v_cache))
+    if rc:
+        raise ValueError("block id out of range")
+
+
+def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, which=None) -> np.ndarray:
+    """fp64 paged decode attention.  q: uint16 [S, H_q, D]; caches uint16
+    [NB, B, H_kv, D]; block_tables int32 [S, W]; seq_lens int32 [S].  Returns
+    float64 [S, H_q, D] (rows outside ``which`` are NaN)."""
+    q = _req(q, np.uint16); k_cache = _req(k_cache, np.uint16); v_cache = _req(v_cache, np.uint16)
+    block_tables = _req(np.ascontiguousarray(block_tables, dtype=np.int32), np.int32)
+    seq_lens = _req(np.ascontiguousarray(seq_lens, dtype=np.int32), np.int32)
+    S, Hq, D = q.shape
+    NB, B, Hkv, D2 = k_cache.shape
+    assert D2 == D and Hq % Hkv == 0 and len(seq_lens) == S and block_tables.shape[0] == S
+    out = np.full((S, Hq, D), np.nan, dtype=np.float64)
+    if which is not None:
+        w = np.ascontiguousarray(which, dtype=np.int32).reshape(-1, 2)
+        wp, nw = _ptr(w), len(w)
+    else:
+        w, wp, nw = None, None, 0
+    rc = _load().oracle_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                               block_tables.shape[1], _ptr(seq_lens), S, Hq, Hkv, D, B, NB,
+                               float(scale), wp, nw, _ptr(out))
+    if rc == -1:
+        raise ValueError("block id out of range or table too narrow")
+    if rc:
+        raise MemoryError("oracle_decode")
+    return out
