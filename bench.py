@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark: one decode step of Llama-3-8B-shaped paged attention on B200.
+
+A step runs, for each of --layers layers (distinct KV caches of the full
+26,785-block pool, so the timed inputs are far larger than L2): the
+copy-on-write copies the step queued (none for the chat workload), the
+slot-mapped KV write of one new token per sequence, and paged decode
+attention.  Inputs are resident in HBM when the timed region starts.
+
+  value  = algorithmic bytes of the step (unique KV bytes the decode reads
+           + the write's and the copies' bytes) / step time, in GB/s;
+  e2e    = the same bytes / time of the same step driven from pinned host
+           buffers (per layer: q, k, v in; out back), copies included;
+  roofline = the decode kernel alone: unique KV bytes per launch / its mean
+           duration (CUDA events on its stream) vs. measured HBM peak.
+
+--impl reference times the CPU oracle (one thread) on a bounded sample of
+the same workload.  With torchrun (N > 1) every rank runs its own replica
+(the path does not shard; no collective is needed) and the time is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "paged decode attention: KV HBM GB/s & % of B200 peak; decode tokens/s per layer"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+WORKLOAD_TEXT = {
+    "chat": "Llama-3-8B chat decode: 64 seqs, len U[512,612], 32 q / 8 KV heads, d=128, block 16, "
+            "26,785-block pool, shuffled free list",
+    "long": "Long-context decode: 8 seqs {32768 x4, 8192 x4}, 32 q / 8 KV heads, d=128, block 16, "
+            "26,785-block pool",
+    "prefix": "Prefix sharing + CoW: 256 seqs, 2040-token shared prefix, suffix U[1,256], "
+              "32 q / 8 KV heads, d=128, block 16",
+    "tiny": "Tiny: 4 seqs {2,18,34,101}, 8 q / 2 KV heads, d=128, block 16, 64-block pool",
+}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="chat")
+    ap.add_argument("--layers", type=int, default=32)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--part-tokens", type=int, default=0, help="split-K partition size (0 = automatic)")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, torch copy_ read+write)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.uuid = None
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            pass
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [r.split(", ") for r in self.lines if r.count(",") >= 8]
+        if self.uuid:
+            mine = [r for r in rows if r[0].strip() == self.uuid]
+            rows = mine or rows
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- bytes
+def algorithmic_bytes(st) -> dict:
+    """Bytes the step must move, per layer."""
+    H, D, B = st.num_kv_heads, st.head_dim, st.block_size
+    row = H * D * 2  # one token's K (or V) row, bf16
+    slots = []
+    for s in range(len(st.ids)):
+        n = int(st.seq_lens_np[s])
+        pos = np.arange(n, dtype=np.int64)
+        slots.append(st.block_tables_np[s, pos // B].astype(np.int64) * B + pos % B)
+    uniq = np.unique(np.concatenate(slots)).size if slots else 0
+    logical = int(st.seq_lens_np.sum())
+    T = st.slot_mapping_np.size
+    P = st.cow_pairs_np.shape[0]
+    return {
+        "decode_kv": uniq * row * 2,  # K and V, each unique slot once
+        "decode_kv_logical": logical * row * 2,
+        "write": T * row * 2 * 2,  # K and V rows read and written
+        "copy": P * B * row * 2 * 2,  # K and V blocks read and written
+        "q_out": 2 * st.q.numel() * 2,
+        "table": int(sum(-(-int(n) // B) for n in st.seq_lens_np)) * 4,
+    }
+
+
+# --------------------------------------------------------------------------- ours
+def run_ours(args, world, rank, local):
+    import synth
+    import paged_kv_cache_333_b200 as pa
+    from paged_kv_cache_333_b200.workload import stage
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if args.part_tokens:
+        pa.pa_decode_set_partition_tokens(args.part_tokens)
+    w = synth.by_name(args.config)
+    st = stage(w, dev, layers=args.layers)
+    L = args.layers
+    nbytes = algorithmic_bytes(st)
+    step_bytes = L * (nbytes["decode_kv"] + nbytes["write"] + nbytes["copy"])
+    stream = torch.cuda.current_stream(dev)
+    S = len(st.ids)
+    has_pairs = st.cow_pairs.shape[0] > 0
+    split = st.workspace is not None
+    launches_per_layer = 2 + (1 if split else 0) + (1 if has_pairs else 0)
+
+    def one_layer(l, ev0=None, ev1=None):
+        kc, vc = st.caches[l]
+        if has_pairs:
+            pa.pa_copy_blocks(kc, vc, st.cow_pairs)
+        pa.pa_write_kv(st.k_new, st.v_new, st.slot_mapping, kc, vc)
+        if ev0 is not None:
+            ev0.record(stream)
+        pa.pa_decode(st.q, kc, vc, st.block_tables, st.seq_lens, st.scale, out=st.out,
+                     max_seq_len=st.max_seq_len, workspace=st.workspace)
+        if ev1 is not None:
+            ev1.record(stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        for l in range(L):
+            one_layer(l)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error(clear=True) == 0
+
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K * L)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for k in range(K):
+        for l in range(L):
+            e0, e1 = evs[k * L + l]
+            one_layer(l, e0, e1)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    dec_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_max = ms_total
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_step = ms_max / K
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    dec_mean_ms = statistics.mean(dec_ms)
+    peak, peak_src = measured_peak()
+    achieved = nbytes["decode_kv"] / (dec_mean_ms * 1e-3) / 1e9
+
+    # ---- end to end: the same step from pinned host buffers -------------------
+    e2e = None
+    if not args.no_e2e:
+        q_h = st.q.cpu().pin_memory()
+        k_h, v_h = st.k_new.cpu().pin_memory(), st.v_new.cpu().pin_memory()
+        sm_h = st.slot_mapping.cpu().pin_memory()
+        bt_h, sl_h = st.block_tables.cpu().pin_memory(), st.seq_lens.cpu().pin_memory()
+        out_h = torch.empty_like(st.out, device="cpu").pin_memory()
+        q_d, k_d, v_d = torch.empty_like(st.q), torch.empty_like(st.k_new), torch.empty_like(st.v_new)
+        sm_d, bt_d, sl_d = (torch.empty_like(st.slot_mapping), torch.empty_like(st.block_tables),
+                            torch.empty_like(st.seq_lens))
+        pairs_h = st.cow_pairs.cpu().pin_memory() if has_pairs else None
+        pairs_d = torch.empty_like(st.cow_pairs) if has_pairs else None
+
+        def e2e_step():
+            sm_d.copy_(sm_h, non_blocking=True)
+            bt_d.copy_(bt_h, non_blocking=True)
+            sl_d.copy_(sl_h, non_blocking=True)
+            if has_pairs:
+                pairs_d.copy_(pairs_h, non_blocking=True)
+            for l in range(L):
+                kc, vc = st.caches[l]
+                q_d.copy_(q_h, non_blocking=True)
+                k_d.copy_(k_h, non_blocking=True)
+                v_d.copy_(v_h, non_blocking=True)
+                if has_pairs:
+                    pa.pa_copy_blocks(kc, vc, pairs_d)
+                pa.pa_write_kv(k_d, v_d, sm_d, kc, vc)
+                pa.pa_decode(q_d, kc, vc, bt_d, sl_d, st.scale, out=st.out, max_seq_len=st.max_seq_len,
+                             workspace=st.workspace)
+                out_h.copy_(st.out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        t0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = t0.elapsed_time(t1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = (sm_h.numel() * 8 + bt_h.numel() * 4 + sl_h.numel() * 4 + (pairs_h.numel() * 8 if has_pairs else 0)
+               + L * (q_h.numel() + k_h.numel() + v_h.numel()) * 2)
+        d2h = L * out_h.numel() * 2
+        e2e = {"value": round(world * step_bytes / (e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e_ms / K, 4)}
+        assert pa.pa_get_device_error(clear=True) == 0
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 K/V/q; seeded shuffled free list)",
+        "config": {
+            "workload": WORKLOAD_TEXT.get(args.config, args.config),
+            "layers_per_step": L,
+            "batch": S,
+            "block_size": st.block_size,
+            "num_blocks": st.num_blocks,
+            "num_q_heads": st.num_q_heads,
+            "num_kv_heads": st.num_kv_heads,
+            "head_dim": st.head_dim,
+            "max_seq_len": st.max_seq_len,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"inputs larger than L2: {L} distinct layer caches, "
+                  f"{L * nbytes['decode_kv'] / 1e9:.2f} GB of KV touched per step",
+        },
+        "pct_of_peak": {"measured": round(100 * value / world / peak, 2),
+                        "nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2)},
+        "decode_tokens_per_s_per_layer": round(world * S / (ms_step / L * 1e-3), 1),
+        "per_op_bytes_per_layer": nbytes,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "pa_decode (partition kernel" + (" + LSE merge)" if split else ")"),
+                     "mean_launch_us": round(dec_mean_ms * 1e3, 3),
+                     "bytes_per_launch": nbytes["decode_kv"], "peak_source": peak_src},
+        "e2e": e2e,
+        "gpu_launches": K * L * launches_per_layer,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# --------------------------------------------------------------------------- oracle
+def _oracle_setup(w):
+    from tests.oracle_stage import stage_oracle
+    ref = stage_oracle(w, decode=False)
+    n = ref["seq_lens"]
+    B = w.shape.block_size
+    row = w.shape.num_kv_heads * w.shape.head_dim * 2
+    pos_slots = [ref["block_tables"][s, np.arange(int(x)) // B].astype(np.int64) * B + np.arange(int(x)) % B
+                 for s, x in enumerate(n)]
+    uniq = np.unique(np.concatenate(pos_slots)).size
+    return ref, uniq * row * 2
+
+
+def _oracle_layer(w, ref, sample_seqs):
+    import oracle
+    which = np.array([(s, j) for s in sample_seqs for j in range(w.shape.num_q_heads)], np.int32)
+    oracle.decode(w.q, ref["k_cache"], ref["v_cache"], ref["block_tables"], ref["seq_lens"], w.scale, which)
+
+
+def cpu_baseline(w, seconds: float) -> dict:
+    """The oracle (plain C, fp64, one thread) on a bounded sample: whole
+    layers of the same workload, repeated until `seconds` have passed."""
+    ref, kv_bytes = _oracle_setup(w)
+    S = len(w.seq_ids)
+    t0 = time.perf_counter()
+    layers = 0
+    while True:
+        _oracle_layer(w, ref, range(S))
+        layers += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(layers * kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{layers} full layer(s) of the same workload ({S} seqs x {w.shape.num_q_heads} heads), "
+                      f"{dt:.1f} s, decode only"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import synth
+    w = synth.by_name(args.config)
+    ref, kv_bytes = _oracle_setup(w)
+    S = len(w.seq_ids)
+    # one step = one full layer of the workload's decode, on one host thread
+    for _ in range(args.warmup):
+        _oracle_layer(w, ref, range(min(S, 8)))
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        _oracle_layer(w, ref, range(S))
+        times.append(time.perf_counter() - t)
+    ms_step = 1e3 * statistics.mean(times)
+    value = kv_bytes / (ms_step * 1e-3) / 1e9
+    sample = f"{args.steps} steps of one full layer ({S} seqs x {w.shape.num_q_heads} heads), decode only"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config), "layers_per_step": 1},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "decode_tokens_per_s_per_layer": round(S / (ms_step * 1e-3), 2),
+    }), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_env()
+    if world > 1 and args.impl == "ours":
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

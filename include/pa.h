@@ -1,0 +1,160 @@
+/*
+ * pa.h -- C ABI of the paged-KV decode path on NVIDIA B200 (sm_100a).
+ *
+ * Three device operations keep a block-major KV pool consistent and read it:
+ *   pa_write_kv     store this step's K/V rows at their slots;
+ *   pa_copy_blocks  copy-on-write block copies;
+ *   pa_decode       decode attention gathered through the block table.
+ *
+ * Memory: every pointer argument named without a host_ prefix is a DEVICE
+ * pointer (cudaMalloc / torch CUDA memory) on the current device.  The caller
+ * allocates and owns every buffer; the library allocates no device memory.
+ * bf16 arrays hold IEEE bfloat16 bit patterns.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  Every call only enqueues work and returns; results are ready when
+ * the stream reaches that point.
+ *
+ * Status: 0 = success; a negative PA_E* code = nothing was enqueued.
+ * Arguments that live on the device (slots, block ids, lengths, copy pairs)
+ * cannot be checked on the host without a synchronisation; the kernels check
+ * them instead and never touch memory outside the caller's arrays: an
+ * out-of-range value is skipped (write, copy) or replaced by an in-range
+ * dummy (decode) and recorded in the device error word read by
+ * pa_get_device_error.  No kernel traps.
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    PA_OK = 0,
+    PA_EINVAL = -1,       /* null pointer, negative size, num_q_heads % num_kv_heads != 0 */
+    PA_EUNSUPPORTED = -2, /* head_dim != 128, block_size not a power of two in [1, 64],
+                             group size not in {1, 2, 4, 8}, pointer not 16-byte aligned */
+    PA_EWORKSPACE = -3,   /* workspace smaller than pa_decode_workspace_bytes() */
+    PA_ECUDA = -4         /* a CUDA call or launch failed (see pa_last_cuda_error) */
+};
+
+/* Bits of the device error word. */
+enum {
+    PA_DEVERR_SLOT = 1,       /* pa_write_kv: slot >= num_blocks * block_size (row skipped) */
+    PA_DEVERR_BLOCK_ID = 2,   /* pa_decode: block id outside [0, num_blocks) (block 0 read instead) */
+    PA_DEVERR_SEQ_LEN = 4,    /* pa_decode: seq_len < 0, > max_seq_len, or needing more than
+                                 max_blocks_per_seq table entries (clamped) */
+    PA_DEVERR_COPY_PAIR = 8,  /* pa_copy_blocks: id outside [0, num_blocks) (pair skipped) */
+    PA_DEVERR_TIMEOUT = 16    /* a pipeline wait gave up after its time limit */
+};
+
+/* One layer's paged KV cache.  k_cache and v_cache are separate tensors of
+ * shape [num_blocks][block_size][num_kv_heads][head_dim] bf16, block-major:
+ * block i owns one contiguous range, and row `slot` of the cache viewed as
+ * [num_blocks*block_size][num_kv_heads*head_dim] is token slot `slot`
+ * ("PagedAttention: fragmentation, blocks, block tables", section 3 "The
+ * slot mapping": block-major backing storage; the r7 walkthrough stores the
+ * token "at flat row 30,608"). */
+typedef struct pa_cache {
+    void *k_cache;
+    void *v_cache;
+    int64_t num_blocks;
+    int32_t block_size;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+} pa_cache_t;
+
+/*
+ * pa_write_kv -- the KV-cache write of one step.
+ * Defined by: "PagedAttention: fragmentation, blocks, block tables",
+ * section 3 "The slot mapping" (the kernel writes new K/V at
+ * slot_mapping[i]; every layer writes the same slot, only the tensor
+ * differs; padded positions carry a PAD value).
+ *   k, v          [num_tokens][num_kv_heads][head_dim] bf16, contiguous.
+ *   slot_mapping  [num_tokens] int64; row i goes to cache row slot_mapping[i];
+ *                 a negative slot is padding and is skipped.  Slots must be
+ *                 distinct (two tokens to one slot: either row may win).
+ * Bit-exact copy of the rows; no arithmetic.
+ */
+PA_API int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping, int64_t num_tokens,
+                const pa_cache_t *cache, void *stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copies.
+ * Defined by: "PagedAttention: fragmentation, blocks, block tables",
+ * copy-on-write passage (a list of (src_block_id, dst_block_id) pairs runs
+ * before the forward pass reads the cache; one assignment
+ * blocks[dst] = blocks[src] over the block-major storage).
+ *   src_dst_pairs [num_pairs][2] int64 (src, dst).  Every dst must be
+ *                 distinct and no dst may also be a src (the pool's pairs
+ *                 always are); the whole block -- all block_size slots, K
+ *                 and V -- is copied bit for bit.
+ */
+PA_API int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
+                   void *stream);
+
+/*
+ * Bytes of scratch pa_decode needs for this batch shape (0 when no sequence
+ * is long enough to be split across CTAs).  Depends only on host values, so
+ * it can be called once per shape and the buffer reused.
+ */
+PA_API size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
+                                 const pa_cache_t *cache);
+
+/*
+ * pa_decode -- decode attention over the paged cache, one query token per
+ * sequence.
+ * Defined by: "PagedAttention: fragmentation, blocks, block tables",
+ * attention-metadata passage (block_table is [num_reqs, max_num_blocks_per_req]
+ * int32; the kernel gathers past K/V by walking row r for
+ * ceil(seq_lens[r] / block_size) entries; max_seq_len may be an upper bound)
+ * and section 2 "The block table" (position p lives in entry p / B at
+ * offset p % B); "The pantry of pigeonholes", "The mechanism: blocks, block
+ * table and the kernel gather".
+ * For sequence s and query head j, with h = j / (num_q_heads / num_kv_heads):
+ *   out[s][j] = sum_t softmax_t(scale * q[s][j] . K[s,h,t]) V[s,h,t],
+ * over the seq_lens[s] tokens of s in logical order; fp32 accumulation,
+ * one rounding to bf16 at the end.  A sequence of length 0 gives zeros.
+ *   q             [num_seqs][num_q_heads][head_dim] bf16.
+ *   block_tables  [num_seqs][max_blocks_per_seq] int32; only the first
+ *                 ceil(seq_lens[s] / block_size) entries of row s are read.
+ *   seq_lens      [num_seqs] int32 on the device, each <= max_seq_len.
+ *   max_seq_len   host-side upper bound of seq_lens (sizes the grid without
+ *                 reading the device).
+ *   out           [num_seqs][num_q_heads][head_dim] bf16.
+ *   workspace     device scratch of at least pa_decode_workspace_bytes(...)
+ *                 bytes (may be NULL when that is 0).  Calls that overlap on
+ *                 the GPU must use different workspaces.
+ */
+PA_API int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+              int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+              int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/* Tokens per split-K partition used by pa_decode: 0 = automatic (the
+ * default), otherwise a multiple of 64.  Host-side setting, process wide;
+ * returns the previous value.  For tuning and tests. */
+PA_API int32_t pa_decode_set_partition_tokens(int32_t tokens);
+
+/* Read (and with clear != 0, reset) the device error word of the current
+ * device.  Synchronises the device.  Returns PA_OK or PA_ECUDA. */
+PA_API int pa_get_device_error(int32_t *host_code, int clear);
+
+/* The last CUDA error string seen by a PA_ECUDA return (static storage). */
+PA_API const char *pa_last_cuda_error(void);
+PA_API const char *pa_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PA_H */

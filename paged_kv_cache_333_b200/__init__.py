@@ -1,0 +1,22 @@
+"""Paged-KV decode path for NVIDIA B200 (sm_100a).
+
+The device path is the C-ABI library ``libpa.so`` (include/pa.h): slot-mapped
+KV write, copy-on-write block copy, and paged decode attention, all in
+hand-written CUDA kernels.  ``libpa_pool.so`` (include/pa_pool.h) is the host
+block pool that produces block tables, slot mappings and copy pairs.  The
+Python functions here only marshal arguments; there is no fallback path, and
+importing the package fails if the libraries have not been built
+(``python paged_kv_cache_333_b200/build.py``).
+"""
+from ._abi import (PA_DEVERR_BLOCK_ID, PA_DEVERR_COPY_PAIR, PA_DEVERR_SEQ_LEN, PA_DEVERR_SLOT,
+                   PA_DEVERR_TIMEOUT, PaError, make_cache, pa_copy_blocks, pa_decode,
+                   pa_decode_set_partition_tokens, pa_decode_workspace_bytes, pa_get_device_error,
+                   pa_write_kv)
+from .pool import BlockPool, PoolError
+
+__all__ = [
+    "pa_write_kv", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
+    "pa_decode_set_partition_tokens", "pa_get_device_error", "make_cache", "PaError",
+    "BlockPool", "PoolError", "PA_DEVERR_SLOT", "PA_DEVERR_BLOCK_ID", "PA_DEVERR_SEQ_LEN",
+    "PA_DEVERR_COPY_PAIR", "PA_DEVERR_TIMEOUT",
+]

@@ -1,0 +1,161 @@
+"""ctypes binding of libpa.so (include/pa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (PyTorch provides device memory and
+streams); each call passes ``data_ptr()`` and the current stream's handle.
+Importing this module fails if libpa.so has not been built: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_333_b200/build.py` "
+                      "(there is no fallback path)")
+lib = ctypes.CDLL(LIB_PATH)
+
+PA_OK, PA_EINVAL, PA_EUNSUPPORTED, PA_EWORKSPACE, PA_ECUDA = 0, -1, -2, -3, -4
+PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+
+EXPORTED = ("pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_bytes", "pa_decode",
+            "pa_decode_set_partition_tokens", "pa_get_device_error", "pa_last_cuda_error",
+            "pa_status_str")
+
+
+class PaCache(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("num_blocks", ctypes.c_int64), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_i32, _i64 = ctypes.c_int32, ctypes.c_int64
+lib.pa_write_kv.argtypes = [_P, _P, _P, _i64, ctypes.POINTER(PaCache), _P]
+lib.pa_write_kv.restype = ctypes.c_int
+lib.pa_copy_blocks.argtypes = [ctypes.POINTER(PaCache), _P, _i64, _P]
+lib.pa_copy_blocks.restype = ctypes.c_int
+lib.pa_decode_workspace_bytes.argtypes = [_i32, _i32, _i32, ctypes.POINTER(PaCache)]
+lib.pa_decode_workspace_bytes.restype = ctypes.c_size_t
+lib.pa_decode.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
+                          _P, _P, ctypes.c_size_t, _P]
+lib.pa_decode.restype = ctypes.c_int
+lib.pa_decode_set_partition_tokens.argtypes = [_i32]
+lib.pa_decode_set_partition_tokens.restype = _i32
+lib.pa_get_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
+lib.pa_get_device_error.restype = ctypes.c_int
+lib.pa_last_cuda_error.argtypes = []
+lib.pa_last_cuda_error.restype = ctypes.c_char_p
+lib.pa_status_str.argtypes = [ctypes.c_int]
+lib.pa_status_str.restype = ctypes.c_char_p
+
+
+class PaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        msg = f"{what}: {lib.pa_status_str(code).decode()} ({code})"
+        if code == PA_ECUDA:
+            msg += f": {lib.pa_last_cuda_error().decode()}"
+        super().__init__(msg)
+        self.code = code
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != PA_OK:
+        raise PaError(rc, what)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> PaCache:
+    """Describe one layer's K and V caches ([num_blocks, block_size, H_kv, D] bf16)."""
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
+        raise ValueError("k_cache and v_cache must both be [num_blocks, block_size, num_kv_heads, head_dim]")
+    nb, bs, hkv, d = k_cache.shape
+    return PaCache(_dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+                   nb, bs, hkv, d)
+
+
+def pa_write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """k_cache.view(-1, H_kv, D)[slot_mapping[i]] = k[i] (and V); negative slots skipped."""
+    cache = make_cache(k_cache, v_cache)
+    n = slot_mapping.numel()
+    if k.shape != v.shape or k.shape[0] != n or tuple(k.shape[1:]) != tuple(k_cache.shape[2:]):
+        raise ValueError("k, v must be [num_tokens, num_kv_heads, head_dim] matching slot_mapping and the cache")
+    _check(lib.pa_write_kv(_dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+                           _dev(slot_mapping, "slot_mapping", torch.int64), n, ctypes.byref(cache),
+                           _stream_ptr(stream)), "pa_write_kv")
+
+
+def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
+    """cache[dst] = cache[src] for each (src, dst) row of an int64 [P, 2] tensor."""
+    cache = make_cache(k_cache, v_cache)
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs, 2]")
+    p = src_dst_pairs.shape[0]
+    ptr = _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if p else None
+    _check(lib.pa_copy_blocks(ctypes.byref(cache), ptr, p, _stream_ptr(stream)), "pa_copy_blocks")
+
+
+def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, max_seq_len: int, k_cache, v_cache) -> int:
+    cache = make_cache(k_cache, v_cache)
+    return int(lib.pa_decode_workspace_bytes(num_seqs, num_q_heads, max_seq_len, ctypes.byref(cache)))
+
+
+def pa_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
+              max_seq_len: int | None = None, workspace=None, stream=None) -> torch.Tensor:
+    """Decode attention over the paged cache; returns ``out`` ([S, H_q, D] bf16).
+
+    ``max_seq_len`` is a host-side upper bound of ``seq_lens``; when omitted it
+    is read from the device (a synchronisation).  ``workspace`` (uint8 CUDA
+    tensor) is allocated here when omitted and needed."""
+    cache = make_cache(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != k_cache.shape[3]:
+        raise ValueError("q must be [num_seqs, num_q_heads, head_dim]")
+    S, Hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, W] and seq_lens [num_seqs]")
+    if max_seq_len is None:
+        max_seq_len = int(seq_lens.max().item()) if S else 0
+    if out is None:
+        out = torch.empty_like(q)
+    need = int(lib.pa_decode_workspace_bytes(S, Hq, max_seq_len, ctypes.byref(cache)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace", torch.uint8) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib.pa_decode(_dev(q, "q", torch.bfloat16), ctypes.byref(cache),
+                         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                         _dev(seq_lens, "seq_lens", torch.int32), S, int(max_seq_len), Hq,
+                         float(scale), _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes,
+                         _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+def pa_decode_set_partition_tokens(tokens: int) -> int:
+    """0 = automatic split-K partition size; else tokens per partition (multiple of 64)."""
+    return int(lib.pa_decode_set_partition_tokens(int(tokens)))
+
+
+def pa_get_device_error(clear: bool = False) -> int:
+    code = _i32(0)
+    _check(lib.pa_get_device_error(ctypes.byref(code), 1 if clear else 0), "pa_get_device_error")
+    return int(code.value)

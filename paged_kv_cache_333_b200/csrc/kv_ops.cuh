@@ -1,0 +1,104 @@
+// The two data-movement kernels of the path: the slot-mapped KV write and
+// the copy-on-write block copy.  Both are pure HBM traffic: 16-byte vector
+// loads and stores, several in flight per thread, every access bounds-checked
+// against the cache extent.
+#pragma once
+
+#include "pa_device.cuh"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------
+// pa_write_kv: one warp per (token, K|V).  A token's row of num_kv_heads *
+// head_dim bf16 values is contiguous both in k/v and in the cache (the cache
+// row index is the slot), so each warp moves one contiguous row.
+// ("PagedAttention: fragmentation, blocks, block tables", section 3 "The
+// slot mapping": the KV-cache write stores the token at flat row slot.)
+// ---------------------------------------------------------------------------
+constexpr int kWriteThreads = 256;
+
+__global__ void __launch_bounds__(kWriteThreads)
+write_kv_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
+                uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, int64_t num_slots,
+                int row_vecs) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kWriteThreads + threadIdx.x) >> 5;
+    const int64_t tok = warp >> 1;
+    if (tok >= num_tokens)
+        return;
+    const int64_t slot = slot_mapping[tok];
+    if (slot < 0)
+        return;  // padding
+    if (slot >= num_slots) {
+        if (lane == 0 && (warp & 1) == 0)
+            flag_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const uint4 *src = ((warp & 1) ? v : k) + tok * row_vecs;
+    uint4 *dst = ((warp & 1) ? v_cache : k_cache) + slot * row_vecs;
+    // 4 loads in flight per lane before the stores (row_vecs is a multiple of 16).
+    for (int base = 0; base < row_vecs; base += 128) {
+        uint4 r[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * 32 + lane;
+            if (i < row_vecs)
+                r[u] = __ldg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * 32 + lane;
+            if (i < row_vecs)
+                dst[i] = r[u];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// pa_copy_blocks: grid = (num_pairs * 2 tensors * chunks_per_block).  Each CTA
+// copies one chunk of up to kCopyChunkVecs 16-byte vectors of one block of one
+// tensor; 4 vectors in flight per thread.  Pairs with an id outside
+// [0, num_blocks) are skipped and flagged.
+// ("PagedAttention: fragmentation, blocks, block tables", copy-on-write
+// passage: blocks[dst] = blocks[src] over the block-major storage.)
+// ---------------------------------------------------------------------------
+constexpr int kCopyThreads = 256;
+constexpr int kCopyChunkVecs = kCopyThreads * 4;
+
+__global__ void __launch_bounds__(kCopyThreads)
+copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                   const int64_t *__restrict__ pairs, int64_t num_blocks, int64_t block_vecs,
+                   int chunks_per_block) {
+    const int64_t item = blockIdx.x;
+    const int chunk = static_cast<int>(item % chunks_per_block);
+    const int64_t pt = item / chunks_per_block;  // pair * 2 + tensor
+    const int64_t pair = pt >> 1;
+    const int64_t src = pairs[2 * pair];
+    const int64_t dst = pairs[2 * pair + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (threadIdx.x == 0 && chunk == 0 && (pt & 1) == 0)
+            flag_error(PA_DEVERR_COPY_PAIR);
+        return;
+    }
+    uint4 *base = (pt & 1) ? v_cache : k_cache;
+    const uint4 *s = base + src * block_vecs;
+    uint4 *d = base + dst * block_vecs;
+    const int64_t begin = static_cast<int64_t>(chunk) * kCopyChunkVecs;
+    const int64_t end = begin + kCopyChunkVecs < block_vecs ? begin + kCopyChunkVecs : block_vecs;
+    uint4 r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int64_t i = begin + u * kCopyThreads + threadIdx.x;
+        if (i < end)
+            r[u] = __ldcs(s + i);  // read once: streaming
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int64_t i = begin + u * kCopyThreads + threadIdx.x;
+        if (i < end)
+            d[i] = r[u];
+    }
+}
+
+}  // namespace pa

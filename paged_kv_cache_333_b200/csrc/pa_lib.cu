@@ -1,0 +1,350 @@
+// C ABI of the paged-KV decode path (declared in include/pa.h): argument
+// validation, launch configuration, TMA descriptor encoding, device error
+// word.  One translation unit so that the device error word is a single
+// symbol without relocatable device code.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "decode.cuh"
+#include "kv_ops.cuh"
+#include "pa.h"
+#include "pa_device.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+int32_t g_part_tokens_override = 0;
+
+int cuda_fail(cudaError_t e, const char *what) {
+    std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", what, cudaGetErrorString(e));
+    return PA_ECUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cache(const pa_cache_t *c) {
+    if (!c || !c->k_cache || !c->v_cache || c->num_blocks <= 0 || c->num_kv_heads <= 0)
+        return PA_EINVAL;
+    if (c->head_dim != pa::kD)
+        return PA_EUNSUPPORTED;
+    const int32_t b = c->block_size;
+    if (b < 1 || b > 64 || (b & (b - 1)) != 0)
+        return PA_EUNSUPPORTED;
+    // TMA row coordinates are int32.
+    if (c->num_blocks * static_cast<int64_t>(b) > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    if (!aligned16(c->k_cache) || !aligned16(c->v_cache))
+        return PA_EUNSUPPORTED;
+    return PA_OK;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();  // clear a sticky "no device" error from the query
+        return 148;          // B200
+    }
+    return n;
+}
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Tokens per split-K partition.  One partition per sequence when the
+// (sequence, KV head) pairs alone fill every resident CTA slot; otherwise
+// long sequences are cut so that about two CTAs per slot are launched.
+// Always a multiple of 64 (so of the tile and of every block size) and at
+// most kMaxPartBlocks table entries.
+int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
+                           int32_t block_size) {
+    const int64_t cap = static_cast<int64_t>(pa::kMaxPartBlocks) * block_size;
+    int64_t part;
+    if (g_part_tokens_override > 0) {
+        part = g_part_tokens_override;
+    } else {
+        const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
+        const int64_t slots = static_cast<int64_t>(sm_count()) * pa::kDecodeCtasPerSm;
+        const int64_t len = max_seq_len > 0 ? max_seq_len : 1;
+        if (units >= slots)
+            part = len;
+        else
+            part = std::max<int64_t>(256, (len * units + 2 * slots - 1) / (2 * slots));
+    }
+    part = round_up(std::max<int64_t>(part, 64), 64);
+    if (part > cap)
+        part = cap / 64 * 64;
+    return static_cast<int32_t>(part);
+}
+
+struct WorkspaceLayout {
+    int32_t part_tokens, num_parts;
+    size_t ml_bytes, acc_offset, total;
+};
+
+WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t max_seq_len, int32_t block_size) {
+    WorkspaceLayout w{};
+    w.part_tokens = choose_part_tokens(num_seqs, num_kv_heads, max_seq_len, block_size);
+    w.num_parts = max_seq_len > 0 ? static_cast<int32_t>((max_seq_len + w.part_tokens - 1) / w.part_tokens) : 1;
+    if (w.num_parts <= 1) {
+        w.num_parts = 1;
+        return w;
+    }
+    const size_t units = static_cast<size_t>(num_seqs) * num_q_heads * w.num_parts;
+    w.ml_bytes = units * sizeof(float2);
+    w.acc_offset = static_cast<size_t>(round_up(static_cast<int64_t>(w.ml_bytes), 256));
+    w.total = w.acc_offset + units * pa::kD * sizeof(float);
+    return w;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D view of one cache tensor: (dim, kv head, slot) with box
+// (128, 1, min(block_size, 16)).
+int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c) {
+    auto fn = encode_fn();
+    if (!fn) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+        return PA_ECUDA;
+    }
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(c->head_dim),
+                                static_cast<cuuint64_t>(c->num_kv_heads),
+                                static_cast<cuuint64_t>(c->num_blocks) * c->block_size};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(c->head_dim) * 2,
+                                   static_cast<cuuint64_t>(c->num_kv_heads) * c->head_dim * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(c->head_dim), 1u,
+                               static_cast<cuuint32_t>(c->block_size < pa::kTile ? c->block_size : pa::kTile)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
+                      static_cast<int>(r));
+        return PA_ECUDA;
+    }
+    return PA_OK;
+}
+
+template <int G>
+int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
+                    int32_t num_kv_heads, cudaStream_t stream) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(pa::decode_partition_kernel<G>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(pa::kDecodeSmemBytes));
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+        attr_set[dev] = true;
+    }
+    dim3 grid(p.num_parts, num_kv_heads, p.num_seqs);
+    pa::decode_partition_kernel<G><<<grid, pa::kDecodeThreads, pa::kDecodeSmemBytes, stream>>>(tk, tv, p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "decode_partition_kernel launch");
+    if (p.num_parts > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.num_q_heads, p.num_seqs, 1);
+        cfg.blockDim = dim3(pa::kD, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel, p);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "decode_merge_kernel launch");
+    }
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping, int64_t num_tokens,
+                const pa_cache_t *cache, void *stream) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_tokens < 0)
+        return PA_EINVAL;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!k || !v || !slot_mapping)
+        return PA_EINVAL;
+    if (!aligned16(k) || !aligned16(v))
+        return PA_EUNSUPPORTED;
+    const int row_vecs = cache->num_kv_heads * cache->head_dim * 2 / 16;
+    const int64_t warps = num_tokens * 2;
+    const int64_t blocks = (warps * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
+    if (blocks > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    pa::write_kv_kernel<<<static_cast<unsigned>(blocks), pa::kWriteThreads, 0,
+                          static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), slot_mapping, num_tokens,
+        static_cast<uint4 *>(cache->k_cache), static_cast<uint4 *>(cache->v_cache),
+        cache->num_blocks * cache->block_size, row_vecs);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "write_kv_kernel launch");
+}
+
+int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
+                   void *stream) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_pairs < 0)
+        return PA_EINVAL;
+    if (num_pairs == 0)
+        return PA_OK;
+    if (!src_dst_pairs)
+        return PA_EINVAL;
+    const int64_t block_vecs =
+        static_cast<int64_t>(cache->block_size) * cache->num_kv_heads * cache->head_dim * 2 / 16;
+    const int chunks = static_cast<int>((block_vecs + pa::kCopyChunkVecs - 1) / pa::kCopyChunkVecs);
+    const int64_t grid = num_pairs * 2 * chunks;
+    if (grid > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    pa::copy_blocks_kernel<<<static_cast<unsigned>(grid), pa::kCopyThreads, 0,
+                             static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4 *>(cache->k_cache), static_cast<uint4 *>(cache->v_cache), src_dst_pairs,
+        cache->num_blocks, block_vecs, chunks);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_kernel launch");
+}
+
+size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
+                                 const pa_cache_t *cache) {
+    if (check_cache(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
+        return 0;
+    return workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size).total;
+}
+
+int32_t pa_decode_set_partition_tokens(int32_t tokens) {
+    const int32_t prev = g_part_tokens_override;
+    g_part_tokens_override = tokens > 0 ? tokens : 0;
+    return prev;
+}
+
+int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+              int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+              int32_t max_seq_len, int32_t num_q_heads, float scale, void *out, void *workspace,
+              size_t workspace_bytes, void *stream) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_seqs < 0 || max_seq_len < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
+        return PA_EINVAL;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (!q || !block_tables || !seq_lens || !out)
+        return PA_EINVAL;
+    if (num_q_heads % cache->num_kv_heads != 0)
+        return PA_EINVAL;
+    const int32_t G = num_q_heads / cache->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return PA_EUNSUPPORTED;
+    if (!aligned16(q) || !aligned16(out))
+        return PA_EUNSUPPORTED;
+    if (num_seqs > 65535 || cache->num_kv_heads > 65535)
+        return PA_EUNSUPPORTED;
+    if (!std::isfinite(scale))
+        return PA_EINVAL;
+
+    const WorkspaceLayout w =
+        workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size);
+    if (w.total > 0 && (workspace == nullptr || workspace_bytes < w.total))
+        return PA_EWORKSPACE;
+    if (w.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return PA_EUNSUPPORTED;
+
+    CUtensorMap tk, tv;
+    if ((rc = encode_cache_map(&tk, cache->k_cache, cache)) != PA_OK)
+        return rc;
+    if ((rc = encode_cache_map(&tv, cache->v_cache, cache)) != PA_OK)
+        return rc;
+
+    pa::DecodeParams p{};
+    p.q = static_cast<const uint4 *>(q);
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.part_ml = w.total ? static_cast<float2 *>(workspace) : nullptr;
+    p.part_acc = w.total ? reinterpret_cast<float *>(static_cast<char *>(workspace) + w.acc_offset) : nullptr;
+    p.num_blocks = cache->num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.block_size = cache->block_size;
+    p.part_tokens = w.part_tokens;
+    p.num_parts = w.num_parts;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);  // log2(e)
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (G) {
+    case 1: return launch_decode_g<1>(tk, tv, p, cache->num_kv_heads, st);
+    case 2: return launch_decode_g<2>(tk, tv, p, cache->num_kv_heads, st);
+    case 4: return launch_decode_g<4>(tk, tv, p, cache->num_kv_heads, st);
+    default: return launch_decode_g<8>(tk, tv, p, cache->num_kv_heads, st);
+    }
+}
+
+int pa_get_device_error(int32_t *host_code, int clear) {
+    if (!host_code)
+        return PA_EINVAL;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaDeviceSynchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, pa::g_device_error, sizeof v);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "read device error word");
+    *host_code = v;
+    if (clear) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(pa::g_device_error, &zero, sizeof zero);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "clear device error word");
+    }
+    return PA_OK;
+}
+
+const char *pa_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *pa_status_str(int status) {
+    switch (status) {
+    case PA_OK: return "ok";
+    case PA_EINVAL: return "invalid argument";
+    case PA_EUNSUPPORTED: return "unsupported shape, size or alignment";
+    case PA_EWORKSPACE: return "workspace too small";
+    case PA_ECUDA: return "CUDA error";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,171 @@
+"""ctypes binding of libpa_pool.so (include/pa_pool.h): the host block pool."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa_pool.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_333_b200/build.py`")
+lib = ctypes.CDLL(LIB_PATH)
+
+PA_POOL_OK, PA_POOL_EINVAL, PA_POOL_ENOSPACE, PA_POOL_ENOSEQ, PA_POOL_EEXIST, PA_POOL_EINVARIANT, \
+    PA_POOL_ERANGE = 0, -1, -2, -3, -4, -5, -6
+PA_COW_SHARED, PA_COW_INHERITED = 0, 1
+
+EXPORTED = ("pa_pool_create", "pa_pool_destroy", "pa_pool_seq_create", "pa_pool_append", "pa_pool_fork",
+            "pa_pool_release", "pa_pool_num_pending_copies", "pa_pool_take_copies", "pa_pool_num_blocks",
+            "pa_pool_block_size", "pa_pool_num_free", "pa_pool_seq_len", "pa_pool_seq_num_blocks",
+            "pa_pool_refcount", "pa_pool_pins", "pa_pool_free_list", "pa_pool_block_table", "pa_pool_seq_lens",
+            "pa_pool_slots", "pa_pool_step_slots", "pa_pool_check", "pa_pool_status_str")
+
+_P, _i32, _i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+lib.pa_pool_create.argtypes = [_i64, _i32, _P, _i32]
+lib.pa_pool_create.restype = _P
+lib.pa_pool_destroy.argtypes = [_P]
+lib.pa_pool_destroy.restype = None
+for _name, _args, _res in [
+    ("pa_pool_seq_create", [_P, _i64], ctypes.c_int),
+    ("pa_pool_append", [_P, _i64, _i64], ctypes.c_int),
+    ("pa_pool_fork", [_P, _i64, _i64], ctypes.c_int),
+    ("pa_pool_release", [_P, _i64], ctypes.c_int),
+    ("pa_pool_num_pending_copies", [_P], _i64),
+    ("pa_pool_take_copies", [_P, _P, _i64], _i64),
+    ("pa_pool_num_blocks", [_P], _i64),
+    ("pa_pool_block_size", [_P], _i32),
+    ("pa_pool_num_free", [_P], _i64),
+    ("pa_pool_seq_len", [_P, _i64], _i64),
+    ("pa_pool_seq_num_blocks", [_P, _i64], _i64),
+    ("pa_pool_refcount", [_P, _i64], _i32),
+    ("pa_pool_pins", [_P, _i64], _i32),
+    ("pa_pool_free_list", [_P, _P, _i64], _i64),
+    ("pa_pool_block_table", [_P, _P, _i32, _i32, _i32, _P], ctypes.c_int),
+    ("pa_pool_seq_lens", [_P, _P, _i32, _P], ctypes.c_int),
+    ("pa_pool_slots", [_P, _i64, _i64, _i64, _P], ctypes.c_int),
+    ("pa_pool_step_slots", [_P, _P, _i32, _i64, _P], ctypes.c_int),
+    ("pa_pool_check", [_P], ctypes.c_int),
+]:
+    getattr(lib, _name).argtypes = _args
+    getattr(lib, _name).restype = _res
+lib.pa_pool_status_str.argtypes = [ctypes.c_int]
+lib.pa_pool_status_str.restype = ctypes.c_char_p
+
+
+class PoolError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {lib.pa_pool_status_str(code).decode()} ({code})")
+        self.code = code
+
+
+def _ok(rc: int, what: str) -> int:
+    if rc < 0:
+        raise PoolError(int(rc), what)
+    return rc
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class BlockPool:
+    """Host KV block pool.  ``append`` returns False (pool unchanged) when too
+    few blocks are free; every other failure raises PoolError."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None, rule: str = "shared"):
+        rule_id = {"shared": PA_COW_SHARED, "inherited": PA_COW_INHERITED}[rule]
+        if free_order is not None:
+            self._order = np.ascontiguousarray(free_order, dtype=np.int32)
+            if self._order.shape != (num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+            fp = _ptr(self._order)
+        else:
+            fp = None
+        self._h = lib.pa_pool_create(int(num_blocks), int(block_size), fp, rule_id)
+        if not self._h:
+            raise PoolError(PA_POOL_EINVAL, "pa_pool_create")
+        self.num_blocks = int(num_blocks)
+        self.block_size = int(block_size)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h:
+            lib.pa_pool_destroy(h)
+            self._h = None
+
+    # -- operations -------------------------------------------------------
+    def create(self, seq_id: int) -> None:
+        _ok(lib.pa_pool_seq_create(self._h, seq_id), "create")
+
+    def append(self, seq_id: int, n: int) -> bool:
+        rc = lib.pa_pool_append(self._h, seq_id, n)
+        if rc == PA_POOL_ENOSPACE:
+            return False
+        _ok(rc, "append")
+        return True
+
+    def fork(self, src: int, dst: int) -> None:
+        _ok(lib.pa_pool_fork(self._h, src, dst), "fork")
+
+    def release(self, seq_id: int) -> None:
+        _ok(lib.pa_pool_release(self._h, seq_id), "release")
+
+    def take_cow_pairs(self) -> np.ndarray:
+        n = _ok(lib.pa_pool_num_pending_copies(self._h), "num_pending_copies")
+        out = np.zeros((max(n, 1), 2), dtype=np.int64)
+        got = _ok(lib.pa_pool_take_copies(self._h, _ptr(out), n), "take_copies")
+        return out[:got]
+
+    # -- queries ------------------------------------------------------------
+    def num_free(self) -> int:
+        return _ok(lib.pa_pool_num_free(self._h), "num_free")
+
+    def seq_len(self, seq_id: int) -> int:
+        return _ok(lib.pa_pool_seq_len(self._h, seq_id), "seq_len")
+
+    def num_blocks_of(self, seq_id: int) -> int:
+        return _ok(lib.pa_pool_seq_num_blocks(self._h, seq_id), "seq_num_blocks")
+
+    def refcount(self, block: int) -> int:
+        """Owner references (tables naming the block)."""
+        return _ok(lib.pa_pool_refcount(self._h, block), "refcount")
+
+    def pins(self, block: int) -> int:
+        """Queued copies naming the block."""
+        return _ok(lib.pa_pool_pins(self._h, block), "pins")
+
+    def free_list(self) -> list[int]:
+        out = np.zeros(self.num_blocks, dtype=np.int32)
+        n = _ok(lib.pa_pool_free_list(self._h, _ptr(out), self.num_blocks), "free_list")
+        return out[:n].tolist()
+
+    def table(self, seq_id: int) -> list[int]:
+        return self.block_table([seq_id], self.num_blocks_of(seq_id))[0].tolist()
+
+    def block_table(self, seq_ids, width: int, pad: int = -1) -> np.ndarray:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        out = np.empty((len(ids), width), dtype=np.int32)
+        _ok(lib.pa_pool_block_table(self._h, _ptr(ids), len(ids), width, pad, _ptr(out)), "block_table")
+        return out
+
+    def seq_lens(self, seq_ids) -> np.ndarray:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        out = np.empty(len(ids), dtype=np.int32)
+        _ok(lib.pa_pool_seq_lens(self._h, _ptr(ids), len(ids), _ptr(out)), "seq_lens")
+        return out
+
+    def slots(self, seq_id: int, pos0: int, count: int) -> np.ndarray:
+        out = np.empty(count, dtype=np.int64)
+        _ok(lib.pa_pool_slots(self._h, seq_id, pos0, count, _ptr(out)), "slots")
+        return out
+
+    def step_slots(self, seq_ids, tokens_per_seq: int) -> np.ndarray:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        out = np.empty(len(ids) * tokens_per_seq, dtype=np.int64)
+        _ok(lib.pa_pool_step_slots(self._h, _ptr(ids), len(ids), tokens_per_seq, _ptr(out)), "step_slots")
+        return out
+
+    def check(self) -> None:
+        _ok(lib.pa_pool_check(self._h), "check")

@@ -1,0 +1,54 @@
+"""The C-ABI libraries load on a machine without a GPU and export every
+function their headers declare; argument validation runs on the host."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared(header: str) -> set:
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text))
+
+
+@pytest.mark.parametrize("header,lib", [("pa.h", "libpa.so"), ("pa_pool.h", "libpa_pool.so")])
+def test_library_exports_every_declared_function(header, lib):
+    names = _declared(header)
+    assert len(names) >= 8
+    so = ctypes.CDLL(os.path.join(ROOT, "paged_kv_cache_333_b200", lib))
+    missing = [n for n in sorted(names) if not hasattr(so, n)]
+    assert not missing, missing
+
+
+def test_binding_lists_match_headers():
+    from paged_kv_cache_333_b200 import _abi, pool
+    assert set(_abi.EXPORTED) == _declared("pa.h")
+    assert set(pool.EXPORTED) == _declared("pa_pool.h")
+
+
+def test_host_side_validation_without_gpu():
+    """Calls rejected on the host never touch the device."""
+    from paged_kv_cache_333_b200._abi import PA_EINVAL, PA_EUNSUPPORTED, PaCache, lib
+    ok = PaCache(16, 16, 64, 16, 2, 128)  # fake, aligned pointers: never dereferenced
+    assert lib.pa_write_kv(16, 16, 16, -1, ctypes.byref(ok), None) == PA_EINVAL
+    bad_d = PaCache(16, 16, 64, 16, 2, 64)
+    assert lib.pa_write_kv(16, 16, 16, 1, ctypes.byref(bad_d), None) == PA_EUNSUPPORTED
+    bad_b = PaCache(16, 16, 64, 12, 2, 128)
+    assert lib.pa_copy_blocks(ctypes.byref(bad_b), 16, 1, None) == PA_EUNSUPPORTED
+    unaligned = PaCache(18, 16, 64, 16, 2, 128)
+    assert lib.pa_copy_blocks(ctypes.byref(unaligned), 16, 1, None) == PA_EUNSUPPORTED
+    assert lib.pa_decode(16, ctypes.byref(ok), 16, 4, 16, 1, 64, 5, 0.1, 16, None, 0, None) == PA_EINVAL
+    assert lib.pa_decode(16, ctypes.byref(ok), 16, 4, 16, 1, 64, 6, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
+    assert lib.pa_decode(16, ctypes.byref(ok), 16, 4, 16, 1, 64, 32, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
+    # empty work is a successful no-op
+    assert lib.pa_write_kv(None, None, None, 0, ctypes.byref(ok), None) == 0
+    assert lib.pa_copy_blocks(ctypes.byref(ok), None, 0, None) == 0
+    assert lib.pa_decode(None, ctypes.byref(ok), None, 0, None, 0, 0, 4, 0.1, None, None, 0, None) == 0
+    # one partition per sequence -> no workspace; long sequences -> some
+    assert lib.pa_decode_workspace_bytes(64, 32, 0, ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))) == 0
+    assert lib.pa_decode_workspace_bytes(8, 32, 32768, ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))) > 0
+    assert lib.pa_status_str(-3) == b"workspace too small"

@@ -1,0 +1,268 @@
+"""Block pool: the oracle pool pinned to the pages, and the product's C++ pool
+checked against it operation by operation (tables, refcounts, free-list order,
+copy pairs, slots), plus the pages' randomized content test."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from oracle.pool import RULE_INHERITED, RULE_SHARED, RefPool
+from paged_kv_cache_333_b200 import BlockPool
+
+
+def _pools(nb, B, order=None, rule="shared"):
+    return RefPool(nb, B, order, rule), BlockPool(nb, B, order, rule)
+
+
+def _same_state(ref: RefPool, prod: BlockPool):
+    assert ref.free_list() == prod.free_list()
+    for b in range(ref.num_blocks):
+        assert ref.refcount(b) == prod.refcount(b), b
+    for sid in ref.tables:
+        assert ref.table(sid) == prod.table(sid), sid
+        assert ref.seq_len(sid) == prod.seq_len(sid)
+    ref.check()
+    prod.check()
+
+
+# ------------------------------------------------------------ pages' examples
+
+
+@pytest.mark.parametrize("make", [lambda: RefPool(3, 4), lambda: BlockPool(3, 4)])
+def test_pagedkv_trace_without_pin(make, golden):
+    """Capacity 3, B=4: create a, append one token, fork b, append to b: the
+    partial shared tail is copied before b writes; releasing both frees all."""
+    g = golden["pagedkv_trace"]
+    pool = make()
+    pool.create("a" and 1)
+    assert pool.append(1, 1)
+    pool.fork(1, 2)
+    (src,) = pool.table(1)
+    assert pool.refcount(src) == 2
+    assert pool.append(2, 1)  # b's tail is partial and shared -> copy
+    pairs = [tuple(map(int, p)) for p in pool.take_cow_pairs()]
+    assert len(pairs) == 1 and pairs[0][0] == src
+    dst = pairs[0][1]
+    assert pool.table(1) == [src] and pool.table(2) == [dst]
+    assert pool.refcount(src) == 1 and pool.refcount(dst) == 1
+    assert pool.seq_len(1) == len(g["read_a"]) and pool.seq_len(2) == len(g["read_b"])
+    pool.check()
+    pool.release(1)
+    pool.release(2)
+    assert pool.num_free() == g["capacity"] == g["free_after_release_all"]
+    pool.check()
+
+
+@pytest.mark.parametrize("cls", [RefPool, BlockPool])
+def test_one_page_pool_cannot_copy_shared_tail(cls):
+    """A failed allocation leaves both sequences intact."""
+    pool = cls(1, 4)
+    pool.create(1)
+    assert pool.append(1, 1)
+    pool.fork(1, 2)
+    before = (pool.table(1), pool.table(2), pool.seq_len(1), pool.seq_len(2), pool.free_list())
+    assert not pool.append(2, 1)
+    after = (pool.table(1), pool.table(2), pool.seq_len(1), pool.seq_len(2), pool.free_list())
+    assert before == after
+    assert pool.refcount(pool.table(1)[0]) == 2
+    pool.check()
+
+
+@pytest.mark.parametrize("cls", [RefPool, BlockPool])
+def test_tail_waste_and_block_counts(cls, golden):
+    g = golden["tail_waste_b16"]
+    pool = cls(64, g["block_size"])
+    for i, n in enumerate(g["lengths"]):
+        pool.create(i)
+        assert pool.append(i, n)
+        slack = pool.num_blocks_of(i) * g["block_size"] - pool.seq_len(i)
+        assert slack == g["unused_tail_slots"][i]
+    s = golden["simulator_step0"]
+    pool = cls(s["pool_blocks"], s["block_size"])
+    pool.create(0)
+    assert pool.append(0, s["tokens"])
+    assert s["pool_blocks"] - pool.num_free() == s["blocks_used"]
+    assert pool.num_blocks_of(0) * s["block_size"] - s["tokens"] == s["paged_slack"]
+
+
+@pytest.mark.parametrize("cls", [RefPool, BlockPool])
+def test_r7_one_block_appended_and_slot(cls, golden):
+    g = golden["r7_decode_step"]
+    nb = 4096
+    order = list(range(nb))
+    order.remove(g["new_physical_block"])
+    order.insert(g["held_blocks"], g["new_physical_block"])  # 257th block popped is 1913
+    pool = cls(nb, g["block_size"], np.array(order, np.int32))
+    pool.create(7)
+    assert pool.append(7, g["committed_tokens"])
+    assert pool.num_blocks_of(7) == g["held_blocks"]
+    free0 = pool.num_free()
+    assert pool.append(7, g["new_tokens"])
+    assert free0 - pool.num_free() == g["blocks_to_allocate"]
+    assert pool.table(7)[g["logical_block"]] == g["new_physical_block"]
+    assert int(pool.slots(7, g["position"], 1)[0]) == g["slot"]
+
+
+@pytest.mark.parametrize("cls", [RefPool, BlockPool])
+def test_lifo_reuse_and_reverse_free_order(cls):
+    pool = cls(8, 4)
+    pool.create(1)
+    assert pool.append(1, 12)  # blocks 0, 1, 2
+    assert pool.table(1) == [0, 1, 2]
+    pool.release(1)  # freed in reverse: 2, 1, 0 prepended as one run
+    assert pool.free_list()[:3] == [2, 1, 0]
+    pool.create(2)
+    assert pool.append(2, 1)
+    assert pool.table(2) == [2]  # the tail of the released sequence is reused first
+
+
+@pytest.mark.parametrize("rule", [RULE_SHARED, RULE_INHERITED])
+@pytest.mark.parametrize("cls", [RefPool, BlockPool])
+def test_prefix_sharing_refcounts(cls, rule, golden):
+    """2040-token prefix, 256 sequences: 127 full blocks shared by all, the
+    8-token tail copied on first write (255 copies under the refcount rule;
+    256 under the partial-hit rule, whose owner writes in place)."""
+    p = golden["prefix_sharing"]
+    B, n = p["block_size"], 256
+    pool = cls(4096, B, None, rule)
+    pool.create(0)
+    assert pool.append(0, p["prefix_tokens"])
+    for sid in range(1, n):
+        pool.fork(0, sid)
+    prefix_blocks = pool.table(0)
+    assert len(prefix_blocks) == p["shared_full_blocks"] + 1
+    assert all(pool.refcount(b) == n for b in prefix_blocks)
+    tail = prefix_blocks[-1]
+    for sid in range(n):
+        assert pool.append(sid, 1)
+    pairs = pool.take_cow_pairs()
+    copies = n - 1
+    assert len(pairs) == copies
+    assert all(int(s) == tail for s, _ in pairs)
+    assert len({int(d) for _, d in pairs}) == copies
+    for b in prefix_blocks[:-1]:
+        assert pool.refcount(b) == n
+    assert pool.refcount(tail) == 1
+    writer = n - 1 if rule == RULE_SHARED else 0  # who writes in place
+    assert pool.table(writer)[-1] == tail
+    pool.check()
+
+
+# ------------------------------------------------------------ product vs oracle
+
+
+def _replay(op, ref, prod, live, content, store, B):
+    """Apply one random op to both pools and to the content model."""
+    kind = op[0]
+    if kind == "create":
+        sid = op[1]
+        ref.create(sid); prod.create(sid)
+        live.append(sid); content[sid] = []
+    elif kind == "append" and live:
+        sid = live[op[1] % len(live)]
+        n = op[2]
+        ok_r, ok_p = ref.append(sid, n), prod.append(sid, n)
+        assert ok_r == ok_p
+        if ok_r:
+            pr, pp = ref.take_cow_pairs(), prod.take_cow_pairs()
+            assert [tuple(x) for x in pr] == [tuple(map(int, x)) for x in pp]
+            # copies: the whole block, all B slots, sources read first
+            snap = {(s, o): store.get(s * B + o) for s, _ in pr for o in range(B)}
+            for s, d in pr:
+                for o in range(B):
+                    store[d * B + o] = snap[(s, o)]
+            start = len(content[sid])
+            slots = prod.slots(sid, start, n)
+            assert slots.tolist() == ref.slots(sid, start, n).tolist()
+            for i, slot in enumerate(slots):
+                val = (sid, start + i)
+                store[int(slot)] = val
+                content[sid].append(val)
+    elif kind == "fork" and live:
+        src = live[op[1] % len(live)]
+        dst = op[2]
+        ref.fork(src, dst); prod.fork(src, dst)
+        live.append(dst); content[dst] = list(content[src])
+    elif kind == "release" and live:
+        sid = live.pop(op[1] % len(live))
+        ref.release(sid); prod.release(sid)
+        del content[sid]
+
+
+@pytest.mark.parametrize("rule", [RULE_SHARED, RULE_INHERITED])
+@pytest.mark.parametrize("seed", range(25))
+def test_random_ops_match_oracle_and_contents(seed, rule):
+    """25 fixed seeds x 200 create/append/fork/release ops: after every op the
+    two pools agree exactly, the invariants hold, and every sequence's pages
+    decode to its own list of tokens (the randomized test described on page 1,
+    without transfer pins)."""
+    B, nb = 4, 24
+    order = synth.make_rng(1000 + seed).permutation(nb).astype(np.int32)
+    ref, prod = _pools(nb, B, order, rule)
+    live, content, store = [], {}, {}
+    for op in synth.random_pool_ops(seed, 200, max_append=9):
+        _replay(op, ref, prod, live, content, store, B)
+        _same_state(ref, prod)
+        for sid in live:
+            table = prod.table(sid)
+            got = [store.get(table[p // B] * B + p % B) for p in range(len(content[sid]))]
+            assert got == content[sid]
+
+
+@pytest.mark.parametrize("name", ["tiny", "chat", "prefix"])
+def test_workload_layouts_match_oracle(name):
+    w = synth.by_name(name)
+    sh = w.shape
+    ref, prod = _pools(sh.num_blocks, sh.block_size, w.free_order)
+    w.ops(ref); w.ops(prod)
+    if w.suffix_ops:
+        w.suffix_ops(ref); w.suffix_ops(prod)
+    pr, pp = ref.take_cow_pairs(), prod.take_cow_pairs()
+    assert [tuple(x) for x in pr] == [tuple(map(int, x)) for x in pp]
+    width = max(ref.num_blocks_of(s) for s in w.seq_ids)
+    assert np.array_equal(ref.block_table(w.seq_ids, width), prod.block_table(w.seq_ids, width))
+    assert ref.free_list() == prod.free_list()
+    prod.check()
+
+
+@pytest.mark.slow
+def test_sweep_churn_layout_matches_oracle():
+    w = synth.sweep(16)
+    sh = w.shape
+    ref, prod = _pools(sh.num_blocks, sh.block_size, w.free_order)
+    w.ops(ref); w.ops(prod)
+    assert ref.free_list() == prod.free_list()
+    used = sh.num_blocks - prod.num_free()
+    assert used == int(0.9 * sh.num_blocks)
+    width = max(ref.num_blocks_of(s) for s in w.seq_ids)
+    assert np.array_equal(ref.block_table(w.seq_ids, width), prod.block_table(w.seq_ids, width))
+    prod.check()
+
+
+def test_errors_and_state_unchanged():
+    pool = BlockPool(4, 4)
+    pool.create(1)
+    with pytest.raises(Exception):
+        pool.create(1)
+    with pytest.raises(Exception):
+        pool.append(99, 1)
+    assert pool.append(1, 16)
+    assert not pool.append(1, 1)  # full
+    assert pool.seq_len(1) == 16 and pool.num_free() == 0
+    with pytest.raises(Exception):
+        pool.block_table([1], 2)  # 4 blocks do not fit in width 2
+    with pytest.raises(Exception):
+        BlockPool(4, 4, np.array([0, 1, 1, 2], np.int32))  # not a permutation
+    pool.check()
+
+
+def test_step_slots_and_padding():
+    pool = BlockPool(16, 4)
+    for sid, n in [(1, 5), (2, 8)]:
+        pool.create(sid)
+        assert pool.append(sid, n)
+    sl = pool.step_slots([1, 2], 1)
+    assert sl.tolist() == [int(pool.slots(1, 4, 1)[0]), int(pool.slots(2, 7, 1)[0])]
+    bt = pool.block_table([1, 2], 3, pad=-7)
+    assert bt[0, 2] == -7 and bt[1, 2] == -7
+    assert oracle.slot_of(bt[1], 7, 4) == sl[1]
