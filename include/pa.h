@@ -141,6 +141,17 @@ PA_API int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *bloc
               int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
               void *workspace, size_t workspace_bytes, void *stream);
 
+/* Which partition kernel pa_decode runs (process wide; returns the previous
+ * value; other values are ignored).  Both compute the same result within
+ * the stated tolerance.
+ *   PA_DECODE_KERNEL_MMA  (default) QK^T and PV of each 16-token tile on
+ *                         tensor cores (mma.m16n8k16, fp32 accumulate), K/V
+ *                         tiles staged by 128B-swizzled TMA loads;
+ *   PA_DECODE_KERNEL_SIMT QK^T, softmax and PV on CUDA cores with warp
+ *                         shuffles (kept for measurement). */
+enum { PA_DECODE_KERNEL_MMA = 0, PA_DECODE_KERNEL_SIMT = 1 };
+PA_API int32_t pa_decode_set_kernel(int32_t kind);
+
 /* Tokens per split-K partition used by pa_decode: 0 = automatic (the
  * default), otherwise a multiple of 64.  Host-side setting, process wide;
  * returns the previous value.  For tuning and tests. */

@@ -24,8 +24,9 @@ PA_OK, PA_EINVAL, PA_EUNSUPPORTED, PA_EWORKSPACE, PA_ECUDA = 0, -1, -2, -3, -4
 PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
 EXPORTED = ("pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_set_partition_tokens", "pa_get_device_error", "pa_last_cuda_error",
-            "pa_status_str")
+            "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
+            "pa_last_cuda_error", "pa_status_str")
+PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
 
 
 class PaCache(ctypes.Structure):
@@ -45,6 +46,8 @@ lib.pa_decode_workspace_bytes.restype = ctypes.c_size_t
 lib.pa_decode.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
                           _P, _P, ctypes.c_size_t, _P]
 lib.pa_decode.restype = ctypes.c_int
+lib.pa_decode_set_kernel.argtypes = [_i32]
+lib.pa_decode_set_kernel.restype = _i32
 lib.pa_decode_set_partition_tokens.argtypes = [_i32]
 lib.pa_decode_set_partition_tokens.restype = _i32
 lib.pa_get_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
@@ -148,6 +151,12 @@ def pa_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=Non
                          float(scale), _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes,
                          _stream_ptr(stream)), "pa_decode")
     return out
+
+
+def pa_decode_set_kernel(kind: str) -> str:
+    """Select the decode partition kernel: "mma" (default) or "simt"; returns the previous one."""
+    prev = lib.pa_decode_set_kernel({"mma": PA_DECODE_KERNEL_MMA, "simt": PA_DECODE_KERNEL_SIMT}[kind])
+    return "mma" if prev == PA_DECODE_KERNEL_MMA else "simt"
 
 
 def pa_decode_set_partition_tokens(tokens: int) -> int:

@@ -49,9 +49,14 @@ constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxPartBlocks = 1024;  // block-table entries one CTA may cover
 constexpr int kDecodeCtasPerSm = 3;
+// A stage is always consumed by the same warp (tile t: stage t % kStages,
+// warp t % 4), so no parity wait can run a full phase ahead.
+static_assert(kStages % kConsumerWarps == 0, "stages must be a multiple of the consumer warps");
 
 struct DecodeParams {
     const uint4 *q;  // [S][Hq][D] bf16, 8 values per uint4
+    const void *k_cache;  // [NB][B][H_kv][D] bf16 (read directly by the cp.async path)
+    const void *v_cache;
     const int32_t *block_tables;
     const int32_t *seq_lens;
     __nv_bfloat16 *out;  // [S][Hq][D]

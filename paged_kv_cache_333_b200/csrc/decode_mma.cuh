@@ -1,0 +1,392 @@
+// Paged decode attention, tensor-core variant (the default pa_decode path).
+//
+// Same contract and same CTA decomposition as decode.cuh (one CTA per
+// (partition, KV head, sequence); a producer warp streams 16-token K/V tiles
+// into a shared-memory ring; four consumer warps take tiles round-robin; the
+// partition's (max, sum, acc) go to `out` or to the split-K workspace).  What
+// changes is the consumer: with G query heads sharing a KV head, one tile's
+// QK^T is a 16 (tokens) x 8 (heads, G real) x 128 contraction and its PV a
+// 128 x 8 x 16 one, small but dense, so each runs as eight
+// mma.m16n8k16 (bf16 in, fp32 accumulate) instead of ~500 FMAs and a
+// 30-shuffle reduce-scatter per lane.  Measured on B200 the CUDA-core
+// consumer spent most of its time issuing those shuffles and FMAs; this one
+// issues about 100 instructions per tile and leaves the kernel bound by HBM.
+//
+// Tile layout in shared memory: each 16-token tile holds K and V as two
+// 64-dim halves each ([half][token][64] bf16, 2 KiB per half, 1 KiB aligned)
+// in the 128-byte swizzle (16-byte chunk c of row r stored at chunk
+// c ^ (r % 8)), which makes every ldmatrix below conflict-free.  For block
+// sizes >= 8 the producer fills a tile with 3-D TMA loads whose box is
+// (64 dims x 1 head x min(B,16) tokens) using the tensor map's 128B swizzle;
+// for block sizes 1, 2 and 4 (boxes would land at offsets that are not
+// multiples of the swizzle atom) the producer warp gathers the rows with
+// 16-byte cp.async copies at the same swizzled positions and signals the
+// stage's barrier with cp.async.mbarrier.arrive.
+//
+// Per tile and consumer warp:
+//   S^T(16x8) = K(16x128) Q^T(128x8): A = K via ldmatrix.x4, B = q (kept in
+//     registers for the whole kernel, rows >= G zero).  Lane holds scores of
+//     tokens lane/4 and lane/4+8 for heads 2(lane%4), 2(lane%4)+1.
+//   online softmax in the log2 domain (scores * scale*log2 e), per-head max
+//     over the 16 tokens with 3 shuffles; p rounded to bf16 for the PV MMA,
+//     the running sum l kept in fp32.
+//   movmatrix.trans turns the two 8x8 bf16 blocks of P^T into the B operand
+//     of the PV MMA without touching shared memory.
+//   O^T(128x8) += V^T(128x16) P^T(16x8): A = V^T via ldmatrix.x4.trans.
+// Unused storage never reaches a result: scores of slots past the sequence
+// end are set to -inf and, in a partial tile, the V rows of those slots are
+// zeroed in shared memory before the MMA (0 * NaN would be NaN).
+#pragma once
+
+#include "decode.cuh"
+
+namespace pa {
+
+constexpr int kStagesM = 4;
+constexpr int kMmaCtasPerSm = 4;
+constexpr int kHalfElems = kTile * 64;  // one 64-dim half of a 16-token tile
+// Tile t lives in stage t % kStagesM and is consumed by warp t % 4.  With a
+// stage count that is a multiple of the consumer-warp count, a stage is only
+// ever consumed by one warp, which has itself consumed the stage's previous
+// phase before it waits on the next one; a parity wait can then never be a
+// full phase early (a parity test cannot tell phase k+2 from phase k).
+static_assert(kStagesM % kConsumerWarps == 0, "stages must be a multiple of the consumer warps");
+
+struct DecodeSmemM {
+    uint16_t kv[kStagesM][4][kHalfElems];  // [stage][K lo, K hi, V lo, V hi][16 x 64]
+    uint64_t full[kStagesM];
+    uint64_t empty[kStagesM];
+    float wm[kConsumerWarps][8];
+    float wl[kConsumerWarps][8];
+    int32_t blocks[kMaxPartBlocks];
+};
+static_assert(sizeof(float) * kConsumerWarps * 8 * kD <= sizeof(uint16_t) * kStagesM * 4 * kHalfElems,
+              "merge scratch must fit in the KV ring");
+constexpr size_t kDecodeSmemBytesM = sizeof(DecodeSmemM) + 1024;
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a swizzled
+// [rows][64] bf16 half-tile.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int G>
+__global__ void __launch_bounds__(kDecodeThreads, kMmaCtasPerSm)
+decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+    constexpr unsigned FULL = 0xffffffffu;
+    extern __shared__ uint8_t smem_raw[];
+    DecodeSmemM &sm = *reinterpret_cast<DecodeSmemM *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const int part = blockIdx.x;
+    const int h = blockIdx.y;
+    const int s = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int B = p.block_size;
+    const bool use_tma = B >= 8;
+
+    const int n = clamp_seq_len(p, s);
+    const int t_begin = part * p.part_tokens;
+    if (part > 0 && t_begin >= n)
+        return;
+    const int t_end = min(n, t_begin + p.part_tokens);
+    const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStagesM; ++i) {
+            mbar_init(&sm.full[i], use_tma ? 1 : 32);
+            mbar_init(&sm.empty[i], 1);
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    // =================================================================== producer
+    if (warp == kConsumerWarps) {
+        if (num_tiles == 0)
+            return;
+        const int first_blk = t_begin / B;
+        const int nblk = (t_end - 1) / B - first_blk + 1;
+        const int32_t *row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + first_blk;
+        for (int i = lane; i < nblk; i += 32) {
+            int32_t b = __ldg(row + i);
+            if (b < 0 || b >= p.num_blocks) {
+                flag_error(PA_DEVERR_BLOCK_ID);
+                b = 0;
+            }
+            sm.blocks[i] = b;
+        }
+        __syncwarp();
+        if (use_tma && lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+        }
+        const uint64_t pol = l2_evict_first_policy();
+        const int Hkv = gridDim.y;
+        int issued = 0;
+        for (int it = 0; it < num_tiles; ++it) {
+            const int slot = it % kStagesM;
+            if (it >= kStagesM) {
+                bool ok = true;
+                if (lane == 0)
+                    ok = mbar_wait(&sm.empty[slot], ((it / kStagesM) + 1) & 1);
+                if (!__shfl_sync(FULL, ok, 0))
+                    break;
+            }
+            const int t0 = t_begin + it * kTile;
+            const int ntok = min(kTile, t_end - t0);
+            uint16_t(*dst)[kHalfElems] = sm.kv[slot];
+            if (use_tma) {
+                const int rows = B < kTile ? B : kTile;
+                const int nb = B >= kTile ? 1 : (ntok + B - 1) / B;
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&sm.full[slot], static_cast<uint32_t>(nb * rows * 128 * 4));
+                __syncwarp();
+                // lane = (box j, part q): q 0..3 = K lo, K hi, V lo, V hi
+                const int j = lane >> 2, q = lane & 3;
+                if (j < nb) {
+                    const int32_t blk = sm.blocks[(t0 + j * rows) / B - first_blk];
+                    const int32_t r = blk * B + ((t0 + j * rows) % B);
+                    tma_load_3d(&dst[q][j * rows * 64], (q < 2) ? &tm_k : &tm_v, (q & 1) * 64, h, r,
+                                &sm.full[slot], pol);
+                }
+            } else {
+                // cp.async gather: lane = (tensor, 16-byte chunk of the 256-byte row)
+                const int tensor = lane >> 4;  // 0 = K, 1 = V
+                const int ch = lane & 15;      // chunk of the row: half = ch / 8
+                const uint16_t *cache = static_cast<const uint16_t *>(tensor ? p.v_cache : p.k_cache);
+                const uint32_t base = smem_addr(&dst[tensor * 2 + (ch >> 3)][0]);
+                for (int i = 0; i < ntok; ++i) {
+                    const int t = t0 + i;
+                    const int64_t blk = sm.blocks[t / B - first_blk];
+                    const int64_t slot_row = blk * B + (t % B);
+                    const uint16_t *src = cache + (slot_row * Hkv + h) * kD + ch * 8;
+                    cp_async16(base + swz(i, ch & 7), src);
+                }
+                cp_async_mbar_arrive(&sm.full[slot]);
+            }
+            issued = it + 1;
+        }
+        if (lane == 0) {
+            for (int sl = 0; sl < kStagesM && sl < issued; ++sl) {
+                const int last = sl + ((issued - 1 - sl) / kStagesM) * kStagesM;
+                mbar_wait(&sm.full[sl], (last / kStagesM) & 1);
+            }
+        }
+        if (!use_tma)
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        return;
+    }
+
+    // =================================================================== consumers
+    // q as the B operand of S^T = K Q^T: for k-step ks, b0 holds q[n][16ks +
+    // 2(lane%4) + {0,1}] and b1 the same 8 dims later, n = lane/4 (zero if
+    // n >= G).  Kept in registers for the whole kernel.
+    const int qn = lane >> 2;
+    const int qk = (lane & 3) * 2;
+    uint32_t qb[8][2];
+    {
+        const int qh = qn < G ? qn : G - 1;  // rows >= G are zero; never read past q
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(p.q) +
+                               ((static_cast<int64_t>(s) * p.num_q_heads + h * G + qh) * kD) / 2;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            qb[ks][0] = qn < G ? __ldg(qrow + (16 * ks + qk) / 2) : 0u;
+            qb[ks][1] = qn < G ? __ldg(qrow + (16 * ks + 8 + qk) / 2) : 0u;
+        }
+    }
+    const float sl2 = p.scale_log2;
+    float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+    float acc[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+
+    // per-lane ldmatrix row/chunk selectors
+    const int k_row = (lane & 7) + (((lane >> 3) & 1) << 3);  // token row for K (A, non-trans)
+    const int k_chk = lane >> 4;                               // +0 / +1 chunk
+    const int v_row = (lane & 7) + ((lane >> 4) << 3);         // token row for V (A, trans)
+    const int v_chk = (lane >> 3) & 1;
+    const int tok0 = lane >> 2;                                // C-fragment rows: tok0, tok0 + 8
+
+    for (int it = warp; it < num_tiles; it += kConsumerWarps) {
+        const int slot = it % kStagesM;
+        bool ok = true;
+        if (lane == 0)
+            ok = mbar_wait(&sm.full[slot], (it / kStagesM) & 1);
+        if (!__shfl_sync(FULL, ok, 0))
+            break;
+        const int ntok = min(kTile, t_end - (t_begin + it * kTile));
+        const uint32_t kb0 = smem_addr(&sm.kv[slot][0][0]);
+        const uint32_t kb1 = smem_addr(&sm.kv[slot][1][0]);
+        const uint32_t vb0 = smem_addr(&sm.kv[slot][2][0]);
+        const uint32_t vb1 = smem_addr(&sm.kv[slot][3][0]);
+
+        if (ntok < kTile) {
+            // zero the V rows of slots past the end (both halves) before the MMA
+            uint4 *v0 = reinterpret_cast<uint4 *>(&sm.kv[slot][2][0]);
+            uint4 *v1 = reinterpret_cast<uint4 *>(&sm.kv[slot][3][0]);
+            for (int idx = ntok * 8 + lane; idx < kTile * 8; idx += 32) {
+                v0[idx] = make_uint4(0, 0, 0, 0);
+                v1[idx] = make_uint4(0, 0, 0, 0);
+            }
+            __syncwarp();
+        }
+
+        // ---- S^T = K Q^T ------------------------------------------------
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            uint32_t a[4];
+            const uint32_t base = (ks < 4) ? kb0 : kb1;
+            ldmatrix_x4(a, base + swz(k_row, (ks & 3) * 2 + k_chk));
+            mma_16816(sc, a, qb[ks][0], qb[ks][1]);
+        }
+        // ---- online softmax (log2 domain) -------------------------------
+        float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
+        if (ntok < kTile) {
+            if (tok0 >= ntok) x0 = x1 = -INFINITY;
+            if (tok0 + 8 >= ntok) x2 = x3 = -INFINITY;
+        }
+        float tA = fmaxf(x0, x2), tB = fmaxf(x1, x3);
+#pragma unroll
+        for (int off = 4; off <= 16; off <<= 1) {
+            tA = fmaxf(tA, __shfl_xor_sync(FULL, tA, off));
+            tB = fmaxf(tB, __shfl_xor_sync(FULL, tB, off));
+        }
+        const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
+        const float aA = exp2f(mA - nA), aB = exp2f(mB - nB);
+        mA = nA;
+        mB = nB;
+        const float p0 = exp2f(x0 - nA), p1 = exp2f(x1 - nB);
+        const float p2 = exp2f(x2 - nA), p3 = exp2f(x3 - nB);
+        lA = fmaf(lA, aA, p0 + p2);
+        lB = fmaf(lB, aB, p1 + p3);
+        const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));  // tokens 0..7
+        const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));  // tokens 8..15
+        // ---- O^T = alpha O^T + V^T P^T ----------------------------------
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            acc[mt][0] *= aA;
+            acc[mt][1] *= aB;
+            acc[mt][2] *= aA;
+            acc[mt][3] *= aB;
+            uint32_t a[4];
+            const int chunk = 2 * mt + v_chk;  // 16-byte chunk of the 128-dim row
+            ldmatrix_x4_trans(a, ((chunk < 8) ? vb0 : vb1) + swz(v_row, chunk & 7));
+            mma_16816(acc[mt], a, pb0, pb1);
+        }
+        if (ntok < kTile)
+            fence_proxy_async_smem();  // order the zero-fill before the next async refill
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sm.empty[slot]);
+    }
+
+    // ---- warp totals (sum over the 8 lanes sharing lane % 4) ----------------
+#pragma unroll
+    for (int off = 4; off <= 16; off <<= 1) {
+        lA += __shfl_xor_sync(FULL, lA, off);
+        lB += __shfl_xor_sync(FULL, lB, off);
+    }
+    if (threadIdx.x == 0)
+        grid_launch_dependents();
+
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    float *wacc = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [warp][8 heads][D]
+    {
+        const int hA = (lane & 3) * 2;
+        float *wa = wacc + (warp * 8 + hA) * kD;
+        float *wb = wa + kD;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d = mt * 16 + tok0;
+            wa[d] = acc[mt][0];
+            wb[d] = acc[mt][1];
+            wa[d + 8] = acc[mt][2];
+            wb[d + 8] = acc[mt][3];
+        }
+        if (lane < 4) {
+            sm.wm[warp][hA] = mA;
+            sm.wm[warp][hA + 1] = mB;
+            sm.wl[warp][hA] = lA;
+            sm.wl[warp][hA + 1] = lB;
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+
+    const int d = threadIdx.x;  // 0..127
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w)
+            M = fmaxf(M, sm.wm[w][g]);
+        float L = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float mw = sm.wm[w][g];
+                if (mw == -INFINITY)
+                    continue;
+                const float sc = exp2f(mw - M);
+                L = fmaf(sm.wl[w][g], sc, L);
+                o = fmaf(wacc[(w * 8 + g) * kD + d], sc, o);
+            }
+        }
+        const int j = h * G + g;
+        if (p.num_parts == 1) {
+            const float r = L > 0.f ? o / L : 0.f;
+            p.out[(static_cast<int64_t>(s) * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(r);
+        } else {
+            const int64_t idx = (static_cast<int64_t>(s) * p.num_q_heads + j) * p.num_parts + part;
+            p.part_acc[idx * kD + d] = o;
+            if (d == 0)
+                p.part_ml[idx] = make_float2(M, L);
+        }
+    }
+}
+
+}  // namespace pa

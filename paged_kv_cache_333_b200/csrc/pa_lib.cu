@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "decode.cuh"
+#include "decode_mma.cuh"
 #include "kv_ops.cuh"
 #include "pa.h"
 #include "pa_device.cuh"
@@ -21,6 +22,11 @@ namespace {
 
 thread_local char g_last_cuda_error[256] = "";
 int32_t g_part_tokens_override = 0;
+int32_t g_decode_kernel = PA_DECODE_KERNEL_MMA;
+
+int ctas_per_sm() {
+    return g_decode_kernel == PA_DECODE_KERNEL_MMA ? pa::kMmaCtasPerSm : pa::kDecodeCtasPerSm;
+}
 
 int cuda_fail(cudaError_t e, const char *what) {
     std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", what, cudaGetErrorString(e));
@@ -58,8 +64,9 @@ int sm_count() {
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // Tokens per split-K partition.  One partition per sequence when the
-// (sequence, KV head) pairs alone fill every resident CTA slot; otherwise
-// long sequences are cut so that about two CTAs per slot are launched.
+// (sequence, KV head) pairs alone fill at least 3/4 of the resident CTA
+// slots (one wave, no merge); otherwise long sequences are cut so that about
+// two CTAs per slot are launched.
 // Always a multiple of 64 (so of the tile and of every block size) and at
 // most kMaxPartBlocks table entries.
 int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
@@ -70,9 +77,9 @@ int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_s
         part = g_part_tokens_override;
     } else {
         const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
-        const int64_t slots = static_cast<int64_t>(sm_count()) * pa::kDecodeCtasPerSm;
+        const int64_t slots = static_cast<int64_t>(sm_count()) * ctas_per_sm();
         const int64_t len = max_seq_len > 0 ? max_seq_len : 1;
-        if (units >= slots)
+        if (4 * units >= 3 * slots)
             part = len;
         else
             part = std::max<int64_t>(256, (len * units + 2 * slots - 1) / (2 * slots));
@@ -117,9 +124,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D view of one cache tensor: (dim, kv head, slot) with box
-// (128, 1, min(block_size, 16)).
-int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c) {
+// 3-D view of one cache tensor: (dim, kv head, slot).  CUDA-core kernel:
+// box (128, 1, min(B, 16)), no swizzle.  Tensor-core kernel: box (64, 1,
+// min(B, 16)) with the 128-byte swizzle, loaded as two 64-dim halves.
+int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c, bool swizzled) {
     auto fn = encode_fn();
     if (!fn) {
         std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
@@ -130,11 +138,12 @@ int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c) {
                                 static_cast<cuuint64_t>(c->num_blocks) * c->block_size};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(c->head_dim) * 2,
                                    static_cast<cuuint64_t>(c->num_kv_heads) * c->head_dim * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(c->head_dim), 1u,
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(swizzled ? 64 : c->head_dim), 1u,
                                static_cast<cuuint32_t>(c->block_size < pa::kTile ? c->block_size : pa::kTile)};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled failed (%d)",
@@ -144,22 +153,45 @@ int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c) {
     return PA_OK;
 }
 
+// Opt a kernel into its dynamic shared memory and the all-shared carveout
+// (so that its CTAs-per-SM target fits), once per device.
+template <typename K>
+int prepare_kernel(K kernel, size_t smem, bool (&done)[64]) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && done[dev])
+        return PA_OK;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute(max dynamic smem)");
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    if (dev >= 0 && dev < 64)
+        done[dev] = true;
+    return PA_OK;
+}
+
 template <int G>
 int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
                     int32_t num_kv_heads, cudaStream_t stream) {
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(pa::decode_partition_kernel<G>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(pa::kDecodeSmemBytes));
-        if (e != cudaSuccess)
-            return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-        attr_set[dev] = true;
-    }
     dim3 grid(p.num_parts, num_kv_heads, p.num_seqs);
-    pa::decode_partition_kernel<G><<<grid, pa::kDecodeThreads, pa::kDecodeSmemBytes, stream>>>(tk, tv, p);
+    if (g_decode_kernel == PA_DECODE_KERNEL_MMA) {
+        static bool done[64] = {};
+        int rc = prepare_kernel(pa::decode_partition_mma_kernel<G>, pa::kDecodeSmemBytesM, done);
+        if (rc)
+            return rc;
+        pa::decode_partition_mma_kernel<G>
+            <<<grid, pa::kDecodeThreads, pa::kDecodeSmemBytesM, stream>>>(tk, tv, p);
+    } else {
+        static bool done[64] = {};
+        int rc = prepare_kernel(pa::decode_partition_kernel<G>, pa::kDecodeSmemBytes, done);
+        if (rc)
+            return rc;
+        pa::decode_partition_kernel<G><<<grid, pa::kDecodeThreads, pa::kDecodeSmemBytes, stream>>>(tk, tv, p);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return cuda_fail(e, "decode_partition_kernel launch");
@@ -244,6 +276,13 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
     return workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size).total;
 }
 
+int32_t pa_decode_set_kernel(int32_t kind) {
+    const int32_t prev = g_decode_kernel;
+    if (kind == PA_DECODE_KERNEL_MMA || kind == PA_DECODE_KERNEL_SIMT)
+        g_decode_kernel = kind;
+    return prev;
+}
+
 int32_t pa_decode_set_partition_tokens(int32_t tokens) {
     const int32_t prev = g_part_tokens_override;
     g_part_tokens_override = tokens > 0 ? tokens : 0;
@@ -282,14 +321,17 @@ int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_table
     if (w.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return PA_EUNSUPPORTED;
 
+    const bool swizzled = g_decode_kernel == PA_DECODE_KERNEL_MMA;
     CUtensorMap tk, tv;
-    if ((rc = encode_cache_map(&tk, cache->k_cache, cache)) != PA_OK)
+    if ((rc = encode_cache_map(&tk, cache->k_cache, cache, swizzled)) != PA_OK)
         return rc;
-    if ((rc = encode_cache_map(&tv, cache->v_cache, cache)) != PA_OK)
+    if ((rc = encode_cache_map(&tv, cache->v_cache, cache, swizzled)) != PA_OK)
         return rc;
 
     pa::DecodeParams p{};
     p.q = static_cast<const uint4 *>(q);
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
     p.block_tables = block_tables;
     p.seq_lens = seq_lens;
     p.out = static_cast<__nv_bfloat16 *>(out);

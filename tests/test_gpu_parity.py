@@ -27,6 +27,15 @@ def pa():
     m.pa_get_device_error(clear=True)
     yield m
     m.pa_decode_set_partition_tokens(0)
+    m.pa_decode_set_kernel("mma")
+
+
+@pytest.fixture(params=["mma", "simt"])
+def kernel(request, pa):
+    """Run the test with each decode partition kernel."""
+    prev = pa.pa_decode_set_kernel(request.param)
+    yield request.param
+    pa.pa_decode_set_kernel(prev)
 
 
 def _bits(t):
@@ -52,6 +61,19 @@ CONFIGS = ["tiny", "chat", "long", "prefix", "sweep_b1", "sweep_b16", "sweep_b32
 
 @pytest.mark.parametrize("name", CONFIGS)
 def test_config_parity(pa, name):
+    _config_parity(pa, name)
+
+
+@pytest.mark.parametrize("name", ["tiny", "chat", "sweep_b1"])
+def test_config_parity_simt_kernel(pa, name):
+    prev = pa.pa_decode_set_kernel("simt")
+    try:
+        _config_parity(pa, name)
+    finally:
+        pa.pa_decode_set_kernel(prev)
+
+
+def _config_parity(pa, name):
     """Full-size workloads: layouts identical, caches bit-exact after the
     history writes, the copy-on-write copies and the step's write, decode
     within tolerance for every (sequence, head)."""
@@ -131,16 +153,16 @@ EDGE_LENS = [0, 1, 2, 15, 16, 17, 31, 33, 63, 64, 65, 127, 129, 300, 1000]
 
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("B", [1, 2, 4, 8, 16, 32, 64])
-def test_group_and_block_sizes(pa, G, B):
+def test_group_and_block_sizes(pa, kernel, G, B):
     Hkv = 2
     q, kc, vc, bt, lens = _random_case(100 + 10 * G + B, EDGE_LENS, B, G * Hkv, Hkv)
     ref = oracle.decode(q, kc, vc, bt, lens, 0.08838834764831845)
-    _close(_run_case(pa, q, kc, vc, bt, lens), ref, f"G={G} B={B}")
+    _close(_run_case(pa, q, kc, vc, bt, lens), ref, f"{kernel} G={G} B={B}")
     assert pa.pa_get_device_error(clear=True) == 0
 
 
 @pytest.mark.parametrize("part", [64, 128, 192, 256, 512, 1024, 4096])
-def test_split_k_partitions_and_merge(pa, part):
+def test_split_k_partitions_and_merge(pa, kernel, part):
     lens = [1, 64, 65, 200, 777, 2049, 4100]
     q, kc, vc, bt, lens_np = _random_case(7, lens, 16, 32, 8)
     ref = oracle.decode(q, kc, vc, bt, lens_np, 0.08838834764831845)
@@ -163,7 +185,7 @@ def test_max_seq_len_upper_bound_is_only_a_bound(pa):
         _close(_run_case(pa, q, kc, vc, bt_wide, lens_np, max_len=m), ref, f"max_seq_len={m}")
 
 
-def test_single_token_returns_v0_bit_exact(pa):
+def test_single_token_returns_v0_bit_exact(pa, kernel):
     q, kc, vc, bt, lens = _random_case(9, [1, 1, 1], 16, 8, 2)
     out = _bits(_run_case(pa, q, kc, vc, bt, lens))
     for s in range(3):
@@ -172,7 +194,7 @@ def test_single_token_returns_v0_bit_exact(pa):
             assert np.array_equal(out[s, j], vc[blk, 0, j // 4])
 
 
-def test_physical_placement_does_not_change_a_bit(pa):
+def test_physical_placement_does_not_change_a_bit(pa, kernel):
     """Same logical K/V, four different placements: identical output bits."""
     lens = [3, 16, 40, 500, 1500]
     outs = []
