@@ -157,6 +157,33 @@ PA_API int32_t pa_decode_set_kernel(int32_t kind);
  * returns the previous value.  For tuning and tests. */
 PA_API int32_t pa_decode_set_partition_tokens(int32_t tokens);
 
+/*
+ * pa_decode_static_ws -- pa_decode without a caller-supplied workspace.
+ * The pages have no counterpart for this call: it exists for callers that
+ * cannot allocate device memory, such as a plugin whose host application
+ * owns every device allocation and hands it no allocator, or a serving loop
+ * that must not call cudaMalloc on its hot path (it can synchronize the
+ * device and stall other work).  Same arguments and result as pa_decode,
+ * minus workspace and workspace_bytes.
+ *   Scratch: a fixed array of PA_DECODE_STATIC_WS_BYTES (8 MiB) in this
+ *   library's device memory, present on every device that loads the library
+ *   until the process exits.  A shape whose pa_decode_workspace_bytes() is
+ *   larger returns PA_EWORKSPACE (message in pa_last_cuda_error) and enqueues
+ *   nothing.  The call allocates nothing.
+ *   Set-up: the first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current and caches it; make that
+ *   first call before any stream capture.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents (nothing in it needs to start at zero).  Calls that may
+ *   overlap on the GPU (other streams, other host threads) race on it:
+ *   serialise them, or use pa_decode with separate workspaces.
+ */
+#define PA_DECODE_STATIC_WS_BYTES (8u * 1024u * 1024u)
+PA_API int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                               int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                               int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
+                               void *stream);
+
 /* Read (and with clear != 0, reset) the device error word of the current
  * device.  Synchronises the device.  Returns PA_OK or PA_ECUDA. */
 PA_API int pa_get_device_error(int32_t *host_code, int clear);

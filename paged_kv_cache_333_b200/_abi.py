@@ -24,7 +24,7 @@ PA_OK, PA_EINVAL, PA_EUNSUPPORTED, PA_EWORKSPACE, PA_ECUDA = 0, -1, -2, -3, -4
 PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
 EXPORTED = ("pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
+            "pa_decode_static_ws", "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
 
@@ -46,6 +46,10 @@ lib.pa_decode_workspace_bytes.restype = ctypes.c_size_t
 lib.pa_decode.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
                           _P, _P, ctypes.c_size_t, _P]
 lib.pa_decode.restype = ctypes.c_int
+lib.pa_decode_static_ws.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
+                                    _P, _P]
+lib.pa_decode_static_ws.restype = ctypes.c_int
+PA_DECODE_STATIC_WS_BYTES = 8 * 1024 * 1024
 lib.pa_decode_set_kernel.argtypes = [_i32]
 lib.pa_decode_set_kernel.restype = _i32
 lib.pa_decode_set_partition_tokens.argtypes = [_i32]
@@ -150,6 +154,30 @@ def pa_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=Non
                          _dev(seq_lens, "seq_lens", torch.int32), S, int(max_seq_len), Hq,
                          float(scale), _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes,
                          _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+def pa_decode_static_ws(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=None,
+                        max_seq_len: int | None = None, stream=None) -> torch.Tensor:
+    """pa_decode for callers that cannot allocate device memory: the split-K
+    scratch lives in the library's fixed device array (8 MiB per device), so
+    no workspace is passed or allocated (``out`` is still the caller's).
+    Calls that overlap on the GPU share that array and must be serialised."""
+    cache = make_cache(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != k_cache.shape[3]:
+        raise ValueError("q must be [num_seqs, num_q_heads, head_dim]")
+    S, Hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, W] and seq_lens [num_seqs]")
+    if max_seq_len is None:
+        max_seq_len = int(seq_lens.max().item()) if S else 0
+    if out is None:
+        raise ValueError("out must be given: this call allocates nothing")
+    _check(lib.pa_decode_static_ws(_dev(q, "q", torch.bfloat16), ctypes.byref(cache),
+                                   _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                                   _dev(seq_lens, "seq_lens", torch.int32), S, int(max_seq_len), Hq,
+                                   float(scale), _dev(out, "out", torch.bfloat16), _stream_ptr(stream)),
+           "pa_decode_static_ws")
     return out
 
 

@@ -376,6 +376,61 @@ int pa_get_device_error(int32_t *host_code, int clear) {
     return PA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// pa_decode_static_ws: pa_decode with its split-K scratch in a fixed device
+// array owned by this library, for callers that cannot allocate device
+// memory (see include/pa.h).  The array is a file-scope __device__ object: one
+// copy per device that loads the library, kept until the process exits.  In
+// host code its name only stands in for the object; the device address comes
+// from cudaGetSymbolAddress, looked up once per device (on the first call made
+// with that device current) and cached.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_decode_static_scratch[PA_DECODE_STATIC_WS_BYTES];
+
+namespace {
+std::mutex g_static_scratch_mu;
+void *g_static_scratch_ptr[64] = {};
+}  // namespace
+
+int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                        int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                        int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
+                        void *stream) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_seqs > 0 && num_q_heads > 0 && max_seq_len >= 0) {
+        const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, max_seq_len, cache);
+        if (need > PA_DECODE_STATIC_WS_BYTES) {
+            std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,
+                          "pa_decode_static_ws: this shape needs %zu bytes of scratch, the static "
+                          "array holds %zu",
+                          need, static_cast<size_t>(PA_DECODE_STATIC_WS_BYTES));
+            return PA_EWORKSPACE;
+        }
+    }
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= 64)
+        return PA_EUNSUPPORTED;
+    void *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+        if (!g_static_scratch_ptr[dev]) {
+            e = cudaGetSymbolAddress(&g_static_scratch_ptr[dev], g_decode_static_scratch);
+            if (e != cudaSuccess) {
+                g_static_scratch_ptr[dev] = nullptr;
+                return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
+            }
+        }
+        scratch = g_static_scratch_ptr[dev];
+    }
+    return pa_decode(q, cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, max_seq_len,
+                     num_q_heads, scale, out, scratch, PA_DECODE_STATIC_WS_BYTES, stream);
+}
+
 const char *pa_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char *pa_status_str(int status) {
