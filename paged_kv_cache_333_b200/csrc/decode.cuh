@@ -250,6 +250,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    grid_dependency_wait();  // the preceding kernel's writes are visible after this
     const int n = clamp_seq_len(p, s);
     const int t_begin = part * p.part_tokens;
     if (part > 0 && t_begin >= n)
@@ -467,6 +468,7 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
 // One CTA per (query head, sequence); thread d owns output dim d.
 __global__ void __launch_bounds__(kD) decode_merge_kernel(const DecodeParams p) {
     grid_dependency_wait();  // partials of the partition kernel are visible after this
+    grid_launch_dependents();
     const int j = blockIdx.x;
     const int s = blockIdx.y;
     const int d = threadIdx.x;

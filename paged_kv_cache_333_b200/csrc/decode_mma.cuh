@@ -2,7 +2,7 @@
 //
 // Same contract and same CTA decomposition as decode.cuh (one CTA per
 // (partition, KV head, sequence); a producer warp streams 16-token K/V tiles
-// into a shared-memory ring; four consumer warps take tiles round-robin; the
+// into a shared-memory ring; consumer warps take tiles round-robin; the
 // partition's (max, sum, acc) go to `out` or to the split-K workspace).  What
 // changes is the consumer: with G query heads sharing a KV head, one tile's
 // QK^T is a 16 (tokens) x 8 (heads, G real) x 128 contraction and its PV a
@@ -33,6 +33,11 @@
 //   movmatrix.trans turns the two 8x8 bf16 blocks of P^T into the B operand
 //     of the PV MMA without touching shared memory.
 //   O^T(128x8) += V^T(128x16) P^T(16x8): A = V^T via ldmatrix.x4.trans.
+// A consumer warp reads the whole tile into registers (K and V^T fragments)
+// and releases the stage before any arithmetic; the CTA has two consumer
+// warps and a six-stage ring, so each warp always has loads in flight for
+// its next two tiles while it computes (up to 4 CTAs, ~190 KiB of loads in
+// flight, per SM).
 // Unused storage never reaches a result: scores of slots past the sequence
 // end are set to -inf and, in a partial tile, the V rows of those slots are
 // zeroed in shared memory before the MMA (0 * NaN would be NaN).
@@ -42,25 +47,30 @@
 
 namespace pa {
 
-constexpr int kStagesM = 4;
+constexpr int kConsumerWarpsM = 2;
+constexpr int kDecodeThreadsM = (kConsumerWarpsM + 1) * 32;
+constexpr int kStagesM = 6;
 constexpr int kMmaCtasPerSm = 4;
+constexpr int kMaxPartBlocksM = 512;    // block-table entries one CTA may cover
 constexpr int kHalfElems = kTile * 64;  // one 64-dim half of a 16-token tile
-// Tile t lives in stage t % kStagesM and is consumed by warp t % 4.  With a
-// stage count that is a multiple of the consumer-warp count, a stage is only
-// ever consumed by one warp, which has itself consumed the stage's previous
-// phase before it waits on the next one; a parity wait can then never be a
-// full phase early (a parity test cannot tell phase k+2 from phase k).
-static_assert(kStagesM % kConsumerWarps == 0, "stages must be a multiple of the consumer warps");
+// Tile t lives in stage t % kStagesM and is consumed by warp t % kConsumerWarpsM.
+// With a stage count that is a multiple of the consumer-warp count, a stage
+// is only ever consumed by one warp, which has itself consumed the stage's
+// previous phase before it waits on the next one; a parity wait can then
+// never be a full phase early (a parity test cannot tell phase k+2 from k).
+// Each consumer warp owns kStagesM / kConsumerWarpsM stages, so loads keep
+// streaming into its other stages while it computes on one.
+static_assert(kStagesM % kConsumerWarpsM == 0, "stages must be a multiple of the consumer warps");
 
 struct DecodeSmemM {
     uint16_t kv[kStagesM][4][kHalfElems];  // [stage][K lo, K hi, V lo, V hi][16 x 64]
     uint64_t full[kStagesM];
     uint64_t empty[kStagesM];
-    float wm[kConsumerWarps][8];
-    float wl[kConsumerWarps][8];
-    int32_t blocks[kMaxPartBlocks];
+    float wm[kConsumerWarpsM][8];
+    float wl[kConsumerWarpsM][8];
+    int32_t blocks[kMaxPartBlocksM];
 };
-static_assert(sizeof(float) * kConsumerWarps * 8 * kD <= sizeof(uint16_t) * kStagesM * 4 * kHalfElems,
+static_assert(sizeof(float) * kConsumerWarpsM * 8 * kD <= sizeof(uint16_t) * kStagesM * 4 * kHalfElems,
               "merge scratch must fit in the KV ring");
 constexpr size_t kDecodeSmemBytesM = sizeof(DecodeSmemM) + 1024;
 
@@ -110,7 +120,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
 }
 
 template <int G>
-__global__ void __launch_bounds__(kDecodeThreads, kMmaCtasPerSm)
+__global__ void __launch_bounds__(kDecodeThreadsM, kMmaCtasPerSm)
 decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
@@ -127,13 +137,8 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int B = p.block_size;
     const bool use_tma = B >= 8;
 
-    const int n = clamp_seq_len(p, s);
-    const int t_begin = part * p.part_tokens;
-    if (part > 0 && t_begin >= n)
-        return;
-    const int t_end = min(n, t_begin + p.part_tokens);
-    const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
-
+    // Set-up that touches no global memory runs before the wait on the
+    // preceding kernel of the stream (programmatic dependent launch).
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesM; ++i) {
             mbar_init(&sm.full[i], use_tma ? 1 : 32);
@@ -141,17 +146,35 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         mbar_init_fence();
     }
+    if (use_tma && warp == kConsumerWarpsM && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    grid_dependency_wait();
+
+    // The producer reads the first 32 table entries of its slice while every
+    // thread reads the sequence length (two loads in flight, not one after
+    // the other).  Entries past the row's end are never read.
+    const int t_begin = part * p.part_tokens;
+    const int first_blk = t_begin / B;
+    const int32_t *row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + first_blk;
+    int32_t first_ids = 0;
+    if (warp == kConsumerWarpsM && lane < p.max_blocks_per_seq - first_blk)
+        first_ids = __ldg(row + lane);
+    const int n = clamp_seq_len(p, s);
+    if (part > 0 && t_begin >= n)
+        return;
+    const int t_end = min(n, t_begin + p.part_tokens);
+    const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
     __syncthreads();
 
     // =================================================================== producer
-    if (warp == kConsumerWarps) {
+    if (warp == kConsumerWarpsM) {
         if (num_tiles == 0)
             return;
-        const int first_blk = t_begin / B;
         const int nblk = (t_end - 1) / B - first_blk + 1;
-        const int32_t *row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + first_blk;
         for (int i = lane; i < nblk; i += 32) {
-            int32_t b = __ldg(row + i);
+            int32_t b = i < 32 ? first_ids : __ldg(row + i);
             if (b < 0 || b >= p.num_blocks) {
                 flag_error(PA_DEVERR_BLOCK_ID);
                 b = 0;
@@ -159,10 +182,6 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             sm.blocks[i] = b;
         }
         __syncwarp();
-        if (use_tma && lane == 0) {
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-        }
         const uint64_t pol = l2_evict_first_policy();
         const int Hkv = gridDim.y;
         int issued = 0;
@@ -251,7 +270,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int v_chk = (lane >> 3) & 1;
     const int tok0 = lane >> 2;                                // C-fragment rows: tok0, tok0 + 8
 
-    for (int it = warp; it < num_tiles; it += kConsumerWarps) {
+    for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
         const int slot = it % kStagesM;
         bool ok = true;
         if (lane == 0)
@@ -265,7 +284,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         const uint32_t vb1 = smem_addr(&sm.kv[slot][3][0]);
 
         if (ntok < kTile) {
-            // zero the V rows of slots past the end (both halves) before the MMA
+            // zero the V rows of slots past the end (both halves) before reading them
             uint4 *v0 = reinterpret_cast<uint4 *>(&sm.kv[slot][2][0]);
             uint4 *v1 = reinterpret_cast<uint4 *>(&sm.kv[slot][3][0]);
             for (int idx = ntok * 8 + lane; idx < kTile * 8; idx += 32) {
@@ -274,16 +293,29 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             __syncwarp();
         }
+        // Pull the whole tile into registers (K as the QK A operand, V^T as
+        // the PV A operand) and hand the stage back to the producer before
+        // any arithmetic, so the next load into it starts as early as possible.
+        uint32_t ka[8][4], va[8][4];
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+            ldmatrix_x4(ka[ks], ((ks < 4) ? kb0 : kb1) + swz(k_row, (ks & 3) * 2 + k_chk));
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int chunk = 2 * mt + v_chk;  // 16-byte chunk of the 128-dim row
+            ldmatrix_x4_trans(va[mt], ((chunk < 8) ? vb0 : vb1) + swz(v_row, chunk & 7));
+        }
+        if (ntok < kTile)
+            fence_proxy_async_smem();  // order the zero-fill before the next async refill
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&sm.empty[slot]);
 
         // ---- S^T = K Q^T ------------------------------------------------
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            uint32_t a[4];
-            const uint32_t base = (ks < 4) ? kb0 : kb1;
-            ldmatrix_x4(a, base + swz(k_row, (ks & 3) * 2 + k_chk));
-            mma_16816(sc, a, qb[ks][0], qb[ks][1]);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+            mma_16816(sc, ka[ks], qb[ks][0], qb[ks][1]);
         // ---- online softmax (log2 domain) -------------------------------
         float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
         if (ntok < kTile) {
@@ -313,16 +345,8 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             acc[mt][1] *= aB;
             acc[mt][2] *= aA;
             acc[mt][3] *= aB;
-            uint32_t a[4];
-            const int chunk = 2 * mt + v_chk;  // 16-byte chunk of the 128-dim row
-            ldmatrix_x4_trans(a, ((chunk < 8) ? vb0 : vb1) + swz(v_row, chunk & 7));
-            mma_16816(acc[mt], a, pb0, pb1);
+            mma_16816(acc[mt], va[mt], pb0, pb1);
         }
-        if (ntok < kTile)
-            fence_proxy_async_smem();  // order the zero-fill before the next async refill
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.empty[slot]);
     }
 
     // ---- warp totals (sum over the 8 lanes sharing lane % 4) ----------------
@@ -334,7 +358,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (threadIdx.x == 0)
         grid_launch_dependents();
 
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
     float *wacc = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [warp][8 heads][D]
     {
         const int hA = (lane & 3) * 2;
@@ -355,36 +379,42 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             sm.wl[warp][hA + 1] = lB;
         }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
 
-    const int d = threadIdx.x;  // 0..127
+    // thread t finishes dims t and t + 64 of every real head
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarps; ++w)
+        for (int w = 0; w < kConsumerWarpsM; ++w)
             M = fmaxf(M, sm.wm[w][g]);
-        float L = 0.f, o = 0.f;
+        float L = 0.f, o[2] = {0.f, 0.f};
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
+            for (int w = 0; w < kConsumerWarpsM; ++w) {
                 const float mw = sm.wm[w][g];
                 if (mw == -INFINITY)
                     continue;
                 const float sc = exp2f(mw - M);
                 L = fmaf(sm.wl[w][g], sc, L);
-                o = fmaf(wacc[(w * 8 + g) * kD + d], sc, o);
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+                    o[u] = fmaf(wacc[(w * 8 + g) * kD + threadIdx.x + 64 * u], sc, o[u]);
             }
         }
         const int j = h * G + g;
-        if (p.num_parts == 1) {
-            const float r = L > 0.f ? o / L : 0.f;
-            p.out[(static_cast<int64_t>(s) * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(r);
-        } else {
-            const int64_t idx = (static_cast<int64_t>(s) * p.num_q_heads + j) * p.num_parts + part;
-            p.part_acc[idx * kD + d] = o;
-            if (d == 0)
-                p.part_ml[idx] = make_float2(M, L);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int d = threadIdx.x + 64 * u;
+            if (p.num_parts == 1) {
+                const float r = L > 0.f ? o[u] / L : 0.f;
+                p.out[(static_cast<int64_t>(s) * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(r);
+            } else {
+                const int64_t idx = (static_cast<int64_t>(s) * p.num_q_heads + j) * p.num_parts + part;
+                p.part_acc[idx * kD + d] = o[u];
+                if (d == 0)
+                    p.part_ml[idx] = make_float2(M, L);
+            }
         }
     }
 }

@@ -22,6 +22,10 @@ write_kv_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                 const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
                 uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, int64_t num_slots,
                 int row_vecs) {
+    // Programmatic dependent launch: let the next kernel's CTAs get resident
+    // now; touch global memory only once the preceding kernel is complete.
+    grid_launch_dependents();
+    grid_dependency_wait();
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kWriteThreads + threadIdx.x) >> 5;
     const int64_t tok = warp >> 1;
@@ -70,6 +74,8 @@ __global__ void __launch_bounds__(kCopyThreads)
 copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                    const int64_t *__restrict__ pairs, int64_t num_blocks, int64_t block_vecs,
                    int chunks_per_block) {
+    grid_launch_dependents();
+    grid_dependency_wait();
     const int64_t item = blockIdx.x;
     const int chunk = static_cast<int>(item % chunks_per_block);
     const int64_t pt = item / chunks_per_block;  // pair * 2 + tensor

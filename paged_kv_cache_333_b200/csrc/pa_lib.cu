@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "decode.cuh"
 #include "decode_mma.cuh"
@@ -66,12 +67,16 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 // Tokens per split-K partition.  One partition per sequence when the
 // (sequence, KV head) pairs alone fill at least 3/4 of the resident CTA
 // slots (one wave, no merge); otherwise long sequences are cut so that about
-// two CTAs per slot are launched.
+// six CTAs per slot are launched (measured on B200 with 8 x {32K, 8K}: 640
+// tokens per partition, 83% of the HBM copy bandwidth, against 70% with two
+// CTAs per slot; more, shorter partitions pay for their merge and set-up).
 // Always a multiple of 64 (so of the tile and of every block size) and at
 // most kMaxPartBlocks table entries.
 int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
                            int32_t block_size) {
-    const int64_t cap = static_cast<int64_t>(pa::kMaxPartBlocks) * block_size;
+    const int64_t max_blocks =
+        g_decode_kernel == PA_DECODE_KERNEL_MMA ? pa::kMaxPartBlocksM : pa::kMaxPartBlocks;
+    const int64_t cap = max_blocks * block_size;
     int64_t part;
     if (g_part_tokens_override > 0) {
         part = g_part_tokens_override;
@@ -82,7 +87,7 @@ int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_s
         if (4 * units >= 3 * slots)
             part = len;
         else
-            part = std::max<int64_t>(256, (len * units + 2 * slots - 1) / (2 * slots));
+            part = std::max<int64_t>(256, (len * units + 6 * slots - 1) / (6 * slots));
     }
     part = round_up(std::max<int64_t>(part, 64), 64);
     if (part > cap)
@@ -153,6 +158,27 @@ int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c, bool swiz
     return PA_OK;
 }
 
+// Every kernel of the library is launched with programmatic stream
+// serialization: its CTAs may become resident while the preceding kernel of
+// the stream is finishing, and each kernel waits for that kernel (to complete
+// and flush) before it reads or writes global memory (griddepcontrol.wait),
+// so stream order is kept.  What overlaps is launch latency and set-up.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Opt a kernel into its dynamic shared memory and the all-shared carveout
 // (so that its CTAs-per-SM target fits), once per device.
 template <typename K>
@@ -183,30 +209,23 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
         int rc = prepare_kernel(pa::decode_partition_mma_kernel<G>, pa::kDecodeSmemBytesM, done);
         if (rc)
             return rc;
-        pa::decode_partition_mma_kernel<G>
-            <<<grid, pa::kDecodeThreads, pa::kDecodeSmemBytesM, stream>>>(tk, tv, p);
+        cudaError_t e = launch_pdl(pa::decode_partition_mma_kernel<G>, grid, dim3(pa::kDecodeThreadsM),
+                                   pa::kDecodeSmemBytesM, stream, tk, tv, p);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "decode_partition_mma_kernel launch");
     } else {
         static bool done[64] = {};
         int rc = prepare_kernel(pa::decode_partition_kernel<G>, pa::kDecodeSmemBytes, done);
         if (rc)
             return rc;
-        pa::decode_partition_kernel<G><<<grid, pa::kDecodeThreads, pa::kDecodeSmemBytes, stream>>>(tk, tv, p);
+        cudaError_t e = launch_pdl(pa::decode_partition_kernel<G>, grid, dim3(pa::kDecodeThreads),
+                                   pa::kDecodeSmemBytes, stream, tk, tv, p);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "decode_partition_kernel launch");
     }
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess)
-        return cuda_fail(e, "decode_partition_kernel launch");
     if (p.num_parts > 1) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(p.num_q_heads, p.num_seqs, 1);
-        cfg.blockDim = dim3(pa::kD, 1, 1);
-        cfg.dynamicSmemBytes = 0;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, pa::decode_merge_kernel, p);
+        cudaError_t e = launch_pdl(pa::decode_merge_kernel, dim3(p.num_q_heads, p.num_seqs, 1), dim3(pa::kD),
+                                   0, stream, p);
         if (e != cudaSuccess)
             return cuda_fail(e, "decode_merge_kernel launch");
     }
@@ -235,12 +254,11 @@ int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping, int64
     const int64_t blocks = (warps * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
     if (blocks > INT32_MAX)
         return PA_EUNSUPPORTED;
-    pa::write_kv_kernel<<<static_cast<unsigned>(blocks), pa::kWriteThreads, 0,
-                          static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), slot_mapping, num_tokens,
-        static_cast<uint4 *>(cache->k_cache), static_cast<uint4 *>(cache->v_cache),
-        cache->num_blocks * cache->block_size, row_vecs);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(pa::write_kv_kernel, dim3(static_cast<unsigned>(blocks)), dim3(pa::kWriteThreads),
+                               0, static_cast<cudaStream_t>(stream), static_cast<const uint4 *>(k),
+                               static_cast<const uint4 *>(v), slot_mapping, num_tokens,
+                               static_cast<uint4 *>(cache->k_cache), static_cast<uint4 *>(cache->v_cache),
+                               cache->num_blocks * cache->block_size, row_vecs);
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "write_kv_kernel launch");
 }
 
@@ -261,11 +279,10 @@ int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_
     const int64_t grid = num_pairs * 2 * chunks;
     if (grid > INT32_MAX)
         return PA_EUNSUPPORTED;
-    pa::copy_blocks_kernel<<<static_cast<unsigned>(grid), pa::kCopyThreads, 0,
-                             static_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4 *>(cache->k_cache), static_cast<uint4 *>(cache->v_cache), src_dst_pairs,
-        cache->num_blocks, block_vecs, chunks);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(pa::copy_blocks_kernel, dim3(static_cast<unsigned>(grid)), dim3(pa::kCopyThreads),
+                               0, static_cast<cudaStream_t>(stream), static_cast<uint4 *>(cache->k_cache),
+                               static_cast<uint4 *>(cache->v_cache), src_dst_pairs, cache->num_blocks,
+                               block_vecs, chunks);
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_kernel launch");
 }
 
