@@ -51,6 +51,12 @@ WORKLOAD_TEXT = {
     "prefix": "Prefix sharing + CoW: 256 seqs, 2040-token shared prefix, suffix U[1,256], "
               "32 q / 8 KV heads, d=128, block 16",
     "tiny": "Tiny: 4 seqs {2,18,34,101}, 8 q / 2 KV heads, d=128, block 16, 64-block pool",
+    "sweep_b1": "Block-size sweep, B=1: 128 seqs, geometric lengths (mean 1000, cap 8192), pool of "
+                "428,560 blocks at 90% occupancy after 10k seeded alloc/free events",
+    "sweep_b16": "Block-size sweep, B=16: 128 seqs, geometric lengths (mean 1000, cap 8192), pool of "
+                 "26,785 blocks at 90% occupancy after 10k seeded alloc/free events",
+    "sweep_b32": "Block-size sweep, B=32: 128 seqs, geometric lengths (mean 1000, cap 8192), pool of "
+                 "13,392 blocks at 90% occupancy after 10k seeded alloc/free events",
 }
 
 

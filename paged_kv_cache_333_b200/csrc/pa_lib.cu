@@ -64,14 +64,16 @@ int sm_count() {
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
-// Tokens per split-K partition.  One partition per sequence when the
-// (sequence, KV head) pairs alone fill at least 3/4 of the resident CTA
-// slots (one wave, no merge); otherwise long sequences are cut so that about
-// six CTAs per slot are launched (measured on B200 with 8 x {32K, 8K}: 640
-// tokens per partition, 83% of the HBM copy bandwidth, against 70% with two
-// CTAs per slot; more, shorter partitions pay for their merge and set-up).
-// Always a multiple of 64 (so of the tile and of every block size) and at
-// most kMaxPartBlocks table entries.
+// Tokens per split-K partition.  One CTA streams its partition at roughly
+// 0.7 us per 16-token tile on B200 (a few tiles in flight per CTA), so the
+// longest partition bounds the kernel's duration whatever the batch looks
+// like: the host only knows max_seq_len, not how lengths are spread.  The
+// partition is therefore kept near 640 tokens (one partition for chat-length
+// sequences; 8 x {32K, 8K} measured at 83% of the HBM copy bandwidth with
+// 640 against 70% with 1792), and grows only when even that would launch
+// more than ~16 CTAs per resident slot for max-length sequences (bounding
+// the merge work and the workspace).  A multiple of 64 (so of the tile and
+// of every block size), and at most the per-CTA table capacity.
 int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
                            int32_t block_size) {
     const int64_t max_blocks =
@@ -84,10 +86,9 @@ int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_s
         const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
         const int64_t slots = static_cast<int64_t>(sm_count()) * ctas_per_sm();
         const int64_t len = max_seq_len > 0 ? max_seq_len : 1;
-        if (4 * units >= 3 * slots)
-            part = len;
-        else
-            part = std::max<int64_t>(256, (len * units + 6 * slots - 1) / (6 * slots));
+        part = std::max<int64_t>(640, (len * units + 16 * slots - 1) / (16 * slots));
+        if (part >= len)
+            part = len;  // a single partition: no merge
     }
     part = round_up(std::max<int64_t>(part, 64), 64);
     if (part > cap)
