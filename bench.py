@@ -144,6 +144,34 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# --------------------------------------------------------------------------- ncu traffic
+def profiled_traffic(config: str):
+    """DRAM bytes (read + write) per decode launch from the committed ncu
+    capture, if that capture was of this workload and of the kernel sources
+    as they are now; otherwise None."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "decode_mma_chat_full.md")
+    try:
+        text = open(prof).read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        line = line.strip()
+        if ":" in line and line.split(":")[0] in ("kernel_sources_sha256_16", "workload", "traffic_bytes_per_launch"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("workload") != config or "traffic_bytes_per_launch" not in fields:
+        return None
+    csrc = os.path.join(ROOT, "paged_kv_cache_333_b200", "csrc")
+    for item in fields.get("kernel_sources_sha256_16", "").split():
+        name, digest = item.split("=")
+        with open(os.path.join(csrc, name), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
+                return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 # --------------------------------------------------------------------------- bytes
 def algorithmic_bytes(st) -> dict:
     """Bytes the step must move, per layer."""
@@ -336,7 +364,8 @@ def run_ours(args, world, rank, local):
         "decode_tokens_per_s_per_layer": round(world * S / (ms_step / L * 1e-3), 1),
         "per_op_bytes_per_layer": nbytes,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(args.config) if not args.part_tokens else None,
                      "kernel": "pa_decode (partition kernel" + (" + LSE merge)" if split else ")"),
                      "mean_launch_us": round(dec_mean_ms * 1e3, 3),
                      "how": f"CUDA graph of {L} back-to-back pa_decode calls (one per layer cache), "
