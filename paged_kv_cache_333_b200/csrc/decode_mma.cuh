@@ -19,9 +19,9 @@
 // sizes >= 8 the producer fills a tile with 3-D TMA loads whose box is
 // (64 dims x 1 head x min(B,16) tokens) using the tensor map's 128B swizzle;
 // for block sizes 1, 2 and 4 (boxes would land at offsets that are not
-// multiples of the swizzle atom) the producer warp gathers the rows with
-// 16-byte cp.async copies at the same swizzled positions and signals the
-// stage's barrier with cp.async.mbarrier.arrive.
+// multiples of the swizzle atom) each consumer warp gathers its own tiles'
+// rows with 16-byte cp.async copies at the same swizzled positions, three
+// tiles ahead of the one it computes on.
 //
 // Per tile and consumer warp:
 //   S^T(16x8) = K(16x128) Q^T(128x8): A = K via ldmatrix.x4, B = q (kept in
@@ -106,10 +106,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
-                 : "memory");
-}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -141,7 +137,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     // preceding kernel of the stream (programmatic dependent launch).
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesM; ++i) {
-            mbar_init(&sm.full[i], use_tma ? 1 : 32);
+            mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 1);
         }
         mbar_init_fence();
@@ -166,12 +162,10 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         return;
     const int t_end = min(n, t_begin + p.part_tokens);
     const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
-    __syncthreads();
-
-    // =================================================================== producer
-    if (warp == kConsumerWarpsM) {
-        if (num_tiles == 0)
-            return;
+    const int Hkv = gridDim.y;
+    // The producer warp copies the partition's slice of the block table into
+    // shared memory (read once, bounds-checked) before the CTA barrier.
+    if (warp == kConsumerWarpsM && num_tiles > 0) {
         const int nblk = (t_end - 1) / B - first_blk + 1;
         for (int i = lane; i < nblk; i += 32) {
             int32_t b = i < 32 ? first_ids : __ldg(row + i);
@@ -181,9 +175,14 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             sm.blocks[i] = b;
         }
-        __syncwarp();
+    }
+    __syncthreads();
+
+    // =================================================================== producer
+    if (warp == kConsumerWarpsM) {
+        if (num_tiles == 0 || !use_tma)
+            return;  // with blocks < 8 tokens each consumer warp gathers its own tiles
         const uint64_t pol = l2_evict_first_policy();
-        const int Hkv = gridDim.y;
         int issued = 0;
         for (int it = 0; it < num_tiles; ++it) {
             const int slot = it % kStagesM;
@@ -197,7 +196,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             const int t0 = t_begin + it * kTile;
             const int ntok = min(kTile, t_end - t0);
             uint16_t(*dst)[kHalfElems] = sm.kv[slot];
-            if (use_tma) {
+            {
                 const int rows = B < kTile ? B : kTile;
                 const int nb = B >= kTile ? 1 : (ntok + B - 1) / B;
                 if (lane == 0)
@@ -211,20 +210,6 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                     tma_load_3d(&dst[q][j * rows * 64], (q < 2) ? &tm_k : &tm_v, (q & 1) * 64, h, r,
                                 &sm.full[slot], pol);
                 }
-            } else {
-                // cp.async gather: lane = (tensor, 16-byte chunk of the 256-byte row)
-                const int tensor = lane >> 4;  // 0 = K, 1 = V
-                const int ch = lane & 15;      // chunk of the row: half = ch / 8
-                const uint16_t *cache = static_cast<const uint16_t *>(tensor ? p.v_cache : p.k_cache);
-                const uint32_t base = smem_addr(&dst[tensor * 2 + (ch >> 3)][0]);
-                for (int i = 0; i < ntok; ++i) {
-                    const int t = t0 + i;
-                    const int64_t blk = sm.blocks[t / B - first_blk];
-                    const int64_t slot_row = blk * B + (t % B);
-                    const uint16_t *src = cache + (slot_row * Hkv + h) * kD + ch * 8;
-                    cp_async16(base + swz(i, ch & 7), src);
-                }
-                cp_async_mbar_arrive(&sm.full[slot]);
             }
             issued = it + 1;
         }
@@ -234,8 +219,6 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                 mbar_wait(&sm.full[sl], (last / kStagesM) & 1);
             }
         }
-        if (!use_tma)
-            asm volatile("cp.async.wait_all;" ::: "memory");
         return;
     }
 
@@ -270,21 +253,15 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int v_chk = (lane >> 3) & 1;
     const int tok0 = lane >> 2;                                // C-fragment rows: tok0, tok0 + 8
 
-    for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
-        const int slot = it % kStagesM;
-        bool ok = true;
-        if (lane == 0)
-            ok = mbar_wait(&sm.full[slot], (it / kStagesM) & 1);
-        if (!__shfl_sync(FULL, ok, 0))
-            break;
-        const int ntok = min(kTile, t_end - (t_begin + it * kTile));
+    // One tile: zero the V rows past the end (partial tile), pull K and V^T
+    // fragments into registers, run `loaded()` (hand the stage back), then
+    // QK^T, the online softmax and PV.
+    auto consume = [&](int slot, int ntok, auto &&loaded) {
         const uint32_t kb0 = smem_addr(&sm.kv[slot][0][0]);
         const uint32_t kb1 = smem_addr(&sm.kv[slot][1][0]);
         const uint32_t vb0 = smem_addr(&sm.kv[slot][2][0]);
         const uint32_t vb1 = smem_addr(&sm.kv[slot][3][0]);
-
         if (ntok < kTile) {
-            // zero the V rows of slots past the end (both halves) before reading them
             uint4 *v0 = reinterpret_cast<uint4 *>(&sm.kv[slot][2][0]);
             uint4 *v1 = reinterpret_cast<uint4 *>(&sm.kv[slot][3][0]);
             for (int idx = ntok * 8 + lane; idx < kTile * 8; idx += 32) {
@@ -293,9 +270,6 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             __syncwarp();
         }
-        // Pull the whole tile into registers (K as the QK A operand, V^T as
-        // the PV A operand) and hand the stage back to the producer before
-        // any arithmetic, so the next load into it starts as early as possible.
         uint32_t ka[8][4], va[8][4];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
@@ -305,11 +279,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             const int chunk = 2 * mt + v_chk;  // 16-byte chunk of the 128-dim row
             ldmatrix_x4_trans(va[mt], ((chunk < 8) ? vb0 : vb1) + swz(v_row, chunk & 7));
         }
-        if (ntok < kTile)
-            fence_proxy_async_smem();  // order the zero-fill before the next async refill
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(&sm.empty[slot]);
+        loaded();
 
         // ---- S^T = K Q^T ------------------------------------------------
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -347,6 +317,68 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             acc[mt][3] *= aB;
             mma_16816(acc[mt], va[mt], pb0, pb1);
         }
+    };
+    auto tile_tokens = [&](int it) { return min(kTile, t_end - (t_begin + it * kTile)); };
+
+    if (use_tma) {
+        // Fed by the producer warp: wait for the stage, release it as soon as
+        // the fragments are in registers.
+        for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
+            const int slot = it % kStagesM;
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait(&sm.full[slot], (it / kStagesM) & 1);
+            if (!__shfl_sync(FULL, ok, 0))
+                break;
+            const int ntok = tile_tokens(it);
+            consume(slot, ntok, [&] {
+                if (ntok < kTile)
+                    fence_proxy_async_smem();  // order the zero-fill before the next async refill
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.empty[slot]);
+            });
+        }
+    } else {
+        // Blocks of 1, 2 or 4 tokens: every row of a tile may live in another
+        // block, so each consumer warp gathers its own tiles with 16-byte
+        // cp.async copies, kAhead tiles ahead, into the stages it owns (tile t
+        // in stage t % kStagesM, always this warp's).  Lane i < 16 computes the
+        // cache row of token i once; the row is broadcast by shuffle to the
+        // lanes that copy its 16 chunks (lanes 0-15 K, 16-31 V).
+        constexpr int kAhead = kStagesM / kConsumerWarpsM;
+        const int tensor = lane >> 4;
+        const int ch = lane & 15;
+        const uint16_t *cache = static_cast<const uint16_t *>(tensor ? p.v_cache : p.k_cache);
+        auto gather = [&](int it) {
+            if (it < num_tiles) {
+                const int slot = it % kStagesM;
+                const int t0 = t_begin + it * kTile;
+                const int ntok = tile_tokens(it);
+                int64_t my_row = 0;
+                if (lane < ntok) {
+                    const int t = t0 + lane;
+                    my_row = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + h;
+                }
+                const uint32_t base = smem_addr(&sm.kv[slot][tensor * 2 + (ch >> 3)][0]);
+                for (int i = 0; i < ntok; ++i) {
+                    const int64_t r = __shfl_sync(FULL, my_row, i);
+                    cp_async16(base + swz(i, ch & 7), cache + r * kD + ch * 8);
+                }
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k)
+            gather(warp + k * kConsumerWarpsM);
+        for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
+            asm volatile("cp.async.wait_group %0;" ::"n"(kAhead - 1) : "memory");
+            __syncwarp();
+            consume(it % kStagesM, tile_tokens(it), [] {});
+            __syncwarp();  // every lane is done with this stage before it is refilled
+            gather(it + kAhead * kConsumerWarpsM);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
 
     // ---- warp totals (sum over the 8 lanes sharing lane % 4) ----------------
