@@ -82,6 +82,22 @@ def dist_env():
     return world, rank, local
 
 
+def reduce_max(value: float, device) -> float:
+    """Max of a per-rank number over all ranks (identity without a process
+    group).  Device times of the replicas are combined this way."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, bytes_per_replica: float, seconds: float) -> float:
+    """GB/s of the whole job: every replica moves bytes_per_replica in the
+    (max over ranks) time."""
+    return world * bytes_per_replica / seconds / 1e9
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -252,12 +268,7 @@ def run_ours(args, world, rank, local):
         t1.record()
         torch.cuda.synchronize()
         barrier()
-        ms = t0.elapsed_time(t1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return reduce_max(t0.elapsed_time(t1), dev)
 
     # eager warm-up (kernel attributes, tensor maps), then graphs
     for l in range(L):
@@ -279,7 +290,7 @@ def run_ours(args, world, rank, local):
         g_dec.replay()
     dec_ms_total = timed(g_dec, K)
     ms_step = ms_total / K
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = whole_job_rate(world, step_bytes, ms_step * 1e-3)
     dec_mean_ms = dec_ms_total / (K * L)
     peak, peak_src = measured_peak()
     achieved = nbytes["decode_kv"] / (dec_mean_ms * 1e-3) / 1e9
@@ -325,7 +336,7 @@ def run_ours(args, world, rank, local):
         h2d = (sm_h.numel() * 8 + bt_h.numel() * 4 + sl_h.numel() * 4 + (pairs_h.numel() * 8 if has_pairs else 0)
                + L * (q_h.numel() + k_h.numel() + v_h.numel()) * 2)
         d2h = L * out_h.numel() * 2
-        e2e = {"value": round(world * step_bytes / (e_ms / K * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e2e = {"value": round(whole_job_rate(world, step_bytes, e_ms / K * 1e-3), 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": round(e_ms / K, 4),
                "how": "CUDA graph of the step with its pinned-host copies: per layer q, k, v in and out back"}

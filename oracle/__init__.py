@@ -55,8 +55,13 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB_PATH)
+        # ORACLE_LIB lets the mutation tests load a copy of the oracle with a
+        # planted mistake; nothing else sets it.
+        path = os.environ.get("ORACLE_LIB")
+        if not path:
+            build()
+            path = _LIB_PATH
+        lib = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i64, i32 = ctypes.c_int64, ctypes.c_int32
         lib.oracle_write_kv.argtypes = [P, P, P, i64, i64, i64, P, P]
