@@ -71,6 +71,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-op", action="store_true")
     ap.add_argument("--part-tokens", type=int, default=0, help="split-K partition size (0 = automatic)")
     return ap.parse_args()
 
@@ -295,6 +296,41 @@ def run_ours(args, world, rank, local):
     peak, peak_src = measured_peak()
     achieved = nbytes["decode_kv"] / (dec_mean_ms * 1e-3) / 1e9
 
+    # ---- per-op times (graphs of one launch per layer) -------------------------
+    per_op = {}
+    if not args.no_per_op:
+        row = st.num_kv_heads * st.head_dim * 2
+        T = st.slot_mapping.numel()
+        pos = st.seq_lens.to(torch.int64) - 1  # decode step: the new token is the last
+        req = torch.arange(len(st.ids), dtype=torch.int32, device=dev)
+        used = st.block_tables_np[st.block_tables_np >= 0]
+        free = np.array(st.pool.free_list(), dtype=np.int64)
+        P = int(min(255, len(np.unique(used)), len(free)))  # a prefix-sharing CoW burst: 255 pairs
+        pairs = torch.from_numpy(np.stack([np.unique(used)[:P].astype(np.int64), free[:P]], 1).copy()).to(dev)
+        blk_bytes = st.block_size * row
+
+        def time_ops(fn, launches):
+            g = capture(fn)
+            g.replay()
+            torch.cuda.synchronize()
+            return timed(g, K) / (K * launches) * 1e3  # us per launch
+
+        us = time_ops(lambda: [pa.pa_write_kv(st.k_new, st.v_new, st.slot_mapping, *st.caches[l])
+                               for l in range(L)], L)
+        per_op["write_kv"] = {"us": round(us, 3), "GB/s": round(T * row * 4 / us / 1e3, 2)}
+        us = time_ops(lambda: [pa.pa_write_kv_positions(st.k_new, st.v_new, pos, req, st.block_tables,
+                                                        *st.caches[l]) for l in range(L)], L)
+        per_op["write_kv_positions"] = {"us": round(us, 3), "GB/s": round(T * row * 4 / us / 1e3, 2)}
+        if P:
+            us = time_ops(lambda: [pa.pa_copy_blocks(*st.caches[l], pairs) for l in range(L)], L)
+            per_op["copy_blocks"] = {"pairs": P, "us": round(us, 3),
+                                     "GB/s": round(P * blk_bytes * 4 / us / 1e3, 2)}
+            us = time_ops(lambda: pa.pa_copy_blocks_layers(st.caches, pairs), 1)
+            per_op["copy_blocks_layers"] = {"pairs": P, "layers": L, "us": round(us, 3),
+                                            "GB/s": round(L * P * blk_bytes * 4 / us / 1e3, 2)}
+        per_op["decode"] = {"us": round(dec_mean_ms * 1e3, 3), "GB/s": round(achieved, 2)}
+        assert pa.pa_get_device_error(clear=True) == 0
+
     # ---- end to end: the same step from pinned host buffers -------------------
     e2e = None
     if not args.no_e2e:
@@ -374,6 +410,7 @@ def run_ours(args, world, rank, local):
                         "nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2)},
         "decode_tokens_per_s_per_layer": round(world * S / (ms_step / L * 1e-3), 1),
         "per_op_bytes_per_layer": nbytes,
+        "per_op": per_op,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(args.config) if not args.part_tokens else None,

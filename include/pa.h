@@ -90,6 +90,37 @@ PA_API int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping
                 const pa_cache_t *cache, void *stream);
 
 /*
+ * pa_compute_slot_mapping -- the slot mapping of a step, on the device.
+ * Defined by: "PagedAttention: fragmentation, blocks, block tables",
+ * section 3 "The slot mapping" (recomputed every step from the block table
+ * and the scheduled tokens' positions: slot = block_table[req][pos / B] * B
+ * + pos % B; tokens that are not written get a PAD value).
+ *   positions     [num_tokens] int64: position of each token in its sequence;
+ *                 a negative position is padding.
+ *   req_indices   [num_tokens] int32: row of block_tables of each token.
+ *   block_tables  [num_reqs][max_blocks_per_seq] int32.
+ *   slot_mapping  [num_tokens] int64 output; padding -> -1.  A token whose
+ *                 request, table entry or block id is out of range also gets
+ *                 -1 and sets PA_DEVERR_SLOT.
+ */
+PA_API int pa_compute_slot_mapping(const int64_t *positions, const int32_t *req_indices, int64_t num_tokens,
+                                   const int32_t *block_tables, int32_t max_blocks_per_seq, int32_t num_reqs,
+                                   int32_t block_size, int64_t num_blocks, int64_t *slot_mapping, void *stream);
+
+/*
+ * pa_write_kv_positions -- pa_write_kv with the slot computed in the kernel
+ * from the token's request row and position (same passage as above), so a
+ * step needs no host-built slot mapping.  Arguments as pa_write_kv and
+ * pa_compute_slot_mapping; cache->block_size and cache->num_blocks give B and
+ * the block-id range.  Out-of-range tokens are skipped and set
+ * PA_DEVERR_SLOT; negative positions are padding.
+ */
+PA_API int pa_write_kv_positions(const void *k, const void *v, const int64_t *positions,
+                                 const int32_t *req_indices, int64_t num_tokens, const int32_t *block_tables,
+                                 int32_t max_blocks_per_seq, int32_t num_reqs, const pa_cache_t *cache,
+                                 void *stream);
+
+/*
  * pa_copy_blocks -- copy-on-write block copies.
  * Defined by: "PagedAttention: fragmentation, blocks, block tables",
  * copy-on-write passage (a list of (src_block_id, dst_block_id) pairs runs
@@ -102,6 +133,18 @@ PA_API int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping
  */
 PA_API int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
                    void *stream);
+
+/*
+ * pa_copy_blocks_layers -- pa_copy_blocks for every layer of a model in one
+ * launch.  Same passage as pa_copy_blocks ("not a per-layer loop": there the
+ * layers alias one storage; here each layer has its own K and V tensors and
+ * one grid covers them all).
+ *   caches      HOST array of num_layers descriptors (<= 128), all with the
+ *               same num_blocks, block_size, num_kv_heads and head_dim.
+ *   src_dst_pairs, num_pairs: as pa_copy_blocks, applied to every layer.
+ */
+PA_API int pa_copy_blocks_layers(const pa_cache_t *caches, int32_t num_layers, const int64_t *src_dst_pairs,
+                                 int64_t num_pairs, void *stream);
 
 /*
  * Bytes of scratch pa_decode needs for this batch shape (0 when no sequence

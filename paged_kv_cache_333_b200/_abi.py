@@ -23,7 +23,8 @@ lib = ctypes.CDLL(LIB_PATH)
 PA_OK, PA_EINVAL, PA_EUNSUPPORTED, PA_EWORKSPACE, PA_ECUDA = 0, -1, -2, -3, -4
 PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
-EXPORTED = ("pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_bytes", "pa_decode",
+EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
+            "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
             "pa_decode_static_ws", "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
@@ -39,7 +40,13 @@ _P = ctypes.c_void_p
 _i32, _i64 = ctypes.c_int32, ctypes.c_int64
 lib.pa_write_kv.argtypes = [_P, _P, _P, _i64, ctypes.POINTER(PaCache), _P]
 lib.pa_write_kv.restype = ctypes.c_int
+lib.pa_compute_slot_mapping.argtypes = [_P, _P, _i64, _P, _i32, _i32, _i32, _i64, _P, _P]
+lib.pa_compute_slot_mapping.restype = ctypes.c_int
+lib.pa_write_kv_positions.argtypes = [_P, _P, _P, _P, _i64, _P, _i32, _i32, ctypes.POINTER(PaCache), _P]
+lib.pa_write_kv_positions.restype = ctypes.c_int
 lib.pa_copy_blocks.argtypes = [ctypes.POINTER(PaCache), _P, _i64, _P]
+lib.pa_copy_blocks_layers.argtypes = [ctypes.POINTER(PaCache), _i32, _P, _i64, _P]
+lib.pa_copy_blocks_layers.restype = ctypes.c_int
 lib.pa_copy_blocks.restype = ctypes.c_int
 lib.pa_decode_workspace_bytes.argtypes = [_i32, _i32, _i32, ctypes.POINTER(PaCache)]
 lib.pa_decode_workspace_bytes.restype = ctypes.c_size_t
@@ -112,6 +119,41 @@ def pa_write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:
                            _stream_ptr(stream)), "pa_write_kv")
 
 
+def pa_compute_slot_mapping(positions, req_indices, block_tables, block_size: int, num_blocks: int,
+                            slot_mapping=None, stream=None):
+    """slot_mapping[i] = block_tables[req[i]][pos[i] // B] * B + pos[i] % B on
+    the device (-1 for padding and for out-of-range tokens)."""
+    n = positions.numel()
+    if req_indices.numel() != n or block_tables.dim() != 2:
+        raise ValueError("positions and req_indices need one entry per token; block_tables is [R, W]")
+    if slot_mapping is None:
+        slot_mapping = torch.empty(n, dtype=torch.int64, device=positions.device)
+    _check(lib.pa_compute_slot_mapping(_dev(positions, "positions", torch.int64),
+                                       _dev(req_indices, "req_indices", torch.int32), n,
+                                       _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                                       block_tables.shape[0], int(block_size), int(num_blocks),
+                                       _dev(slot_mapping, "slot_mapping", torch.int64), _stream_ptr(stream)),
+           "pa_compute_slot_mapping")
+    return slot_mapping
+
+
+def pa_write_kv_positions(k, v, positions, req_indices, block_tables, k_cache, v_cache, stream=None) -> None:
+    """pa_write_kv with each token's slot computed in the kernel from its
+    request row and position."""
+    cache = make_cache(k_cache, v_cache)
+    n = positions.numel()
+    if k.shape != v.shape or k.shape[0] != n or tuple(k.shape[1:]) != tuple(k_cache.shape[2:]):
+        raise ValueError("k, v must be [num_tokens, num_kv_heads, head_dim] matching positions and the cache")
+    if req_indices.numel() != n or block_tables.dim() != 2:
+        raise ValueError("req_indices needs one entry per token; block_tables is [R, W]")
+    _check(lib.pa_write_kv_positions(_dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+                                     _dev(positions, "positions", torch.int64),
+                                     _dev(req_indices, "req_indices", torch.int32), n,
+                                     _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                                     block_tables.shape[0], ctypes.byref(cache), _stream_ptr(stream)),
+           "pa_write_kv_positions")
+
+
 def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
     """cache[dst] = cache[src] for each (src, dst) row of an int64 [P, 2] tensor."""
     cache = make_cache(k_cache, v_cache)
@@ -120,6 +162,16 @@ def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
     p = src_dst_pairs.shape[0]
     ptr = _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if p else None
     _check(lib.pa_copy_blocks(ctypes.byref(cache), ptr, p, _stream_ptr(stream)), "pa_copy_blocks")
+
+
+def pa_copy_blocks_layers(caches, src_dst_pairs, stream=None) -> None:
+    """pa_copy_blocks over a list of (k_cache, v_cache) layers, one launch."""
+    arr = (PaCache * max(1, len(caches)))(*[make_cache(k, v) for k, v in caches])
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs, 2]")
+    p = src_dst_pairs.shape[0]
+    ptr = _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if p else None
+    _check(lib.pa_copy_blocks_layers(arr, len(caches), ptr, p, _stream_ptr(stream)), "pa_copy_blocks_layers")
 
 
 def pa_decode_workspace_bytes(num_seqs: int, num_q_heads: int, max_seq_len: int, k_cache, v_cache) -> int:

@@ -263,6 +263,51 @@ int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping, int64
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "write_kv_kernel launch");
 }
 
+int pa_compute_slot_mapping(const int64_t *positions, const int32_t *req_indices, int64_t num_tokens,
+                            const int32_t *block_tables, int32_t max_blocks_per_seq, int32_t num_reqs,
+                            int32_t block_size, int64_t num_blocks, int64_t *slot_mapping, void *stream) {
+    if (num_tokens < 0 || max_blocks_per_seq < 0 || num_reqs < 0 || num_blocks <= 0 || block_size <= 0)
+        return PA_EINVAL;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!positions || !req_indices || !slot_mapping || (num_reqs > 0 && !block_tables))
+        return PA_EINVAL;
+    const int64_t blocks = (num_tokens + pa::kSlotThreads - 1) / pa::kSlotThreads;
+    if (blocks > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::slot_mapping_kernel, dim3(static_cast<unsigned>(blocks)), dim3(pa::kSlotThreads),
+                               0, static_cast<cudaStream_t>(stream), positions, req_indices, num_tokens,
+                               block_tables, max_blocks_per_seq, num_reqs, block_size, num_blocks, slot_mapping);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "slot_mapping_kernel launch");
+}
+
+int pa_write_kv_positions(const void *k, const void *v, const int64_t *positions, const int32_t *req_indices,
+                          int64_t num_tokens, const int32_t *block_tables, int32_t max_blocks_per_seq,
+                          int32_t num_reqs, const pa_cache_t *cache, void *stream) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_tokens < 0 || max_blocks_per_seq < 0 || num_reqs < 0)
+        return PA_EINVAL;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!k || !v || !positions || !req_indices || (num_reqs > 0 && !block_tables))
+        return PA_EINVAL;
+    if (!aligned16(k) || !aligned16(v))
+        return PA_EUNSUPPORTED;
+    const int row_vecs = cache->num_kv_heads * cache->head_dim * 2 / 16;
+    const int64_t blocks = (num_tokens * 2 * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
+    if (blocks > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::write_kv_positions_kernel, dim3(static_cast<unsigned>(blocks)),
+                               dim3(pa::kWriteThreads), 0, static_cast<cudaStream_t>(stream),
+                               static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), positions,
+                               req_indices, num_tokens, block_tables, max_blocks_per_seq, num_reqs,
+                               cache->block_size, cache->num_blocks, static_cast<uint4 *>(cache->k_cache),
+                               static_cast<uint4 *>(cache->v_cache), row_vecs);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "write_kv_positions_kernel launch");
+}
+
 int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
                    void *stream) {
     int rc = check_cache(cache);
@@ -285,6 +330,37 @@ int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_
                                static_cast<uint4 *>(cache->v_cache), src_dst_pairs, cache->num_blocks,
                                block_vecs, chunks);
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_kernel launch");
+}
+
+int pa_copy_blocks_layers(const pa_cache_t *caches, int32_t num_layers, const int64_t *src_dst_pairs,
+                          int64_t num_pairs, void *stream) {
+    if (!caches || num_layers < 0 || num_layers > pa::kMaxLayers || num_pairs < 0)
+        return num_layers > pa::kMaxLayers ? PA_EUNSUPPORTED : PA_EINVAL;
+    pa::LayerPtrs lp{};
+    for (int32_t l = 0; l < num_layers; ++l) {
+        const int rc = check_cache(&caches[l]);
+        if (rc)
+            return rc;
+        if (caches[l].num_blocks != caches[0].num_blocks || caches[l].block_size != caches[0].block_size ||
+            caches[l].num_kv_heads != caches[0].num_kv_heads)
+            return PA_EINVAL;  // one pair list needs one block geometry
+        lp.k[l] = static_cast<uint4 *>(caches[l].k_cache);
+        lp.v[l] = static_cast<uint4 *>(caches[l].v_cache);
+    }
+    if (num_layers == 0 || num_pairs == 0)
+        return PA_OK;
+    if (!src_dst_pairs)
+        return PA_EINVAL;
+    const pa_cache_t *c = &caches[0];
+    const int64_t block_vecs = static_cast<int64_t>(c->block_size) * c->num_kv_heads * c->head_dim * 2 / 16;
+    const int chunks = static_cast<int>((block_vecs + pa::kCopyChunkVecs - 1) / pa::kCopyChunkVecs);
+    const int64_t grid = num_pairs * 2 * chunks;
+    if (grid > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::copy_blocks_layers_kernel, dim3(static_cast<unsigned>(grid), num_layers),
+                               dim3(pa::kCopyThreads), 0, static_cast<cudaStream_t>(stream), lp, src_dst_pairs,
+                               c->num_blocks, block_vecs, chunks);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_layers_kernel launch");
 }
 
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
