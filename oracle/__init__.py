@@ -71,6 +71,15 @@ def _load():
         lib.oracle_decode.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                       ctypes.c_double, P, i64, P]
         lib.oracle_decode.restype = ctypes.c_int
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = ctypes.c_double
+        lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+        lib.oracle_write_kv_fp8.argtypes = [P, P, P, i64, i64, i64, ctypes.c_float, ctypes.c_float, P, P]
+        lib.oracle_write_kv_fp8.restype = ctypes.c_int
+        lib.oracle_decode_fp8.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
+                                          ctypes.c_double, ctypes.c_double, ctypes.c_double, P]
+        lib.oracle_decode_fp8.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -172,4 +181,54 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, which=None
         raise ValueError("block id out of range or table too narrow")
     if rc:
         raise MemoryError("oracle_decode")
+    return out
+
+
+# ----------------------------------------------------------------------------
+# FP8 (OCP E4M3) KV cache ("The pantry of pigeonholes", "The 10 knobs", knob 4)
+# ----------------------------------------------------------------------------
+
+
+def e4m3_to_float64(codes) -> np.ndarray:
+    """Exact value of e4m3 codes (uint8 array)."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_to_double(int(x)) for x in c.reshape(-1)], np.float64).reshape(c.shape)
+
+
+def e4m3_from_float32(x) -> np.ndarray:
+    """e4m3 codes of float32 values: nearest even, |x| >= 448 saturates, NaN -> 0x7F."""
+    lib = _load()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([lib.oracle_e4m3_from_float(float(v)) for v in a.reshape(-1)], np.uint8).reshape(a.shape)
+
+
+def write_kv_fp8(k, v, slots, k_cache, v_cache, k_scale: float, v_scale: float) -> None:
+    """In place: codes of (bf16 row) / scale at the slots (negative = skip)."""
+    k = _req(k, np.uint16); v = _req(v, np.uint16); slots = _req(slots, np.int64)
+    k_cache = _req(k_cache, np.uint8); v_cache = _req(v_cache, np.uint8)
+    row = int(np.prod(k.shape[1:]))
+    rc = _load().oracle_write_kv_fp8(_ptr(k), _ptr(v), _ptr(slots), len(slots), row, k_cache.size // row,
+                                     float(k_scale), float(v_scale), _ptr(k_cache), _ptr(v_cache))
+    if rc:
+        raise ValueError("slot out of range")
+
+
+def decode_fp8(q, k_cache, v_cache, block_tables, seq_lens, scale: float, k_scale: float,
+               v_scale: float) -> np.ndarray:
+    """fp64 decode over an e4m3 cache (value = code value * scale of its tensor)."""
+    q = _req(q, np.uint16); k_cache = _req(k_cache, np.uint8); v_cache = _req(v_cache, np.uint8)
+    block_tables = _req(np.ascontiguousarray(block_tables, dtype=np.int32), np.int32)
+    seq_lens = _req(np.ascontiguousarray(seq_lens, dtype=np.int32), np.int32)
+    S, Hq, D = q.shape
+    NB, B, Hkv, D2 = k_cache.shape
+    assert D2 == D and Hq % Hkv == 0
+    out = np.full((S, Hq, D), np.nan, dtype=np.float64)
+    rc = _load().oracle_decode_fp8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                   block_tables.shape[1], _ptr(seq_lens), S, Hq, Hkv, D, B, NB,
+                                   float(scale), float(k_scale), float(v_scale), _ptr(out))
+    if rc == -1:
+        raise ValueError("block id out of range or table too narrow")
+    if rc:
+        raise MemoryError("oracle_decode_fp8")
     return out

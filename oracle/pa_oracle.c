@@ -202,3 +202,175 @@ int oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_
     free(z);
     return rc;
 }
+
+/* ------------------------------------------------------------------------
+ * FP8 (e4m3) KV cache.  The pages list an FP8 KV cache as a knob that halves
+ * the bytes per token ("The pantry of pigeonholes", "The 10 knobs", knob 4
+ * kv_cache_dtype; "How it connects to the rest of the stack", KV
+ * quantisation).  The format is OCP FP8 E4M3: 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits, no infinities, S.1111.111 = NaN, largest
+ * finite 448 = 1.75 * 2^8, subnormals m/8 * 2^-6 (smallest 2^-9).
+ * A stored code c of a tensor with scale s stands for value(c) * s.
+ * ------------------------------------------------------------------------ */
+
+/* value of an e4m3 code, exact in double */
+double oracle_e4m3_to_double(uint8_t c)
+{
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* x rounded to the nearest integer, ties to even (x has few significant
+ * bits here, so x + 0.5 is exact) */
+static double round_half_even(double x)
+{
+    double r = floor(x + 0.5);
+    if (r - x == 0.5 && fmod(r, 2.0) != 0.0)
+        r -= 1.0;
+    return r;
+}
+
+/* e4m3 code of a float: round to nearest even, magnitudes at or above 448
+ * (infinities included) saturate to 448, NaN gives 0x7F. */
+uint8_t oracle_e4m3_from_float(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    const uint8_t sign = (uint8_t)((u >> 31) << 7);
+    if (f != f)
+        return 0x7F;
+    const double a = fabs((double)f);
+    if (a >= 448.0)
+        return (uint8_t)(sign | 0x7E);
+    if (a < ldexp(1.0, -6)) {               /* subnormal range: k * 2^-9 */
+        const double k = round_half_even(a / ldexp(1.0, -9));
+        return (uint8_t)(sign | (uint8_t)k); /* k == 8 encodes 2^-6 (exponent 1) */
+    }
+    int e = (int)floor(log2(a));
+    if (ldexp(1.0, e) > a)                  /* guard log2 rounding */
+        e -= 1;
+    if (ldexp(1.0, e + 1) <= a)
+        e += 1;
+    double q = round_half_even((a / ldexp(1.0, e) - 1.0) * 8.0);
+    if (q == 8.0) {
+        q = 0.0;
+        e += 1;
+    }
+    if (e + 7 > 15 || (e + 7 == 15 && q > 6.0))
+        return (uint8_t)(sign | 0x7E);
+    return (uint8_t)(sign | ((e + 7) << 3) | (uint8_t)q);
+}
+
+/*
+ * FP8 write: each bf16 value x of token i's K (V) row is stored as the code
+ * of x / k_scale (x / v_scale), the quotient taken in float (IEEE division,
+ * round to nearest), at flat row slot_mapping[i] (negative = padding).
+ */
+int oracle_write_kv_fp8(const uint16_t *k, const uint16_t *v, const int64_t *slot_mapping,
+                        int64_t num_tokens, int64_t row_elems, int64_t num_slots, float k_scale,
+                        float v_scale, uint8_t *k_cache, uint8_t *v_cache)
+{
+    for (int64_t i = 0; i < num_tokens; ++i)
+        if (slot_mapping[i] >= num_slots)
+            return -1;
+    for (int64_t i = 0; i < num_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        for (int64_t e = 0; e < row_elems; ++e) {
+            const float kx = (float)bf16_to_double(k[i * row_elems + e]);
+            const float vx = (float)bf16_to_double(v[i * row_elems + e]);
+            k_cache[slot * row_elems + e] = oracle_e4m3_from_float(kx / k_scale);
+            v_cache[slot * row_elems + e] = oracle_e4m3_from_float(vx / v_scale);
+        }
+    }
+    return 0;
+}
+
+/*
+ * FP8 decode: as oracle_decode, with K_t[d] = value(code) * k_scale and
+ * V_t[d] = value(code) * v_scale (in double).
+ */
+int oracle_decode_fp8(const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                      const int32_t *block_tables, int32_t max_blocks_per_seq,
+                      const int32_t *seq_lens, int32_t num_seqs, int32_t num_q_heads,
+                      int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                      int64_t num_blocks, double scale, double k_scale, double v_scale,
+                      double *out)
+{
+    const int32_t group = num_q_heads / num_kv_heads;
+    int64_t max_n = 0;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        if (seq_lens[s] > max_n)
+            max_n = seq_lens[s];
+    double *kk = (double *)malloc((size_t)(max_n + 1) * head_dim * sizeof(double));
+    double *vv = (double *)malloc((size_t)(max_n + 1) * head_dim * sizeof(double));
+    double *z = (double *)malloc((size_t)(max_n + 1) * sizeof(double));
+    if (!kk || !vv || !z) {
+        free(kk); free(vv); free(z);
+        return -2;
+    }
+    int rc = 0;
+    for (int32_t s = 0; s < num_seqs && rc == 0; ++s) {
+        for (int32_t j = 0; j < num_q_heads && rc == 0; ++j) {
+            const int32_t h = j / group;
+            const int64_t n = seq_lens[s];
+            double *o = out + ((int64_t)s * num_q_heads + j) * head_dim;
+            if (n == 0) {
+                for (int32_t d = 0; d < head_dim; ++d)
+                    o[d] = 0.0;
+                continue;
+            }
+            if ((n + block_size - 1) / block_size > max_blocks_per_seq) {
+                rc = -1;
+                break;
+            }
+            for (int64_t t = 0; t < n; ++t) {
+                const int64_t blk = block_tables[(int64_t)s * max_blocks_per_seq + t / block_size];
+                if (blk < 0 || blk >= num_blocks) {
+                    rc = -1;
+                    break;
+                }
+                const int64_t row = (blk * block_size + t % block_size) * num_kv_heads + h;
+                for (int32_t d = 0; d < head_dim; ++d) {
+                    kk[t * head_dim + d] = oracle_e4m3_to_double(k_cache[row * head_dim + d]) * k_scale;
+                    vv[t * head_dim + d] = oracle_e4m3_to_double(v_cache[row * head_dim + d]) * v_scale;
+                }
+            }
+            if (rc)
+                break;
+            const uint16_t *qr = q + ((int64_t)s * num_q_heads + j) * head_dim;
+            double zmax = -INFINITY;
+            for (int64_t t = 0; t < n; ++t) {
+                double acc = 0.0;
+                for (int32_t d = 0; d < head_dim; ++d)
+                    acc += bf16_to_double(qr[d]) * kk[t * head_dim + d];
+                z[t] = scale * acc;
+                if (z[t] > zmax)
+                    zmax = z[t];
+            }
+            double denom = 0.0;
+            for (int64_t t = 0; t < n; ++t) {
+                z[t] = exp(z[t] - zmax);
+                denom += z[t];
+            }
+            for (int32_t d = 0; d < head_dim; ++d) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < n; ++t)
+                    acc += z[t] * vv[t * head_dim + d];
+                o[d] = acc / denom;
+            }
+        }
+    }
+    free(kk);
+    free(vv);
+    free(z);
+    return rc;
+}

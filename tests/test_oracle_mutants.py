@@ -28,15 +28,21 @@ MUTANTS = {
     "copy_in_place_chain": ("    /* gather */", "    goto scatter_now;\n    /* gather */"),
     "copy_wrong_direction": ("k_cache[d * block_elems + e] = tmp[(2 * p) * block_elems + e];",
                              "k_cache[pairs[2 * p] * block_elems + e] = tmp[(2 * p) * block_elems + e];"),
+    "e4m3_bias_8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_ties_away": ("    if (r - x == 0.5 && fmod(r, 2.0) != 0.0)\n        r -= 1.0;", ""),
+    "e4m3_no_saturation": ("    if (a >= 448.0)\n        return (uint8_t)(sign | 0x7E);", "    if (a >= 480.0)\n        return 0x7F;"),
+    "fp8_write_multiplies": ("oracle_e4m3_from_float(kx / k_scale)", "oracle_e4m3_from_float(kx * k_scale)"),
+    "fp8_v_scale_dropped": ("vv[t * head_dim + d] = oracle_e4m3_to_double(v_cache[row * head_dim + d]) * v_scale;",
+                            "vv[t * head_dim + d] = oracle_e4m3_to_double(v_cache[row * head_dim + d]);"),
 }
-PINS = ["tests/test_oracle_decode.py", "tests/test_oracle_formulas.py"]
+PINS = ["tests/test_oracle_decode.py", "tests/test_oracle_formulas.py", "tests/test_oracle_fp8.py"]
 
 
 def _build(name, tmp_path):
     src = open(SRC).read()
     old, new = MUTANTS[name]
-    assert src.count(old) == 1, name
-    mutated = src.replace(old, new)
+    assert src.count(old) >= 1, name
+    mutated = src.replace(old, new, 1)  # the first occurrence: the bf16 functions
     if name == "copy_in_place_chain":
         # read-modify-write pair by pair instead of reading all sources first
         mutated = mutated.replace("    /* scatter */", "scatter_now:\n    /* scatter */")
