@@ -73,6 +73,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-op", action="store_true")
     ap.add_argument("--part-tokens", type=int, default=0, help="split-K partition size (0 = automatic)")
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
+                    help="KV cache element type (fp8 = OCP E4M3 codes with per-tensor scales)")
     return ap.parse_args()
 
 
@@ -193,7 +195,8 @@ def profiled_traffic(config: str):
 def algorithmic_bytes(st) -> dict:
     """Bytes the step must move, per layer."""
     H, D, B = st.num_kv_heads, st.head_dim, st.block_size
-    row = H * D * 2  # one token's K (or V) row, bf16
+    esz = 1 if st.kv_dtype == "fp8" else 2
+    row = H * D * esz  # one token's K (or V) row in the cache
     slots = []
     for s in range(len(st.ids)):
         n = int(st.seq_lens_np[s])
@@ -206,7 +209,7 @@ def algorithmic_bytes(st) -> dict:
     return {
         "decode_kv": uniq * row * 2,  # K and V, each unique slot once
         "decode_kv_logical": logical * row * 2,
-        "write": T * row * 2 * 2,  # K and V rows read and written
+        "write": T * H * D * 2 * 2 + T * row * 2,  # bf16 K and V rows read, cache rows written
         "copy": P * B * row * 2 * 2,  # K and V blocks read and written
         "q_out": 2 * st.q.numel() * 2,
         "table": int(sum(-(-int(n) // B) for n in st.seq_lens_np)) * 4,
@@ -224,7 +227,8 @@ def run_ours(args, world, rank, local):
     if args.part_tokens:
         pa.pa_decode_set_partition_tokens(args.part_tokens)
     w = synth.by_name(args.config)
-    st = stage(w, dev, layers=args.layers)
+    fp8 = args.kv_dtype == "fp8"
+    st = stage(w, dev, layers=args.layers, kv_dtype=args.kv_dtype)
     L = args.layers
     nbytes = algorithmic_bytes(st)
     step_bytes = L * (nbytes["decode_kv"] + nbytes["write"] + nbytes["copy"])
@@ -234,15 +238,28 @@ def run_ours(args, world, rank, local):
     split = st.workspace is not None
     launches_per_layer = 2 + (1 if split else 0) + (1 if has_pairs else 0)
 
+    def write_op(k, v, slots, kc, vc):
+        if fp8:
+            pa.pa_write_kv_fp8(k, v, slots, kc, vc, st.k_scale, st.v_scale)
+        else:
+            pa.pa_write_kv(k, v, slots, kc, vc)
+
+    def decode_op(q, kc, vc, bt, lens):
+        if fp8:
+            pa.pa_decode_fp8(q, kc, vc, st.k_scale, st.v_scale, bt, lens, st.scale, out=st.out,
+                             max_seq_len=st.max_seq_len, workspace=st.workspace)
+        else:
+            pa.pa_decode(q, kc, vc, bt, lens, st.scale, out=st.out, max_seq_len=st.max_seq_len,
+                         workspace=st.workspace)
+
     def layer_ops(l, with_decode=True, with_write=True):
         kc, vc = st.caches[l]
         if with_write:
             if has_pairs:
                 pa.pa_copy_blocks(kc, vc, st.cow_pairs)
-            pa.pa_write_kv(st.k_new, st.v_new, st.slot_mapping, kc, vc)
+            write_op(st.k_new, st.v_new, st.slot_mapping, kc, vc)
         if with_decode:
-            pa.pa_decode(st.q, kc, vc, st.block_tables, st.seq_lens, st.scale, out=st.out,
-                         max_seq_len=st.max_seq_len, workspace=st.workspace)
+            decode_op(st.q, kc, vc, st.block_tables, st.seq_lens)
 
     def barrier():
         if world > 1:
@@ -298,7 +315,7 @@ def run_ours(args, world, rank, local):
 
     # ---- per-op times (graphs of one launch per layer) -------------------------
     per_op = {}
-    if not args.no_per_op:
+    if not args.no_per_op and not fp8:
         row = st.num_kv_heads * st.head_dim * 2
         T = st.slot_mapping.numel()
         pos = st.seq_lens.to(torch.int64) - 1  # decode step: the new token is the last
@@ -358,9 +375,8 @@ def run_ours(args, world, rank, local):
                 v_d.copy_(v_h, non_blocking=True)
                 if has_pairs:
                     pa.pa_copy_blocks(kc, vc, pairs_d)
-                pa.pa_write_kv(k_d, v_d, sm_d, kc, vc)
-                pa.pa_decode(q_d, kc, vc, bt_d, sl_d, st.scale, out=st.out, max_seq_len=st.max_seq_len,
-                             workspace=st.workspace)
+                write_op(k_d, v_d, sm_d, kc, vc)
+                decode_op(q_d, kc, vc, bt_d, sl_d)
                 out_h.copy_(st.out, non_blocking=True)
 
         e2e_step()
@@ -389,7 +405,7 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16 (fp8 e4m3 KV cache)" if fp8 else "bf16",
         "data": "synthetic (seeded N(0,1) bf16 K/V/q; seeded shuffled free list)",
         "config": {
             "workload": WORKLOAD_TEXT.get(args.config, args.config),
@@ -402,6 +418,7 @@ def run_ours(args, world, rank, local):
             "head_dim": st.head_dim,
             "max_seq_len": st.max_seq_len,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "kv_cache": f"fp8 e4m3, k_scale {st.k_scale}, v_scale {st.v_scale}" if fp8 else "bf16",
             "l2": f"inputs larger than L2: {L} distinct layer caches, "
                   f"{L * nbytes['decode_kv'] / 1e9:.2f} GB of KV touched per step",
             "timing": "CUDA graph of the whole step (all layers), replayed --steps times",
@@ -413,8 +430,9 @@ def run_ours(args, world, rank, local):
         "per_op": per_op,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(args.config) if not args.part_tokens else None,
-                     "kernel": "pa_decode (partition kernel" + (" + LSE merge)" if split else ")"),
+                     "traffic": profiled_traffic(args.config) if not (args.part_tokens or fp8) else None,
+                     "kernel": ("pa_decode_fp8" if fp8 else "pa_decode") + " (partition kernel"
+                               + (" + LSE merge)" if split else ")"),
                      "mean_launch_us": round(dec_mean_ms * 1e3, 3),
                      "how": f"CUDA graph of {L} back-to-back pa_decode calls (one per layer cache), "
                             f"{K} replays timed with CUDA events on the replay stream; mean per call",

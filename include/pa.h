@@ -227,6 +227,40 @@ PA_API int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int
                                int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
                                void *stream);
 
+/* ------------------------------------------------------------------------
+ * FP8 KV cache ("The pantry of pigeonholes", "The 10 knobs", knob 4
+ * kv_cache_dtype, and "How it connects to the rest of the stack": moving the
+ * KV to FP8 halves the bytes per token).  Codes are OCP FP8 E4M3 (one byte,
+ * bias 7, no infinities, largest finite 448); a code c of the K (V) tensor
+ * stands for value(c) * k_scale (v_scale), one scale per tensor.
+ * ------------------------------------------------------------------------ */
+typedef struct pa_cache_fp8 {
+    void *k_cache; /* [num_blocks][block_size][num_kv_heads][head_dim] e4m3 codes */
+    void *v_cache;
+    int64_t num_blocks;
+    int32_t block_size;
+    int32_t num_kv_heads;
+    int32_t head_dim;
+    float k_scale; /* > 0 */
+    float v_scale; /* > 0 */
+} pa_cache_fp8_t;
+
+/* pa_write_kv into an FP8 cache: each bf16 value x is stored as the code of
+ * x / scale, the quotient in fp32 (IEEE division), rounded to the nearest
+ * e4m3 value with ties to even and saturated at +-448 (infinities too).
+ * Slots as pa_write_kv (negative = padding; out of range flagged). */
+PA_API int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_mapping, int64_t num_tokens,
+                           const pa_cache_fp8_t *cache, void *stream);
+/* pa_decode over an FP8 cache: same contract and output as pa_decode, with
+ * K = value(code) * k_scale and V = value(code) * v_scale.  q and out stay
+ * bf16.  Scratch per pa_decode_fp8_workspace_bytes. */
+PA_API size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
+                                            const pa_cache_fp8_t *cache);
+PA_API int pa_decode_fp8(const void *q, const pa_cache_fp8_t *cache, const int32_t *block_tables,
+                         int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                         int32_t max_seq_len, int32_t num_q_heads, float scale, void *out, void *workspace,
+                         size_t workspace_bytes, void *stream);
+
 /* Read (and with clear != 0, reset) the device error word of the current
  * device.  Synchronises the device.  Returns PA_OK or PA_ECUDA. */
 PA_API int pa_get_device_error(int32_t *host_code, int clear);

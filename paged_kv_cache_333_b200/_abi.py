@@ -25,7 +25,8 @@ PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_COPY_PAIR, PA_D
 
 EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
             "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_static_ws", "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
+            "pa_decode_static_ws", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
+            "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
 
@@ -34,6 +35,13 @@ class PaCache(ctypes.Structure):
     _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
                 ("num_blocks", ctypes.c_int64), ("block_size", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32)]
+
+
+class PaCacheFp8(ctypes.Structure):
+    _fields_ = [("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+                ("num_blocks", ctypes.c_int64), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 _P = ctypes.c_void_p
@@ -57,6 +65,13 @@ lib.pa_decode_static_ws.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _
                                     _P, _P]
 lib.pa_decode_static_ws.restype = ctypes.c_int
 PA_DECODE_STATIC_WS_BYTES = 8 * 1024 * 1024
+lib.pa_write_kv_fp8.argtypes = [_P, _P, _P, _i64, ctypes.POINTER(PaCacheFp8), _P]
+lib.pa_write_kv_fp8.restype = ctypes.c_int
+lib.pa_decode_fp8_workspace_bytes.argtypes = [_i32, _i32, _i32, ctypes.POINTER(PaCacheFp8)]
+lib.pa_decode_fp8_workspace_bytes.restype = ctypes.c_size_t
+lib.pa_decode_fp8.argtypes = [_P, ctypes.POINTER(PaCacheFp8), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
+                              _P, _P, ctypes.c_size_t, _P]
+lib.pa_decode_fp8.restype = ctypes.c_int
 lib.pa_decode_set_kernel.argtypes = [_i32]
 lib.pa_decode_set_kernel.restype = _i32
 lib.pa_decode_set_partition_tokens.argtypes = [_i32]
@@ -106,6 +121,61 @@ def make_cache(k_cache: torch.Tensor, v_cache: torch.Tensor) -> PaCache:
     nb, bs, hkv, d = k_cache.shape
     return PaCache(_dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
                    nb, bs, hkv, d)
+
+
+def make_cache_fp8(k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: float, v_scale: float) -> PaCacheFp8:
+    """Describe one layer's FP8 (E4M3) caches: [num_blocks, block_size, H_kv, D]
+    uint8 (or float8_e4m3fn) codes, value = code * scale of its tensor."""
+    if k_cache.shape != v_cache.shape or k_cache.dim() != 4:
+        raise ValueError("k_cache and v_cache must both be [num_blocks, block_size, num_kv_heads, head_dim]")
+    kc = k_cache.view(torch.uint8) if k_cache.dtype != torch.uint8 else k_cache
+    vc = v_cache.view(torch.uint8) if v_cache.dtype != torch.uint8 else v_cache
+    nb, bs, hkv, d = k_cache.shape
+    return PaCacheFp8(_dev(kc, "k_cache", torch.uint8), _dev(vc, "v_cache", torch.uint8), nb, bs, hkv, d,
+                      float(k_scale), float(v_scale))
+
+
+def pa_write_kv_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale: float, v_scale: float, stream=None) -> None:
+    """KV write into an FP8 cache: code of (bf16 value / scale), nearest even, saturating."""
+    cache = make_cache_fp8(k_cache, v_cache, k_scale, v_scale)
+    n = slot_mapping.numel()
+    if k.shape != v.shape or k.shape[0] != n or tuple(k.shape[1:]) != tuple(k_cache.shape[2:]):
+        raise ValueError("k, v must be [num_tokens, num_kv_heads, head_dim] matching slot_mapping and the cache")
+    _check(lib.pa_write_kv_fp8(_dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
+                               _dev(slot_mapping, "slot_mapping", torch.int64), n, ctypes.byref(cache),
+                               _stream_ptr(stream)), "pa_write_kv_fp8")
+
+
+def pa_decode_fp8_workspace_bytes(num_seqs: int, num_q_heads: int, max_seq_len: int, k_cache, v_cache,
+                                  k_scale: float = 1.0, v_scale: float = 1.0) -> int:
+    cache = make_cache_fp8(k_cache, v_cache, k_scale, v_scale)
+    return int(lib.pa_decode_fp8_workspace_bytes(num_seqs, num_q_heads, max_seq_len, ctypes.byref(cache)))
+
+
+def pa_decode_fp8(q, k_cache, v_cache, k_scale: float, v_scale: float, block_tables, seq_lens, scale: float,
+                  out=None, max_seq_len: int | None = None, workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode over an FP8 cache (q and out bf16)."""
+    cache = make_cache_fp8(k_cache, v_cache, k_scale, v_scale)
+    if q.dim() != 3 or q.shape[2] != k_cache.shape[3]:
+        raise ValueError("q must be [num_seqs, num_q_heads, head_dim]")
+    S, Hq, _ = q.shape
+    if block_tables.dim() != 2 or block_tables.shape[0] != S or seq_lens.shape != (S,):
+        raise ValueError("block_tables must be [num_seqs, W] and seq_lens [num_seqs]")
+    if max_seq_len is None:
+        max_seq_len = int(seq_lens.max().item()) if S else 0
+    if out is None:
+        out = torch.empty_like(q)
+    need = int(lib.pa_decode_fp8_workspace_bytes(S, Hq, max_seq_len, ctypes.byref(cache)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace", torch.uint8) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib.pa_decode_fp8(_dev(q, "q", torch.bfloat16), ctypes.byref(cache),
+                             _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                             _dev(seq_lens, "seq_lens", torch.int32), S, int(max_seq_len), Hq, float(scale),
+                             _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes, _stream_ptr(stream)),
+           "pa_decode_fp8")
+    return out
 
 
 def pa_write_kv(k, v, slot_mapping, k_cache, v_cache, stream=None) -> None:

@@ -71,6 +71,8 @@ struct DecodeParams {
     int32_t part_tokens;
     int32_t num_parts;
     float scale_log2;
+    float k_scale;  // FP8 caches: value = code * k_scale (1 otherwise)
+    float v_scale;  // FP8 caches: value = code * v_scale (1 otherwise)
 };
 
 struct DecodeSmem {

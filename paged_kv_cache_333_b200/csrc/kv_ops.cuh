@@ -4,6 +4,8 @@
 // against the cache extent.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "pa_device.cuh"
 
 namespace pa {
@@ -141,6 +143,50 @@ write_kv_positions_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__
             if (i < row_vecs)
                 dst[i] = r[u];
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// pa_write_kv_fp8: the KV write into an FP8 (OCP E4M3) cache.  Each bf16
+// value x becomes the code of x / scale: the quotient in fp32 (IEEE division),
+// rounded to the nearest e4m3 value (ties to even), saturating at +-448.
+// One warp per (token, K|V); a lane turns 8 bf16 (16 bytes) into 8 codes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kWriteThreads)
+write_kv_fp8_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v,
+                    const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
+                    uint2 *__restrict__ k_cache, uint2 *__restrict__ v_cache, int64_t num_slots,
+                    int row_vecs, float k_scale, float v_scale) {
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kWriteThreads + threadIdx.x) >> 5;
+    const int64_t tok = warp >> 1;
+    if (tok >= num_tokens)
+        return;
+    const int64_t slot = slot_mapping[tok];
+    if (slot < 0)
+        return;
+    if (slot >= num_slots) {
+        if (lane == 0 && (warp & 1) == 0)
+            flag_error(PA_DEVERR_SLOT);
+        return;
+    }
+    const bool is_v = warp & 1;
+    const uint4 *src = (is_v ? v : k) + tok * row_vecs;
+    uint2 *dst = (is_v ? v_cache : k_cache) + slot * row_vecs;
+    const float sc = is_v ? v_scale : k_scale;
+    for (int i = lane; i < row_vecs; i += 32) {
+        const uint4 u = __ldg(src + i);
+        float f[8];
+        unpack8(u, f);
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t c = __nv_cvt_float_to_fp8(__fdiv_rn(f[e], sc), __NV_SATFINITE, __NV_E4M3);
+            w[e >> 2] |= (c & 0xffu) << (8 * (e & 3));
+        }
+        dst[i] = make_uint2(w[0], w[1]);
     }
 }
 

@@ -15,6 +15,7 @@
 
 #include "decode.cuh"
 #include "decode_mma.cuh"
+#include "decode_fp8.cuh"
 #include "kv_ops.cuh"
 #include "pa.h"
 #include "pa_device.cuh"
@@ -25,9 +26,7 @@ thread_local char g_last_cuda_error[256] = "";
 int32_t g_part_tokens_override = 0;
 int32_t g_decode_kernel = PA_DECODE_KERNEL_MMA;
 
-int ctas_per_sm() {
-    return g_decode_kernel == PA_DECODE_KERNEL_MMA ? pa::kMmaCtasPerSm : pa::kDecodeCtasPerSm;
-}
+
 
 int cuda_fail(cudaError_t e, const char *what) {
     std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", what, cudaGetErrorString(e));
@@ -75,16 +74,16 @@ int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 // the merge work and the workspace).  A multiple of 64 (so of the tile and
 // of every block size), and at most the per-CTA table capacity.
 int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_seq_len,
-                           int32_t block_size) {
-    const int64_t max_blocks =
-        g_decode_kernel == PA_DECODE_KERNEL_MMA ? pa::kMaxPartBlocksM : pa::kMaxPartBlocks;
+                           int32_t block_size, bool tensor_core_kernel) {
+    const int64_t max_blocks = tensor_core_kernel ? pa::kMaxPartBlocksM : pa::kMaxPartBlocks;
     const int64_t cap = max_blocks * block_size;
     int64_t part;
     if (g_part_tokens_override > 0) {
         part = g_part_tokens_override;
     } else {
         const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
-        const int64_t slots = static_cast<int64_t>(sm_count()) * ctas_per_sm();
+        const int64_t slots = static_cast<int64_t>(sm_count()) *
+                              (tensor_core_kernel ? pa::kMmaCtasPerSm : pa::kDecodeCtasPerSm);
         const int64_t len = max_seq_len > 0 ? max_seq_len : 1;
         part = std::max<int64_t>(640, (len * units + 16 * slots - 1) / (16 * slots));
         if (part >= len)
@@ -102,9 +101,10 @@ struct WorkspaceLayout {
 };
 
 WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
-                                 int32_t max_seq_len, int32_t block_size) {
+                                 int32_t max_seq_len, int32_t block_size,
+                                 bool tensor_core_kernel = g_decode_kernel == PA_DECODE_KERNEL_MMA) {
     WorkspaceLayout w{};
-    w.part_tokens = choose_part_tokens(num_seqs, num_kv_heads, max_seq_len, block_size);
+    w.part_tokens = choose_part_tokens(num_seqs, num_kv_heads, max_seq_len, block_size, tensor_core_kernel);
     w.num_parts = max_seq_len > 0 ? static_cast<int32_t>((max_seq_len + w.part_tokens - 1) / w.part_tokens) : 1;
     if (w.num_parts <= 1) {
         w.num_parts = 1;
@@ -133,7 +133,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 3-D view of one cache tensor: (dim, kv head, slot).  CUDA-core kernel:
 // box (128, 1, min(B, 16)), no swizzle.  Tensor-core kernel: box (64, 1,
 // min(B, 16)) with the 128-byte swizzle, loaded as two 64-dim halves.
-int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c, bool swizzled) {
+int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c, bool swizzled, bool fp8 = false) {
     auto fn = encode_fn();
     if (!fn) {
         std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
@@ -142,12 +142,16 @@ int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c, bool swiz
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(c->head_dim),
                                 static_cast<cuuint64_t>(c->num_kv_heads),
                                 static_cast<cuuint64_t>(c->num_blocks) * c->block_size};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(c->head_dim) * 2,
-                                   static_cast<cuuint64_t>(c->num_kv_heads) * c->head_dim * 2};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(swizzled ? 64 : c->head_dim), 1u,
+    const cuuint64_t esz = fp8 ? 1 : 2;
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(c->head_dim) * esz,
+                                   static_cast<cuuint64_t>(c->num_kv_heads) * c->head_dim * esz};
+    // one row of the box is at most 128 bytes under the 128-byte swizzle
+    const cuuint32_t inner = swizzled ? static_cast<cuuint32_t>(128 / esz) : static_cast<cuuint32_t>(c->head_dim);
+    const cuuint32_t box[3] = {inner, 1u,
                                static_cast<cuuint32_t>(c->block_size < pa::kTile ? c->block_size : pa::kTile)};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+    CUresult r = fn(tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
+                    strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -233,6 +237,50 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
     return PA_OK;
 }
 
+}  // namespace
+
+namespace {
+pa_cache_t as_cache(const pa_cache_fp8_t *c) {
+    pa_cache_t r{};
+    r.k_cache = c->k_cache;
+    r.v_cache = c->v_cache;
+    r.num_blocks = c->num_blocks;
+    r.block_size = c->block_size;
+    r.num_kv_heads = c->num_kv_heads;
+    r.head_dim = c->head_dim;
+    return r;
+}
+
+int check_cache_fp8(const pa_cache_fp8_t *c) {
+    if (!c)
+        return PA_EINVAL;
+    const pa_cache_t b = as_cache(c);
+    const int rc = check_cache(&b);
+    if (rc)
+        return rc;
+    if (!(c->k_scale > 0.f) || !(c->v_scale > 0.f) || !std::isfinite(c->k_scale) || !std::isfinite(c->v_scale))
+        return PA_EINVAL;
+    return PA_OK;
+}
+
+template <int G>
+int launch_decode_fp8_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
+                        int32_t num_kv_heads, cudaStream_t stream) {
+    static bool done[64] = {};
+    int rc = prepare_kernel(pa::decode_partition_fp8_kernel<G>, pa::kDecodeSmemBytesF, done);
+    if (rc)
+        return rc;
+    cudaError_t e = launch_pdl(pa::decode_partition_fp8_kernel<G>, dim3(p.num_parts, num_kv_heads, p.num_seqs),
+                               dim3(pa::kDecodeThreadsM), pa::kDecodeSmemBytesF, stream, tk, tv, p);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "decode_partition_fp8_kernel launch");
+    if (p.num_parts > 1) {
+        e = launch_pdl(pa::decode_merge_kernel, dim3(p.num_q_heads, p.num_seqs, 1), dim3(pa::kD), 0, stream, p);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "decode_merge_kernel launch");
+    }
+    return PA_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -363,6 +411,104 @@ int pa_copy_blocks_layers(const pa_cache_t *caches, int32_t num_layers, const in
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_layers_kernel launch");
 }
 
+
+int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_mapping, int64_t num_tokens,
+                    const pa_cache_fp8_t *cache, void *stream) {
+    int rc = check_cache_fp8(cache);
+    if (rc)
+        return rc;
+    if (num_tokens < 0)
+        return PA_EINVAL;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!k || !v || !slot_mapping)
+        return PA_EINVAL;
+    if (!aligned16(k) || !aligned16(v))
+        return PA_EUNSUPPORTED;
+    const int row_vecs = cache->num_kv_heads * cache->head_dim * 2 / 16;
+    const int64_t blocks = (num_tokens * 2 * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
+    if (blocks > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::write_kv_fp8_kernel, dim3(static_cast<unsigned>(blocks)), dim3(pa::kWriteThreads),
+                               0, static_cast<cudaStream_t>(stream), static_cast<const uint4 *>(k),
+                               static_cast<const uint4 *>(v), slot_mapping, num_tokens,
+                               static_cast<uint2 *>(cache->k_cache), static_cast<uint2 *>(cache->v_cache),
+                               cache->num_blocks * cache->block_size, row_vecs, cache->k_scale, cache->v_scale);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "write_kv_fp8_kernel launch");
+}
+
+size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
+                                     const pa_cache_fp8_t *cache) {
+    if (check_cache_fp8(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
+        return 0;
+    return workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size, true).total;
+}
+
+int pa_decode_fp8(const void *q, const pa_cache_fp8_t *cache, const int32_t *block_tables,
+                  int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs, int32_t max_seq_len,
+                  int32_t num_q_heads, float scale, void *out, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+    int rc = check_cache_fp8(cache);
+    if (rc)
+        return rc;
+    if (num_seqs < 0 || max_seq_len < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
+        return PA_EINVAL;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (!q || !block_tables || !seq_lens || !out)
+        return PA_EINVAL;
+    if (num_q_heads % cache->num_kv_heads != 0)
+        return PA_EINVAL;
+    const int32_t G = num_q_heads / cache->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return PA_EUNSUPPORTED;
+    if (!aligned16(q) || !aligned16(out))
+        return PA_EUNSUPPORTED;
+    if (num_seqs > 65535 || cache->num_kv_heads > 65535)
+        return PA_EUNSUPPORTED;
+    if (!std::isfinite(scale))
+        return PA_EINVAL;
+    const WorkspaceLayout w =
+        workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size, true);
+    if (w.total > 0 && (workspace == nullptr || workspace_bytes < w.total))
+        return PA_EWORKSPACE;
+    if (w.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return PA_EUNSUPPORTED;
+    const pa_cache_t view = as_cache(cache);
+    CUtensorMap tk, tv;
+    if ((rc = encode_cache_map(&tk, cache->k_cache, &view, true, true)) != PA_OK)
+        return rc;
+    if ((rc = encode_cache_map(&tv, cache->v_cache, &view, true, true)) != PA_OK)
+        return rc;
+    pa::DecodeParams p{};
+    p.q = static_cast<const uint4 *>(q);
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.part_ml = w.total ? static_cast<float2 *>(workspace) : nullptr;
+    p.part_acc = w.total ? reinterpret_cast<float *>(static_cast<char *>(workspace) + w.acc_offset) : nullptr;
+    p.num_blocks = cache->num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.block_size = cache->block_size;
+    p.part_tokens = w.part_tokens;
+    p.num_parts = w.num_parts;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);  // log2(e)
+    p.k_scale = cache->k_scale;
+    p.v_scale = cache->v_scale;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (G) {
+    case 1: return launch_decode_fp8_g<1>(tk, tv, p, cache->num_kv_heads, st);
+    case 2: return launch_decode_fp8_g<2>(tk, tv, p, cache->num_kv_heads, st);
+    case 4: return launch_decode_fp8_g<4>(tk, tv, p, cache->num_kv_heads, st);
+    default: return launch_decode_fp8_g<8>(tk, tv, p, cache->num_kv_heads, st);
+    }
+}
+
 size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
                                  const pa_cache_t *cache) {
     if (check_cache(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
@@ -440,6 +586,8 @@ int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_table
     p.part_tokens = w.part_tokens;
     p.num_parts = w.num_parts;
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);  // log2(e)
+    p.k_scale = 1.f;
+    p.v_scale = 1.f;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (G) {

@@ -18,10 +18,12 @@ import dataclasses
 import numpy as np
 import torch
 
-from ._abi import pa_copy_blocks, pa_decode, pa_decode_workspace_bytes, pa_write_kv
+from ._abi import (pa_copy_blocks, pa_decode, pa_decode_fp8, pa_decode_fp8_workspace_bytes,
+                   pa_decode_workspace_bytes, pa_write_kv, pa_write_kv_fp8)
 from .pool import BlockPool
 
 POISON_BITS = 0x7FC1  # a bf16 quiet NaN
+POISON_FP8 = 0x7F  # the e4m3 NaN code
 
 
 def to_device_bf16(a: np.ndarray, device) -> torch.Tensor:
@@ -61,9 +63,12 @@ class DeviceStep:
     slot_mapping_np: np.ndarray
     cow_pairs_np: np.ndarray
     history_pairs_np: np.ndarray
+    kv_dtype: str = "bf16"
+    k_scale: float = 1.0
+    v_scale: float = 1.0
 
 
-def _write_rows(w, pool, kc, vc, items, device, chunk_tokens=1 << 16):
+def _write_rows(w, pool, kc, vc, items, device, chunk_tokens=1 << 16, fp8_scales=None):
     """Write logical rows (sid, a, b) at the pool's slots, in chunks."""
     buf_k, buf_v, buf_s, n = [], [], [], 0
 
@@ -73,7 +78,10 @@ def _write_rows(w, pool, kc, vc, items, device, chunk_tokens=1 << 16):
             k = to_device_bf16(np.concatenate(buf_k), device)
             v = to_device_bf16(np.concatenate(buf_v), device)
             s = torch.from_numpy(np.concatenate(buf_s)).to(device)
-            pa_write_kv(k, v, s, kc, vc)
+            if fp8_scales is None:
+                pa_write_kv(k, v, s, kc, vc)
+            else:
+                pa_write_kv_fp8(k, v, s, kc, vc, *fp8_scales)
         buf_k, buf_v, buf_s, n = [], [], [], 0
 
     for sid, a, b in items:
@@ -88,24 +96,34 @@ def _write_rows(w, pool, kc, vc, items, device, chunk_tokens=1 << 16):
     flush()
 
 
-def stage(w, device="cuda", layers: int = 1, rule: str = "shared", poison: bool = True) -> DeviceStep:
+def stage(w, device="cuda", layers: int = 1, rule: str = "shared", poison: bool = True,
+          kv_dtype: str = "bf16", k_scale: float = 1.0 / 64, v_scale: float = 1.0 / 64) -> DeviceStep:
+    """kv_dtype "bf16" (default) or "fp8" (E4M3 codes, value = code * scale)."""
     sh = w.shape
     pool = BlockPool(sh.num_blocks, sh.block_size, w.free_order, rule)
     w.ops(pool)
-    fill = POISON_BITS if poison else 0
     shape = (sh.num_blocks, sh.block_size, sh.num_kv_heads, sh.head_dim)
-    kc = torch.full(shape, fill, dtype=torch.int16, device=device).view(torch.bfloat16)
-    vc = torch.full(shape, fill, dtype=torch.int16, device=device).view(torch.bfloat16)
+    fp8 = kv_dtype == "fp8"
+    if fp8:
+        fill = POISON_FP8 if poison else 0
+        kc = torch.full(shape, fill, dtype=torch.uint8, device=device)
+        vc = torch.full(shape, fill, dtype=torch.uint8, device=device)
+        scales = (k_scale, v_scale)
+    else:
+        fill = POISON_BITS if poison else 0
+        kc = torch.full(shape, fill, dtype=torch.int16, device=device).view(torch.bfloat16)
+        vc = torch.full(shape, fill, dtype=torch.int16, device=device).view(torch.bfloat16)
+        scales = None
 
     if w.shared_len:
-        _write_rows(w, pool, kc, vc, [(w.seq_ids[0], 0, w.shared_len)], device)
+        _write_rows(w, pool, kc, vc, [(w.seq_ids[0], 0, w.shared_len)], device, fp8_scales=scales)
     if w.suffix_ops is not None:
         w.suffix_ops(pool)
     hist_pairs = pool.take_cow_pairs()
     if len(hist_pairs):
         pa_copy_blocks(kc, vc, torch.from_numpy(hist_pairs).to(device))
     _write_rows(w, pool, kc, vc,
-                [(sid, w.shared_len, pool.seq_len(sid)) for sid in w.seq_ids], device)
+                [(sid, w.shared_len, pool.seq_len(sid)) for sid in w.seq_ids], device, fp8_scales=scales)
 
     # the step: one new token per sequence
     for sid in w.seq_ids:
@@ -123,7 +141,10 @@ def stage(w, device="cuda", layers: int = 1, rule: str = "shared", poison: bool 
     S = len(w.seq_ids)
     q = to_device_bf16(w.q, device)
     max_len = int(lens.max()) if S else 0
-    need = pa_decode_workspace_bytes(S, sh.num_q_heads, max_len, kc, vc)
+    if fp8:
+        need = pa_decode_fp8_workspace_bytes(S, sh.num_q_heads, max_len, kc, vc, k_scale, v_scale)
+    else:
+        need = pa_decode_workspace_bytes(S, sh.num_q_heads, max_len, kc, vc)
     ws = torch.empty(need, dtype=torch.uint8, device=device) if need else None
     return DeviceStep(
         pool=pool, ids=list(w.seq_ids), num_q_heads=sh.num_q_heads, num_kv_heads=sh.num_kv_heads,
@@ -134,15 +155,22 @@ def stage(w, device="cuda", layers: int = 1, rule: str = "shared", poison: bool 
         block_tables=torch.from_numpy(bt).to(device), seq_lens=torch.from_numpy(lens).to(device),
         max_seq_len=max_len, scale=w.scale, out=torch.empty_like(q), workspace=ws,
         block_tables_np=bt, seq_lens_np=lens, slot_mapping_np=slots,
-        cow_pairs_np=pairs.reshape(-1, 2), history_pairs_np=hist_pairs.reshape(-1, 2))
+        cow_pairs_np=pairs.reshape(-1, 2), history_pairs_np=hist_pairs.reshape(-1, 2),
+        kv_dtype=kv_dtype, k_scale=k_scale, v_scale=v_scale)
 
 
 def run_step(st: DeviceStep, layer: int = 0, stream=None, out: torch.Tensor | None = None) -> torch.Tensor:
     """One decode step on one layer: queued copies, the step's KV write, decode."""
     kc, vc = st.caches[layer]
+    out = st.out if out is None else out
+    if st.kv_dtype == "fp8":
+        if st.cow_pairs.shape[0]:
+            raise NotImplementedError("copy-on-write pairs with an FP8 cache")
+        pa_write_kv_fp8(st.k_new, st.v_new, st.slot_mapping, kc, vc, st.k_scale, st.v_scale, stream=stream)
+        return pa_decode_fp8(st.q, kc, vc, st.k_scale, st.v_scale, st.block_tables, st.seq_lens, st.scale,
+                             out=out, max_seq_len=st.max_seq_len, workspace=st.workspace, stream=stream)
     if st.cow_pairs.shape[0]:
         pa_copy_blocks(kc, vc, st.cow_pairs, stream=stream)
     pa_write_kv(st.k_new, st.v_new, st.slot_mapping, kc, vc, stream=stream)
-    return pa_decode(st.q, kc, vc, st.block_tables, st.seq_lens, st.scale,
-                     out=st.out if out is None else out, max_seq_len=st.max_seq_len,
-                     workspace=st.workspace, stream=stream)
+    return pa_decode(st.q, kc, vc, st.block_tables, st.seq_lens, st.scale, out=out,
+                     max_seq_len=st.max_seq_len, workspace=st.workspace, stream=stream)
