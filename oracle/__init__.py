@@ -8,7 +8,9 @@ when it is missing instead of falling back to anything here.
 Contents
 --------
 - ``pa_oracle.c`` (compiled to ``liboracle.so`` by :func:`build`): write,
-  copy-on-write block copy and decode attention in plain C, fp64.
+  copy-on-write block copy, decode attention, attention of several query
+  tokens per request (query_start_loc, causal) and the FP8 (E4M3) write and
+  decode, in plain C, fp64.
 - :func:`slot_of` / :func:`slot_mapping` / :func:`blocks_for` /
   :func:`tail_waste`: the slot, block-count and waste formulas, in Python.
 - ``oracle.pool``: a pure-Python model of the block pool (free list,
@@ -23,6 +25,10 @@ How each piece is pinned to something other than itself (the tests under
   dominant key gives its V row; a single token gives V_0 exactly), invariance
   under any permutation of physical blocks and any block size, brute force on
   tiny inputs, NaN poison in unused storage;
+- multi-token attention: whole and chunked prefill against ``torch``'s causal
+  scaled dot-product attention in float64, one row per request equal to the
+  decode, running means of V under all-equal keys, placement and block-size
+  invariance;
 - slot / block / waste formulas: the worked examples printed on the pages
   (slot 30,608 for request r7; cdiv(4097, 16) = 257; tail waste 15/1/0/15;
   the simulator's 4 blocks, 2 slots of slack, 50 slots of contiguous waste);
@@ -71,6 +77,9 @@ def _load():
         lib.oracle_decode.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                       ctypes.c_double, P, i64, P]
         lib.oracle_decode.restype = ctypes.c_int
+        lib.oracle_attention.argtypes = [P, P, P, P, i32, P, P, i32, i32, i32, i32, i32, i64,
+                                         ctypes.c_double, P]
+        lib.oracle_attention.restype = ctypes.c_int
         lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_to_double.restype = ctypes.c_double
         lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
@@ -181,6 +190,35 @@ def decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, which=None
         raise ValueError("block id out of range or table too narrow")
     if rc:
         raise MemoryError("oracle_decode")
+    return out
+
+
+def attention(q, k_cache, v_cache, block_tables, query_start_loc, seq_lens, scale: float) -> np.ndarray:
+    """fp64 attention of several query tokens per request over the paged cache
+    (causal within each request: query row i of a request with q_len rows and
+    n computed tokens attends to positions 0 .. n - q_len + i).  q: uint16
+    [T, H_q, D] with T = query_start_loc[-1]; caches uint16 [NB, B, H_kv, D];
+    block_tables int32 [R, W]; query_start_loc int32 [R + 1]; seq_lens int32
+    [R].  Returns float64 [T, H_q, D]."""
+    q = _req(q, np.uint16); k_cache = _req(k_cache, np.uint16); v_cache = _req(v_cache, np.uint16)
+    block_tables = _req(np.ascontiguousarray(block_tables, dtype=np.int32), np.int32)
+    qsl = _req(np.ascontiguousarray(query_start_loc, dtype=np.int32), np.int32)
+    seq_lens = _req(np.ascontiguousarray(seq_lens, dtype=np.int32), np.int32)
+    T, Hq, D = q.shape
+    NB, B, Hkv, D2 = k_cache.shape
+    R = len(seq_lens)
+    assert D2 == D and Hq % Hkv == 0 and len(qsl) == R + 1 and block_tables.shape[0] == R
+    assert qsl[0] == 0 and qsl[-1] == T
+    out = np.full((T, Hq, D), np.nan, dtype=np.float64)
+    rc = _load().oracle_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                                  block_tables.shape[1], _ptr(qsl), _ptr(seq_lens), R, Hq, Hkv, D, B, NB,
+                                  float(scale), _ptr(out))
+    if rc == -1:
+        raise ValueError("block id out of range or table too narrow")
+    if rc == -3:
+        raise ValueError("a request has more query rows than computed tokens")
+    if rc:
+        raise MemoryError("oracle_attention")
     return out
 
 

@@ -203,6 +203,116 @@ int oracle_decode(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_
     return rc;
 }
 
+/*
+ * Attention for several query tokens per request over the paged cache
+ * ("PagedAttention: fragmentation, blocks, block tables", the attention
+ * metadata passage: query_start_loc is [num_reqs + 1], the start of each
+ * request's rows in the query tensor; seq_lens is [num_reqs], the computed
+ * tokens of each request; max_query_len is the longest query).
+ *
+ * Reading (the pages name the fields but do not spell the masking out): the
+ * q_len = query_start_loc[r+1] - query_start_loc[r] query rows of request r
+ * are its last q_len tokens, whose K/V are already in the cache and counted
+ * in n = seq_lens[r].  Query row i (0-based within the request) is the token
+ * at position n - q_len + i and attends to positions 0 .. n - q_len + i
+ * (causal).  q_len = 1 is one decode step; q_len = n is a whole prefill.
+ *
+ * For each request r, query row i and query head j (KV head h = j / group):
+ *   1. rebuild the contiguous K and V of (r, h) through the block table;
+ *   2. z_t = scale * q[row][j] . K_t for t = 0 .. n - q_len + i;
+ *   3. p_t = exp(z_t - max z) / sum exp(z - max z);
+ *   4. out[row][j] = sum_t p_t V_t.
+ * `out` is double [num_tokens][num_q_heads][head_dim] with num_tokens =
+ * query_start_loc[num_reqs].  Returns 0; -1 for a block id out of range or a
+ * table too narrow; -2 on OOM; -3 for q_len < 0 or q_len > n.
+ */
+int oracle_attention(const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                     const int32_t *block_tables, int32_t max_blocks_per_seq,
+                     const int32_t *query_start_loc, const int32_t *seq_lens, int32_t num_reqs,
+                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t block_size, int64_t num_blocks, double scale, double *out)
+{
+    const int32_t group = num_q_heads / num_kv_heads;
+    int64_t max_n = 0;
+    for (int32_t r = 0; r < num_reqs; ++r) {
+        int64_t q_len = (int64_t)query_start_loc[r + 1] - query_start_loc[r];
+        if (q_len < 0 || q_len > seq_lens[r])
+            return -3;
+        if (seq_lens[r] > max_n)
+            max_n = seq_lens[r];
+    }
+    double *kk = (double *)malloc((size_t)(max_n + 1) * head_dim * sizeof(double));
+    double *vv = (double *)malloc((size_t)(max_n + 1) * head_dim * sizeof(double));
+    double *z = (double *)malloc((size_t)(max_n + 1) * sizeof(double));
+    if (!kk || !vv || !z) {
+        free(kk); free(vv); free(z);
+        return -2;
+    }
+    int rc = 0;
+    for (int32_t r = 0; r < num_reqs && rc == 0; ++r) {
+        const int64_t n = seq_lens[r];
+        const int64_t row0 = query_start_loc[r];
+        const int64_t q_len = query_start_loc[r + 1] - row0;
+        if (q_len == 0)
+            continue;
+        if ((n + block_size - 1) / block_size > max_blocks_per_seq) {
+            rc = -1;
+            break;
+        }
+        for (int32_t h = 0; h < num_kv_heads && rc == 0; ++h) {
+            /* 1. contiguous K, V of (r, h) */
+            for (int64_t t = 0; t < n; ++t) {
+                int64_t blk = block_tables[(int64_t)r * max_blocks_per_seq + t / block_size];
+                if (blk < 0 || blk >= num_blocks) {
+                    rc = -1;
+                    break;
+                }
+                int64_t slot_row = (blk * block_size + t % block_size) * num_kv_heads + h;
+                for (int32_t d = 0; d < head_dim; ++d) {
+                    kk[t * head_dim + d] = bf16_to_double(k_cache[slot_row * head_dim + d]);
+                    vv[t * head_dim + d] = bf16_to_double(v_cache[slot_row * head_dim + d]);
+                }
+            }
+            if (rc)
+                break;
+            for (int64_t i = 0; i < q_len; ++i) {
+                const int64_t visible = n - q_len + i + 1; /* positions 0 .. n - q_len + i */
+                for (int32_t j = h * group; j < (h + 1) * group; ++j) {
+                    const uint16_t *qr = q + ((row0 + i) * num_q_heads + j) * head_dim;
+                    double *o = out + ((row0 + i) * num_q_heads + j) * head_dim;
+                    /* 2. scores */
+                    double zmax = -INFINITY;
+                    for (int64_t t = 0; t < visible; ++t) {
+                        double acc = 0.0;
+                        for (int32_t d = 0; d < head_dim; ++d)
+                            acc += bf16_to_double(qr[d]) * kk[t * head_dim + d];
+                        z[t] = scale * acc;
+                        if (z[t] > zmax)
+                            zmax = z[t];
+                    }
+                    /* 3. softmax weights and their sum */
+                    double denom = 0.0;
+                    for (int64_t t = 0; t < visible; ++t) {
+                        z[t] = exp(z[t] - zmax);
+                        denom += z[t];
+                    }
+                    /* 4. weighted sum of V */
+                    for (int32_t d = 0; d < head_dim; ++d) {
+                        double acc = 0.0;
+                        for (int64_t t = 0; t < visible; ++t)
+                            acc += z[t] * vv[t * head_dim + d];
+                        o[d] = acc / denom;
+                    }
+                }
+            }
+        }
+    }
+    free(kk);
+    free(vv);
+    free(z);
+    return rc;
+}
+
 /* ------------------------------------------------------------------------
  * FP8 (e4m3) KV cache.  The pages list an FP8 KV cache as a knob that halves
  * the bytes per token ("The pantry of pigeonholes", "The 10 knobs", knob 4

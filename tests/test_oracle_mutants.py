@@ -28,6 +28,13 @@ MUTANTS = {
     "copy_in_place_chain": ("    /* gather */", "    goto scatter_now;\n    /* gather */"),
     "copy_wrong_direction": ("k_cache[d * block_elems + e] = tmp[(2 * p) * block_elems + e];",
                              "k_cache[pairs[2 * p] * block_elems + e] = tmp[(2 * p) * block_elems + e];"),
+    "attn_no_causal_mask": ("const int64_t visible = n - q_len + i + 1;", "const int64_t visible = n;"),
+    "attn_top_left_causal": ("const int64_t visible = n - q_len + i + 1;", "const int64_t visible = i + 1;"),
+    "attn_excludes_own_token": ("const int64_t visible = n - q_len + i + 1;", "const int64_t visible = n - q_len + i;"),
+    "attn_rows_reversed": ("const uint16_t *qr = q + ((row0 + i) * num_q_heads + j) * head_dim;",
+                           "const uint16_t *qr = q + ((row0 + q_len - 1 - i) * num_q_heads + j) * head_dim;"),
+    "attn_gqa_modulo": ("for (int32_t j = h * group; j < (h + 1) * group; ++j) {",
+                        "for (int32_t j = h; j < num_q_heads; j += num_kv_heads) {"),
     "e4m3_bias_8": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "e4m3_ties_away": ("    if (r - x == 0.5 && fmod(r, 2.0) != 0.0)\n        r -= 1.0;", ""),
     "e4m3_no_saturation": ("    if (a >= 448.0)\n        return (uint8_t)(sign | 0x7E);", "    if (a >= 480.0)\n        return 0x7F;"),
@@ -35,7 +42,8 @@ MUTANTS = {
     "fp8_v_scale_dropped": ("vv[t * head_dim + d] = oracle_e4m3_to_double(v_cache[row * head_dim + d]) * v_scale;",
                             "vv[t * head_dim + d] = oracle_e4m3_to_double(v_cache[row * head_dim + d]);"),
 }
-PINS = ["tests/test_oracle_decode.py", "tests/test_oracle_formulas.py", "tests/test_oracle_fp8.py"]
+PINS = ["tests/test_oracle_decode.py", "tests/test_oracle_formulas.py", "tests/test_oracle_fp8.py",
+        "tests/test_oracle_attention.py"]
 
 
 def _build(name, tmp_path):
