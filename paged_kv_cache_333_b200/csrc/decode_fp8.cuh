@@ -5,25 +5,40 @@
 // stack": moving the KV to FP8 halves the bytes per token).  A stored code c
 // of the K (V) tensor stands for value(c) * k_scale (v_scale).
 //
-// Same CTA decomposition, producer and split-K as decode_mma.cuh; a 16-token
-// tile is now 2 KiB of K and 2 KiB of V (rows of 128 one-byte codes, 128-byte
-// swizzle), so the ring has twice the stages for the same bytes in flight.
-// The consumer feeds the codes straight into f16 tensor-core MMAs (every
-// e4m3 value is exact in f16), without a staging pass through shared memory:
-//   * K: ldmatrix (b16) on the code tile gives each lane four consecutive
-//     codes of a row (dims 4(lane%4)..+3 of a 16-dim chunk); converted to two
-//     f16 pairs they fill the A-operand slots of MMA k-indices 2q, 2q+1
-//     (dims 4q, 4q+1) and 2q+8, 2q+9 (dims 4q+2, 4q+3), q = lane % 4.  The
-//     reduction dimension is only reordered, so q's B operand is loaded with
-//     the same order and S^T is unchanged.
-//   * V: ldmatrix.trans (b16) on the code tile gives each lane codes of two
-//     consecutive tokens for a pair of dims (2r, 2r+1), r = lane / 4; a byte
-//     permute splits them into the (token, token+1) pairs of dim 2r and of dim
-//     2r+1, which become A-operand rows r and r+8 of V^T.  Only the output rows
-//     of O^T are reordered (row m <-> dim 2m, row m+8 <-> dim 2m+1), which the
-//     epilogue undoes.
-//   * scales: k_scale joins the softmax scale (scores * scale*k_scale*log2 e);
-//     v_scale multiplies the partition's accumulator in the epilogue.
+// Same CTA decomposition, producer and split-K as decode_mma.cuh.  With half
+// the bytes per token the consumer, not HBM, would set the pace if every code
+// were first converted to f16 (one conversion per two codes, about 2x the
+// instructions of the bf16 consumer per byte).  Here the codes go into the
+// FP8 tensor-core MMA as they are (mma.m16n8k32, e4m3 x e4m3, fp32
+// accumulate), and the two operands that are not codes are written as sums of
+// two e4m3 numbers:
+//   * q: each query head is scaled by a power of two 2^s_j that brings its
+//     largest |element| into [128, 256), then split as q' = hi + lo with
+//     hi = e4m3(q'), lo = e4m3(q' - hi).  For a bf16 q this is exact (the
+//     residual of rounding 8 significant bits to 4 has at most 4) except for
+//     elements below 2^-10 of the head's largest, whose error is under 2^-18
+//     of it.  S = K.hi + K.lo (two MMAs), and 2^-s_j joins the score scale.
+//   * P: probabilities are formed as 256 * 2^(x - m) (the factor cancels in
+//     acc / l and in the split-K merge), rounded to f16 for the movmatrix
+//     transpose, then split the same way; hi + lo keeps 8 significant bits,
+//     the precision bf16 P has in the bf16 kernel.
+// A tile is 32 tokens (4 KiB of K codes + 4 KiB of V codes, 128-byte
+// swizzled rows of 128 codes), which gives four independent MMA chains for
+// S^T and spreads the per-tile softmax reductions over twice the tokens.
+//
+// Operand layouts (lane = 4g + t):
+//   * K (A of S^T = K Q^T, m16 tokens x k32 dims): ldmatrix.x4 (b16) on the
+//     code tile gives exactly the e4m3 A fragment (row g / g+8, codes
+//     4t..4t+3 and 16+4t..16+4t+3 of the 32-dim step): no rearrangement.
+//   * P^T (B of O^T = V^T P^T, k32 tokens x n8 heads): movmatrix.trans of the
+//     f16 pairs leaves lane (g, t) with head g at tokens {2t, 2t+1} of each
+//     8-token group; the B fragment's k index 4t + i (+16) is assigned the
+//     tokens {2t, 2t+1, 8+2t, 9+2t} (+16): a permutation of the reduction.
+//   * V^T (A of the same MMA, m16 dims x k32 tokens): ldmatrix.x4.trans (b16)
+//     gives lane (g, t) the codes of dims 16c+2g, 16c+2g+1 for tokens 2t, 2t+1
+//     of each 8-token group; one byte permute per register builds the A
+//     fragment with the same token permutation, A row g <-> dim 16c + 2g and
+//     row g+8 <-> dim 16c + 2g + 1 (undone in the epilogue).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -33,12 +48,13 @@
 
 namespace pa {
 
-constexpr int kStagesF = 12;
-constexpr int kTileBytesF = kTile * kD;  // 16 tokens x 128 one-byte codes
+constexpr int kTileF = 32;
+constexpr int kStagesF = 6;
+constexpr int kTileBytesF = kTileF * kD;  // 32 tokens x 128 one-byte codes
 static_assert(kStagesF % kConsumerWarpsM == 0, "stages must be a multiple of the consumer warps");
 
 struct DecodeSmemF {
-    uint8_t kv[kStagesF][2][kTileBytesF];  // [stage][K, V][16 x 128], 128B-swizzled rows
+    uint8_t kv[kStagesF][2][kTileBytesF];  // [stage][K, V][32 x 128], 128B-swizzled rows
     uint64_t full[kStagesF];
     uint64_t empty[kStagesF];
     float wm[kConsumerWarpsM][8];
@@ -49,13 +65,28 @@ static_assert(sizeof(float) * kConsumerWarpsM * 8 * kD <= sizeof(uint8_t) * kSta
               "merge scratch must fit in the KV ring");
 constexpr size_t kDecodeSmemBytesF = sizeof(DecodeSmemF) + 1024;
 
-__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                              uint32_t b1) {
+// D = A(16x32 e4m3, row) * B(32x8 e4m3, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// Two f16 (low half first) -> two e4m3 codes (low byte first), nearest even,
+// saturating.
+__device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t h2) {
+    __half2_raw r;
+    r.x = static_cast<unsigned short>(h2 & 0xffffu);
+    r.y = static_cast<unsigned short>(h2 >> 16);
+    return __nv_cvt_halfraw2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
 }
 
 // Two e4m3 codes (low byte first) -> two f16 values (exact), low half first.
@@ -65,9 +96,30 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-    const __half2 v = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&v);
+// f16x2 value v -> (hi, lo) e4m3x2 code pairs with v ~ hi + lo (hi nearest to
+// v, lo nearest to the residual v - hi, which f16 holds exactly).
+__device__ __forceinline__ void split_f16x2(uint32_t v, uint32_t &hi, uint32_t &lo) {
+    hi = f16x2_to_e4m3x2(v);
+    const uint32_t back = e4m3x2_to_f16x2(hi);
+    const __half2 r = __hsub2(*reinterpret_cast<const __half2 *>(&v), *reinterpret_cast<const __half2 *>(&back));
+    lo = f16x2_to_e4m3x2(*reinterpret_cast<const uint32_t *>(&r));
+}
+
+// Four floats -> (hi, lo) codes, byte i from x[i].
+__device__ __forceinline__ void split_f32x4(const float (&x)[4], uint32_t &hi, uint32_t &lo) {
+    uint32_t hc[2], lc[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const __nv_fp8x2_storage_t c =
+            __nv_cvt_float2_to_fp8x2(make_float2(x[2 * k], x[2 * k + 1]), __NV_SATFINITE, __NV_E4M3);
+        const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(c, __NV_E4M3);
+        const float r0 = x[2 * k] - __half2float(__ushort_as_half(b.x));  // raw bits, not a numeric cast
+        const float r1 = x[2 * k + 1] - __half2float(__ushort_as_half(b.y));
+        hc[k] = c;
+        lc[k] = __nv_cvt_float2_to_fp8x2(make_float2(r0, r1), __NV_SATFINITE, __NV_E4M3);
+    }
+    hi = hc[0] | (hc[1] << 16);
+    lo = lc[0] | (lc[1] << 16);
 }
 
 template <int G>
@@ -111,7 +163,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (part > 0 && t_begin >= n)
         return;
     const int t_end = min(n, t_begin + p.part_tokens);
-    const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTile - 1) / kTile : 0;
+    const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTileF - 1) / kTileF : 0;
     const int Hkv = gridDim.y;
     if (warp == kConsumerWarpsM && num_tiles > 0) {
         const int nblk = (t_end - 1) / B - first_blk + 1;
@@ -131,6 +183,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         if (num_tiles == 0 || !use_tma)
             return;
         const uint64_t pol = l2_evict_first_policy();
+        const int rows = B < kTileF ? B : kTileF;  // tokens per box (the tensor map's box height)
         int issued = 0;
         for (int it = 0; it < num_tiles; ++it) {
             const int slot = it % kStagesF;
@@ -141,10 +194,9 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                 if (!__shfl_sync(FULL, ok, 0))
                     break;
             }
-            const int t0 = t_begin + it * kTile;
-            const int ntok = min(kTile, t_end - t0);
-            const int rows = B < kTile ? B : kTile;
-            const int nb = B >= kTile ? 1 : (ntok + B - 1) / B;
+            const int t0 = t_begin + it * kTileF;
+            const int ntok = min(kTileF, t_end - t0);
+            const int nb = (ntok + rows - 1) / rows;  // boxes per tensor (blocks of B < 32 tokens)
             if (lane == 0)
                 mbar_arrive_expect_tx(&sm.full[slot], static_cast<uint32_t>(nb * rows * kD * 2));
             __syncwarp();
@@ -166,71 +218,117 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
 
     // =================================================================== consumers
-    // q as the B operand, with the reduction order of the K fragments: for
-    // k-step ks, b0 = q[n][16ks + 4(lane%4) + {0,1}], b1 = ... + {2,3}.
-    const int qn = lane >> 2;
-    const int q4 = (lane & 3) * 4;
-    uint32_t qb[8][2];
+    const int g = lane >> 2;  // MMA group: S^T token row / B column (head)
+    const int t4 = lane & 3;  // thread in group
+    // q as the B operand of S^T, split into e4m3 hi + lo after a per-head
+    // power-of-two scale.  Lane (g, t) holds head g, dims 32kk + 4t + i
+    // (register 0) and 32kk + 16 + 4t + i (register 1) of k-step kk.
+    uint32_t qh[4][2], ql[4][2];
+    float sl2A, sl2B;  // score scale (log2 domain) of heads 2t and 2t+1
     {
-        const int qh = qn < G ? qn : G - 1;
+        const int qr = g < G ? g : G - 1;
         const __nv_bfloat16 *qrow = reinterpret_cast<const __nv_bfloat16 *>(p.q) +
-                                    (static_cast<int64_t>(s) * p.num_q_heads + h * G + qh) * kD;
+                                    (static_cast<int64_t>(s) * p.num_q_heads + h * G + qr) * kD;
+        float qv[4][2][4];
+        float amax = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint2 u = __ldg(reinterpret_cast<const uint2 *>(qrow + 16 * ks + q4));
-            const float a0 = bf16lo(u.x), a1 = bf16hi(u.x), a2 = bf16lo(u.y), a3 = bf16hi(u.y);
-            qb[ks][0] = qn < G ? pack_f16x2(a0, a1) : 0u;
-            qb[ks][1] = qn < G ? pack_f16x2(a2, a3) : 0u;
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(qrow + 32 * kk + 16 * r + 4 * t4));
+                qv[kk][r][0] = g < G ? bf16lo(u.x) : 0.f;
+                qv[kk][r][1] = g < G ? bf16hi(u.x) : 0.f;
+                qv[kk][r][2] = g < G ? bf16lo(u.y) : 0.f;
+                qv[kk][r][3] = g < G ? bf16hi(u.y) : 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    amax = fmaxf(amax, fabsf(qv[kk][r][i]));
+            }
         }
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
+        // 2^sh brings amax into [128, 256): amax in [2^(e-1), 2^e) -> sh = 8 - e.
+        int sh = 0;
+        if (amax > 0.f && amax <= 3.0e38f) {
+            int e;
+            frexpf(amax, &e);
+            sh = max(-120, min(126, 8 - e));
+        }
+        const float up = __int_as_float((127 + sh) << 23);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                float x[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    x[i] = qv[kk][r][i] * up;
+                split_f32x4(x, qh[kk][r], ql[kk][r]);
+            }
+        }
+        const float base = p.scale_log2 * p.k_scale;
+        const int shA = __shfl_sync(FULL, sh, 8 * t4);      // head 2t lives in group 2t
+        const int shB = __shfl_sync(FULL, sh, 8 * t4 + 4);  // head 2t+1 in group 2t+1
+        sl2A = base * __int_as_float((127 - shA) << 23);
+        sl2B = base * __int_as_float((127 - shB) << 23);
     }
-    const float sl2 = p.scale_log2 * p.k_scale;
     float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
     float acc[8][4];
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-        acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    for (int c = 0; c < 8; ++c)
+        acc[c][0] = acc[c][1] = acc[c][2] = acc[c][3] = 0.f;
 
-    const int mi = lane >> 3;                                  // which 8x8 matrix of an x4 load
+    const int mi = lane >> 3;  // which 8x8 matrix of an x4 load this lane addresses
     const int k_tok = (lane & 7) + ((mi & 1) << 3), k_chk = mi >> 1;
-    const int v_tok = (lane & 7) + ((mi >> 1) << 3), v_chk = mi & 1;
-    const int tok0 = lane >> 2;
 
     auto consume = [&](int slot, int ntok, auto &&loaded) {
         const uint32_t kb = smem_addr(&sm.kv[slot][0][0]);
         const uint32_t vb = smem_addr(&sm.kv[slot][1][0]);
-        if (ntok < kTile) {
+        if (ntok < kTileF) {
             uint4 *v = reinterpret_cast<uint4 *>(&sm.kv[slot][1][0]);
-            for (int idx = ntok * 8 + lane; idx < kTile * 8; idx += 32)
+            for (int idx = ntok * 8 + lane; idx < kTileF * 8; idx += 32)
                 v[idx] = make_uint4(0, 0, 0, 0);
             __syncwarp();
         }
-        uint32_t kr[4][4], vr[4][4];
+        // ---- S^T = K Q^T for tokens 16mt + {g, g+8}, heads 2t, 2t+1
+        float shi[2][4], slo[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            ldmatrix_x4(kr[j], kb + swz(k_tok, 2 * j + k_chk));
-            ldmatrix_x4_trans(vr[j], vb + swz(v_tok, 2 * j + v_chk));
-        }
-        loaded();
-
-        // ---- S^T = K Q^T: k-step 2j+hf uses registers 2hf (tokens 0-7) and 2hf+1 (8-15)
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+            for (int i = 0; i < 4; ++i)
+                shi[mt][i] = slo[mt][i] = 0.f;
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const uint32_t lo = kr[j][2 * hf], hi = kr[j][2 * hf + 1];
-                const uint32_t a[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi), e4m3x2_to_f16x2(lo >> 16),
-                                       e4m3x2_to_f16x2(hi >> 16)};
-                mma_16816_f16(sc, a, qb[2 * j + hf][0], qb[2 * j + hf][1]);
+        for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+                uint32_t kf[4];
+                ldmatrix_x4(kf, kb + swz(16 * mt + k_tok, 2 * kk + k_chk));
+                mma_16832_e4m3(shi[mt], kf, qh[kk][0], qh[kk][1]);
+                mma_16832_e4m3(slo[mt], kf, ql[kk][0], ql[kk][1]);
             }
         }
+        // V^T fragments: matrix i of load c = tokens 8i..8i+7, dims 16c..16c+15;
+        // the stage is released once they are in registers.
+        uint32_t vf[8][4];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            ldmatrix_x4_trans(vf[c], vb + swz(lane, c));
+        loaded();
         // ---- online softmax (log2 domain) -------------------------------
-        float x0 = sc[0] * sl2, x1 = sc[1] * sl2, x2 = sc[2] * sl2, x3 = sc[3] * sl2;
-        if (ntok < kTile) {
-            if (tok0 >= ntok) x0 = x1 = -INFINITY;
-            if (tok0 + 8 >= ntok) x2 = x3 = -INFINITY;
+        float x[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            x[mt][0] = (shi[mt][0] + slo[mt][0]) * sl2A;
+            x[mt][1] = (shi[mt][1] + slo[mt][1]) * sl2B;
+            x[mt][2] = (shi[mt][2] + slo[mt][2]) * sl2A;
+            x[mt][3] = (shi[mt][3] + slo[mt][3]) * sl2B;
+            if (ntok < kTileF) {
+                if (16 * mt + g >= ntok) x[mt][0] = x[mt][1] = -INFINITY;
+                if (16 * mt + g + 8 >= ntok) x[mt][2] = x[mt][3] = -INFINITY;
+            }
         }
-        float tA = fmaxf(x0, x2), tB = fmaxf(x1, x3);
+        float tA = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+        float tB = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
 #pragma unroll
         for (int off = 4; off <= 16; off <<= 1) {
             tA = fmaxf(tA, __shfl_xor_sync(FULL, tA, off));
@@ -240,32 +338,50 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         const float aA = exp2f(mA - nA), aB = exp2f(mB - nB);
         mA = nA;
         mB = nB;
-        const float p0 = exp2f(x0 - nA), p1 = exp2f(x1 - nB);
-        const float p2 = exp2f(x2 - nA), p3 = exp2f(x3 - nB);
-        lA = fmaf(lA, aA, p0 + p2);
-        lB = fmaf(lB, aB, p1 + p3);
-        const uint32_t pb0 = movmatrix_trans(pack_f16x2(p0, p1));  // tokens 0..7
-        const uint32_t pb1 = movmatrix_trans(pack_f16x2(p2, p3));  // tokens 8..15
-        // ---- O^T += V^T P^T: m-tile 2j+hh from matrices hh (tokens 0-7) and 2+hh (8-15)
+        // 256 * 2^(x - m): p in [0, 256], clear of the e4m3 subnormals
+        const float oA = nA - 8.f, oB = nB - 8.f;
+        float pr[2][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int mt = 0; mt < 2; ++mt) {
+            pr[mt][0] = exp2f(x[mt][0] - oA);
+            pr[mt][1] = exp2f(x[mt][1] - oB);
+            pr[mt][2] = exp2f(x[mt][2] - oA);
+            pr[mt][3] = exp2f(x[mt][3] - oB);
+        }
+        lA = fmaf(lA, aA, (pr[0][0] + pr[0][2]) + (pr[1][0] + pr[1][2]));
+        lB = fmaf(lB, aB, (pr[0][1] + pr[0][3]) + (pr[1][1] + pr[1][3]));
+        // P^T as the B operand: movmatrix k gives head g, tokens 8k + 2t, 8k + 2t + 1
+        uint32_t ph[4], pl[4];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int mt = 2 * j + hh;
-                acc[mt][0] *= aA;
-                acc[mt][1] *= aB;
-                acc[mt][2] *= aA;
-                acc[mt][3] *= aB;
-                const uint32_t lo = vr[j][hh], hi = vr[j][2 + hh];
-                const uint32_t a[4] = {e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x4420)),   // dim 2r, tokens 0-7
-                                       e4m3x2_to_f16x2(__byte_perm(lo, 0, 0x4431)),   // dim 2r+1
-                                       e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x4420)),   // dim 2r, tokens 8-15
-                                       e4m3x2_to_f16x2(__byte_perm(hi, 0, 0x4431))};  // dim 2r+1
-                mma_16816_f16(acc[mt], a, pb0, pb1);
+        for (int mt = 0; mt < 2; ++mt) {
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t u = movmatrix_trans(pack_f16x2(pr[mt][2 * hf], pr[mt][2 * hf + 1]));
+                split_f16x2(u, ph[2 * mt + hf], pl[2 * mt + hf]);
             }
         }
+        const uint32_t pbh0 = __byte_perm(ph[0], ph[1], 0x5410), pbh1 = __byte_perm(ph[2], ph[3], 0x5410);
+        const uint32_t pbl0 = __byte_perm(pl[0], pl[1], 0x5410), pbl1 = __byte_perm(pl[2], pl[3], 0x5410);
+        // ---- O^T = alpha O^T + V^T P^T: d-tile c, A row g <-> dim 16c+2g, row
+        // g+8 <-> 16c+2g+1.  The tile's product starts from zero and joins the
+        // running sum in fp32 outside the MMA, so the sum over thousands of
+        // tiles does not depend on how the FP8 MMA rounds its accumulator.
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t a[4] = {__byte_perm(vf[c][0], vf[c][1], 0x6420),   // dim 2g, tokens 2t,2t+1,8+2t,9+2t
+                                   __byte_perm(vf[c][0], vf[c][1], 0x7531),   // dim 2g+1
+                                   __byte_perm(vf[c][2], vf[c][3], 0x6420),   // dim 2g, tokens +16
+                                   __byte_perm(vf[c][2], vf[c][3], 0x7531)};  // dim 2g+1, tokens +16
+            float o[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_16832_e4m3(o, a, pbh0, pbh1);
+            mma_16832_e4m3(o, a, pbl0, pbl1);
+            acc[c][0] = fmaf(acc[c][0], aA, o[0]);
+            acc[c][1] = fmaf(acc[c][1], aB, o[1]);
+            acc[c][2] = fmaf(acc[c][2], aA, o[2]);
+            acc[c][3] = fmaf(acc[c][3], aB, o[3]);
+        }
     };
-    auto tile_tokens = [&](int it) { return min(kTile, t_end - (t_begin + it * kTile)); };
+    auto tile_tokens = [&](int it) { return min(kTileF, t_end - (t_begin + it * kTileF)); };
 
     if (use_tma) {
         for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
@@ -277,7 +393,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                 break;
             const int ntok = tile_tokens(it);
             consume(slot, ntok, [&] {
-                if (ntok < kTile)
+                if (ntok < kTileF)
                     fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0)
@@ -293,7 +409,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         auto gather = [&](int it) {
             if (it < num_tiles) {
                 const int slot = it % kStagesF;
-                const int t0 = t_begin + it * kTile;
+                const int t0 = t_begin + it * kTileF;
                 const int ntok = tile_tokens(it);
                 int64_t my_row = 0;
                 if (lane < ntok) {
@@ -334,16 +450,16 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
     float *wacc = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [warp][8 heads][D]
     {
-        const int hA = (lane & 3) * 2;
+        const int hA = t4 * 2;
         float *wa = wacc + (warp * 8 + hA) * kD;
         float *wb = wa + kD;
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            const int d = mt * 16 + 2 * tok0;  // O^T row m <-> dim 2m, row m+8 <-> dim 2m+1
-            wa[d] = acc[mt][0];
-            wb[d] = acc[mt][1];
-            wa[d + 1] = acc[mt][2];
-            wb[d + 1] = acc[mt][3];
+        for (int c = 0; c < 8; ++c) {
+            const int d = c * 16 + 2 * g;  // O^T row g <-> dim 16c+2g, row g+8 <-> dim 16c+2g+1
+            wa[d] = acc[c][0];
+            wb[d] = acc[c][1];
+            wa[d + 1] = acc[c][2];
+            wb[d + 1] = acc[c][3];
         }
         if (lane < 4) {
             sm.wm[warp][hA] = mA;
@@ -354,26 +470,26 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int gq = 0; gq < G; ++gq) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kConsumerWarpsM; ++w)
-            M = fmaxf(M, sm.wm[w][g]);
+            M = fmaxf(M, sm.wm[w][gq]);
         float L = 0.f, o[2] = {0.f, 0.f};
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kConsumerWarpsM; ++w) {
-                const float mw = sm.wm[w][g];
+                const float mw = sm.wm[w][gq];
                 if (mw == -INFINITY)
                     continue;
                 const float sc = exp2f(mw - M);
-                L = fmaf(sm.wl[w][g], sc, L);
+                L = fmaf(sm.wl[w][gq], sc, L);
 #pragma unroll
                 for (int u = 0; u < 2; ++u)
-                    o[u] = fmaf(wacc[(w * 8 + g) * kD + threadIdx.x + 64 * u], sc, o[u]);
+                    o[u] = fmaf(wacc[(w * 8 + gq) * kD + threadIdx.x + 64 * u], sc, o[u]);
             }
         }
-        const int jq = h * G + g;
+        const int jq = h * G + gq;
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int d = threadIdx.x + 64 * u;

@@ -147,8 +147,9 @@ int encode_cache_map(CUtensorMap *tm, void *base, const pa_cache_t *c, bool swiz
                                    static_cast<cuuint64_t>(c->num_kv_heads) * c->head_dim * esz};
     // one row of the box is at most 128 bytes under the 128-byte swizzle
     const cuuint32_t inner = swizzled ? static_cast<cuuint32_t>(128 / esz) : static_cast<cuuint32_t>(c->head_dim);
-    const cuuint32_t box[3] = {inner, 1u,
-                               static_cast<cuuint32_t>(c->block_size < pa::kTile ? c->block_size : pa::kTile)};
+    // box height: one block, at most one tile (16 tokens of bf16, 32 of fp8)
+    const int32_t tile = fp8 ? pa::kTileF : pa::kTile;
+    const cuuint32_t box[3] = {inner, 1u, static_cast<cuuint32_t>(c->block_size < tile ? c->block_size : tile)};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
                     strides, box, estr,

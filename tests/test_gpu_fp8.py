@@ -118,7 +118,43 @@ def test_fp8_scales_fold_exactly(pa):
     assert torch.equal(c, a)
 
 
-@pytest.mark.parametrize("name", ["chat", "sweep_b1"])
+def _scale_heads(q, factors):
+    f = np.asarray(factors, np.float32)[None, :, None]
+    return synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(q) * f)
+
+
+def test_fp8_query_magnitudes_per_head(pa):
+    """The kernel scales each query head by a power of two before splitting
+    it into two e4m3 terms; heads 10^-6 .. 10^3 apart, in one KV group and in
+    different groups, must all match the oracle."""
+    fac = [1e-6, 3e-3, 1.0, 40.0, 2e-4, 7.0, 0.5, 900.0]
+    q, kc, vc, bt, n = _case(81, [1, 31, 32, 33, 500, 1500], 16, 8, 2)
+    q = _scale_heads(q, fac)
+    ref = oracle.decode_fp8(q, kc, vc, bt, n, 0.08838834764831845 / 64, KS, VS)
+    _close(_run(pa, q, kc, vc, bt, n, scale=0.08838834764831845 / 64), ref, "per-head magnitudes")
+
+
+def test_fp8_query_wide_dynamic_range(pa):
+    """One query element 2^12 larger than the rest of its head: the small
+    elements fall below the split's exact range and must still not matter."""
+    q, kc, vc, bt, n = _case(82, [77, 640], 32, 8, 8)
+    qf = synth.bf16_bits_to_f32(q) * np.float32(1e-3)
+    qf[:, :, 5] = 4.0
+    q = synth.f32_to_bf16_bits(qf)
+    ref = oracle.decode_fp8(q, kc, vc, bt, n, 0.5, KS, VS)
+    _close(_run(pa, q, kc, vc, bt, n, scale=0.5), ref, "wide dynamic range")
+
+
+@pytest.mark.parametrize("scale", [1e-4, 0.3, 2.0])
+def test_fp8_flat_and_peaked_softmax(pa, scale):
+    """Nearly uniform weights (small scale) and nearly one-hot ones (large
+    scale): the probabilities' two-term split covers both ends."""
+    q, kc, vc, bt, n = _case(83, [5, 64, 999, 3000], 16, 16, 4)
+    ref = oracle.decode_fp8(q, kc, vc, bt, n, scale, KS, VS)
+    _close(_run(pa, q, kc, vc, bt, n, scale=scale), ref, f"scale={scale}")
+
+
+@pytest.mark.parametrize("name", ["chat", "sweep_b1", "long"])
 def test_fp8_workload_parity(pa, name):
     """A full-size workload staged into FP8 caches by the GPU write: codes
     equal the oracle's, decode within tolerance of the fp8 oracle."""
