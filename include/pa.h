@@ -55,7 +55,10 @@ enum {
     PA_DEVERR_SEQ_LEN = 4,    /* pa_decode: seq_len < 0, > max_seq_len, or needing more than
                                  max_blocks_per_seq table entries (clamped) */
     PA_DEVERR_COPY_PAIR = 8,  /* pa_copy_blocks: id outside [0, num_blocks) (pair skipped) */
-    PA_DEVERR_TIMEOUT = 16    /* a pipeline wait gave up after its time limit */
+    PA_DEVERR_TIMEOUT = 16,   /* a pipeline wait gave up after its time limit */
+    PA_DEVERR_QUERY_LOC = 32  /* pa_attention: query_start_loc not a non-decreasing split of
+                                 [0, num_tokens), or a request with more rows than tokens or
+                                 than max_query_len (its rows are left unwritten) */
 };
 
 /* One layer's paged KV cache.  k_cache and v_cache are separate tensors of
@@ -183,6 +186,42 @@ PA_API int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *bloc
               int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
               int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_attention -- attention of several query tokens per request over the
+ * paged cache (speculative tokens, chunks of a prefill; one row per request
+ * is a decode step).
+ * Defined by: "PagedAttention: fragmentation, blocks, block tables", the
+ * attention-metadata passage: query_start_loc [num_reqs + 1] gives the start
+ * of each request's rows in the query tensor, seq_lens [num_reqs] the
+ * computed tokens of each request, max_query_len the longest query, and the
+ * block table is walked as for pa_decode.  The pages do not spell the mask
+ * out; the reading taken is the causal one: the q_len = query_start_loc[r+1]
+ * - query_start_loc[r] rows of request r are its last q_len tokens (their K/V
+ * already written and counted in n = seq_lens[r]), and row i attends to
+ * positions 0 .. n - q_len + i.  For row i of request r and query head j
+ * (h = j / (num_q_heads / num_kv_heads)):
+ *   out[q0 + i][j] = sum_{t <= n-q_len+i} softmax_t(scale * q[q0+i][j] . K[r,h,t]) V[r,h,t].
+ *   q                [num_tokens][num_q_heads][head_dim] bf16 (16-byte aligned).
+ *   query_start_loc  [num_reqs + 1] int32 on the device: 0 = loc[0] <= loc[1]
+ *                    <= ... <= loc[num_reqs] = num_tokens, each step at most
+ *                    max_query_len and at most that request's seq_len
+ *                    (checked on the device: PA_DEVERR_QUERY_LOC).
+ *   max_query_len    host-side upper bound of the rows per request (sizes the grid).
+ *   block_tables, seq_lens, max_seq_len  as for pa_decode, per request.
+ *   out              [num_tokens][num_q_heads][head_dim] bf16.
+ *   workspace        device scratch of at least pa_attention_workspace_bytes(...)
+ *                    bytes (may be NULL when that is 0).
+ * Supports the bf16 cache; group sizes 1, 2, 4, 8.  Returns PA_EUNSUPPORTED
+ * when num_reqs * ceil(max_query_len * group / 32) exceeds 65535.
+ */
+PA_API size_t pa_attention_workspace_bytes(int32_t num_reqs, int32_t num_tokens, int32_t max_query_len,
+                                           int32_t num_q_heads, int32_t max_seq_len, const pa_cache_t *cache);
+PA_API int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_loc, int32_t num_reqs,
+                        int32_t max_query_len, const pa_cache_t *cache, const int32_t *block_tables,
+                        int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t max_seq_len,
+                        int32_t num_q_heads, float scale, void *out, void *workspace, size_t workspace_bytes,
+                        void *stream);
 
 /* Which partition kernel pa_decode runs (process wide; returns the previous
  * value; other values are ignored).  Both compute the same result within

@@ -22,10 +22,11 @@ lib = ctypes.CDLL(LIB_PATH)
 
 PA_OK, PA_EINVAL, PA_EUNSUPPORTED, PA_EWORKSPACE, PA_ECUDA = 0, -1, -2, -3, -4
 PA_DEVERR_SLOT, PA_DEVERR_BLOCK_ID, PA_DEVERR_SEQ_LEN, PA_DEVERR_COPY_PAIR, PA_DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+PA_DEVERR_QUERY_LOC = 32
 
 EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
             "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_static_ws", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
+            "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
             "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
@@ -64,6 +65,11 @@ lib.pa_decode.restype = ctypes.c_int
 lib.pa_decode_static_ws.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
                                     _P, _P]
 lib.pa_decode_static_ws.restype = ctypes.c_int
+lib.pa_attention_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, ctypes.POINTER(PaCache)]
+lib.pa_attention_workspace_bytes.restype = ctypes.c_size_t
+lib.pa_attention.argtypes = [_P, _i32, _P, _i32, _i32, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32,
+                             ctypes.c_float, _P, _P, ctypes.c_size_t, _P]
+lib.pa_attention.restype = ctypes.c_int
 PA_DECODE_STATIC_WS_BYTES = 8 * 1024 * 1024
 lib.pa_write_kv_fp8.argtypes = [_P, _P, _P, _i64, ctypes.POINTER(PaCacheFp8), _P]
 lib.pa_write_kv_fp8.restype = ctypes.c_int
@@ -276,6 +282,48 @@ def pa_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=Non
                          _dev(seq_lens, "seq_lens", torch.int32), S, int(max_seq_len), Hq,
                          float(scale), _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes,
                          _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+def pa_attention_workspace_bytes(num_reqs: int, num_tokens: int, max_query_len: int, num_q_heads: int,
+                                 max_seq_len: int, k_cache, v_cache) -> int:
+    cache = make_cache(k_cache, v_cache)
+    return int(lib.pa_attention_workspace_bytes(num_reqs, num_tokens, max_query_len, num_q_heads, max_seq_len,
+                                                ctypes.byref(cache)))
+
+
+def pa_attention(q, query_start_loc, k_cache, v_cache, block_tables, seq_lens, scale: float,
+                 max_query_len: int, out=None, max_seq_len: int | None = None, workspace=None,
+                 stream=None) -> torch.Tensor:
+    """Attention of several query rows per request (the last q_len tokens of
+    each, causal); returns ``out`` ([num_tokens, H_q, D] bf16).
+
+    ``query_start_loc`` is int32 [num_reqs + 1] on the device;
+    ``max_query_len`` and ``max_seq_len`` are host-side upper bounds (the
+    latter read from the device when omitted, a synchronisation)."""
+    cache = make_cache(k_cache, v_cache)
+    if q.dim() != 3 or q.shape[2] != k_cache.shape[3]:
+        raise ValueError("q must be [num_tokens, num_q_heads, head_dim]")
+    T, Hq, _ = q.shape
+    R = seq_lens.shape[0]
+    if query_start_loc.shape != (R + 1,) or block_tables.dim() != 2 or block_tables.shape[0] != R:
+        raise ValueError("query_start_loc must be [num_reqs + 1], block_tables [num_reqs, W]")
+    if max_seq_len is None:
+        max_seq_len = int(seq_lens.max().item()) if R else 0
+    if out is None:
+        out = torch.empty_like(q)
+    need = int(lib.pa_attention_workspace_bytes(R, T, int(max_query_len), Hq, int(max_seq_len),
+                                                ctypes.byref(cache)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace", torch.uint8) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib.pa_attention(_dev(q, "q", torch.bfloat16), T, _dev(query_start_loc, "query_start_loc", torch.int32),
+                            R, int(max_query_len), ctypes.byref(cache),
+                            _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+                            _dev(seq_lens, "seq_lens", torch.int32), int(max_seq_len), Hq, float(scale),
+                            _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes, _stream_ptr(stream)),
+           "pa_attention")
     return out
 
 

@@ -467,32 +467,36 @@ decode_partition_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
 }
 
-// One CTA per (query head, sequence); thread d owns output dim d.
+// One CTA per (query head, group of rows); thread d owns output dim d.  The
+// grid's y extent may be smaller than the row count (at most 65535), so each
+// CTA strides over rows.  A row's partition count follows from its length
+// (seq_lens[s]; for pa_attention the per-row visible length).
 __global__ void __launch_bounds__(kD) decode_merge_kernel(const DecodeParams p) {
     grid_dependency_wait();  // partials of the partition kernel are visible after this
     grid_launch_dependents();
     const int j = blockIdx.x;
-    const int s = blockIdx.y;
     const int d = threadIdx.x;
-    const int n = clamp_seq_len(p, s);
-    const int parts = n > 0 ? (n + p.part_tokens - 1) / p.part_tokens : 0;
-    const int64_t base = (static_cast<int64_t>(s) * p.num_q_heads + j) * p.num_parts;
-    float M = -INFINITY;
-    for (int i = 0; i < parts; ++i)
-        M = fmaxf(M, p.part_ml[base + i].x);
-    float L = 0.f, o = 0.f;
-    if (M != -INFINITY) {
-        for (int i = 0; i < parts; ++i) {
-            const float2 ml = p.part_ml[base + i];
-            if (ml.x == -INFINITY)
-                continue;
-            const float w = exp2f(ml.x - M);
-            L = fmaf(ml.y, w, L);
-            o = fmaf(p.part_acc[(base + i) * kD + d], w, o);
+    for (int s = blockIdx.y; s < p.num_seqs; s += gridDim.y) {
+        const int n = clamp_seq_len(p, s);
+        const int parts = n > 0 ? (n + p.part_tokens - 1) / p.part_tokens : 0;
+        const int64_t base = (static_cast<int64_t>(s) * p.num_q_heads + j) * p.num_parts;
+        float M = -INFINITY;
+        for (int i = 0; i < parts; ++i)
+            M = fmaxf(M, p.part_ml[base + i].x);
+        float L = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+            for (int i = 0; i < parts; ++i) {
+                const float2 ml = p.part_ml[base + i];
+                if (ml.x == -INFINITY)
+                    continue;
+                const float w = exp2f(ml.x - M);
+                L = fmaf(ml.y, w, L);
+                o = fmaf(p.part_acc[(base + i) * kD + d], w, o);
+            }
         }
+        const float r = L > 0.f ? o / L : 0.f;
+        p.out[(static_cast<int64_t>(s) * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(r);
     }
-    const float r = L > 0.f ? o / L : 0.f;
-    p.out[(static_cast<int64_t>(s) * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(r);
 }
 
 }  // namespace pa

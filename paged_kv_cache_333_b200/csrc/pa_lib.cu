@@ -13,6 +13,7 @@
 #include <mutex>
 #include <utility>
 
+#include "attend.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "decode_fp8.cuh"
@@ -241,6 +242,59 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
 }  // namespace
 
 namespace {
+// pa_attention's grid and scratch: column chunks per request, the split-K
+// partition (same heuristic as decode, over requests x chunks), and the
+// (m, l), acc and per-row length arrays when there is more than one
+// partition.
+struct AttendLayout {
+    int32_t chunks, part_tokens, num_parts;
+    size_t acc_offset, len_offset, total;
+};
+
+AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_query_len, int32_t num_q_heads,
+                           int32_t num_kv_heads, int32_t max_seq_len, int32_t block_size) {
+    AttendLayout a{};
+    const int64_t G = num_q_heads / num_kv_heads;
+    a.chunks = static_cast<int32_t>(std::max<int64_t>(1, (static_cast<int64_t>(max_query_len) * G +
+                                                          pa::kAttendCols - 1) / pa::kAttendCols));
+    const int64_t units = std::min<int64_t>(INT32_MAX, static_cast<int64_t>(num_reqs) * a.chunks);
+    a.part_tokens = choose_part_tokens(static_cast<int32_t>(units), num_kv_heads, max_seq_len, block_size, true);
+    a.num_parts = max_seq_len > 0 ? (max_seq_len + a.part_tokens - 1) / a.part_tokens : 1;
+    if (a.num_parts <= 1) {
+        a.num_parts = 1;
+        return a;
+    }
+    const size_t cells = static_cast<size_t>(num_tokens) * num_q_heads * a.num_parts;
+    a.acc_offset = static_cast<size_t>(round_up(static_cast<int64_t>(cells * sizeof(float2)), 256));
+    a.len_offset = static_cast<size_t>(round_up(static_cast<int64_t>(a.acc_offset + cells * pa::kD * sizeof(float)), 256));
+    a.total = a.len_offset + static_cast<size_t>(num_tokens) * sizeof(int32_t);
+    return a;
+}
+
+template <int G>
+int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap, int32_t num_kv_heads,
+                    cudaStream_t stream) {
+    static bool done[64] = {};
+    int rc = prepare_kernel(pa::attend_partition_kernel<G>, pa::kAttendSmemBytes, done);
+    if (rc)
+        return rc;
+    const dim3 grid(ap.d.num_parts, num_kv_heads, ap.d.num_seqs * ap.chunks);
+    cudaError_t e = launch_pdl(pa::attend_partition_kernel<G>, grid, dim3(pa::kAttendThreads), pa::kAttendSmemBytes,
+                               stream, tk, tv, ap);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "attend_partition_kernel launch");
+    if (ap.d.num_parts > 1) {
+        pa::DecodeParams md = ap.d;  // merge per query row, each with its visible length
+        md.seq_lens = ap.row_len;
+        md.num_seqs = ap.num_tokens;
+        e = launch_pdl(pa::decode_merge_kernel, dim3(md.num_q_heads, std::min(ap.num_tokens, 65535), 1),
+                       dim3(pa::kD), 0, stream, md);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "decode_merge_kernel launch");
+    }
+    return PA_OK;
+}
+
 pa_cache_t as_cache(const pa_cache_fp8_t *c) {
     pa_cache_t r{};
     r.k_cache = c->k_cache;
@@ -515,6 +569,89 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
     if (check_cache(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
         return 0;
     return workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size).total;
+}
+
+size_t pa_attention_workspace_bytes(int32_t num_reqs, int32_t num_tokens, int32_t max_query_len,
+                                    int32_t num_q_heads, int32_t max_seq_len, const pa_cache_t *cache) {
+    if (check_cache(cache) != PA_OK || num_reqs <= 0 || num_tokens <= 0 || max_query_len <= 0 ||
+        num_q_heads <= 0 || max_seq_len < 0 || num_q_heads % cache->num_kv_heads != 0)
+        return 0;
+    return attend_layout(num_reqs, num_tokens, max_query_len, num_q_heads, cache->num_kv_heads, max_seq_len,
+                         cache->block_size)
+        .total;
+}
+
+int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_loc, int32_t num_reqs,
+                 int32_t max_query_len, const pa_cache_t *cache, const int32_t *block_tables,
+                 int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t max_seq_len, int32_t num_q_heads,
+                 float scale, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_tokens < 0 || num_reqs < 0 || max_query_len < 0 || max_seq_len < 0 || num_q_heads <= 0 ||
+        max_blocks_per_seq < 0)
+        return PA_EINVAL;
+    if (num_reqs == 0 || num_tokens == 0 || max_query_len == 0)
+        return PA_OK;
+    if (!q || !query_start_loc || !block_tables || !seq_lens || !out)
+        return PA_EINVAL;
+    if (num_q_heads % cache->num_kv_heads != 0)
+        return PA_EINVAL;
+    const int32_t G = num_q_heads / cache->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return PA_EUNSUPPORTED;
+    if (!aligned16(q) || !aligned16(out))
+        return PA_EUNSUPPORTED;
+    if (!std::isfinite(scale))
+        return PA_EINVAL;
+    const AttendLayout a = attend_layout(num_reqs, num_tokens, max_query_len, num_q_heads, cache->num_kv_heads,
+                                         max_seq_len, cache->block_size);
+    if (static_cast<int64_t>(num_reqs) * a.chunks > 65535 || cache->num_kv_heads > 65535)
+        return PA_EUNSUPPORTED;
+    if (a.total > 0 && (workspace == nullptr || workspace_bytes < a.total))
+        return PA_EWORKSPACE;
+    if (a.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return PA_EUNSUPPORTED;
+
+    CUtensorMap tk, tv;
+    if ((rc = encode_cache_map(&tk, cache->k_cache, cache, true)) != PA_OK)
+        return rc;
+    if ((rc = encode_cache_map(&tv, cache->v_cache, cache, true)) != PA_OK)
+        return rc;
+
+    pa::AttendParams ap{};
+    pa::DecodeParams &p = ap.d;
+    p.q = static_cast<const uint4 *>(q);
+    p.k_cache = cache->k_cache;
+    p.v_cache = cache->v_cache;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.part_ml = a.total ? static_cast<float2 *>(workspace) : nullptr;
+    p.part_acc = a.total ? reinterpret_cast<float *>(static_cast<char *>(workspace) + a.acc_offset) : nullptr;
+    p.num_blocks = cache->num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_reqs;
+    p.max_seq_len = max_seq_len;
+    p.num_q_heads = num_q_heads;
+    p.block_size = cache->block_size;
+    p.part_tokens = a.part_tokens;
+    p.num_parts = a.num_parts;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);  // log2(e)
+    p.k_scale = 1.f;
+    p.v_scale = 1.f;
+    ap.query_start_loc = query_start_loc;
+    ap.row_len = a.total ? reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + a.len_offset) : nullptr;
+    ap.num_tokens = num_tokens;
+    ap.max_query_len = max_query_len;
+    ap.chunks = a.chunks;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (G) {
+    case 1: return launch_attend_g<1>(tk, tv, ap, cache->num_kv_heads, st);
+    case 2: return launch_attend_g<2>(tk, tv, ap, cache->num_kv_heads, st);
+    case 4: return launch_attend_g<4>(tk, tv, ap, cache->num_kv_heads, st);
+    default: return launch_attend_g<8>(tk, tv, ap, cache->num_kv_heads, st);
+    }
 }
 
 int32_t pa_decode_set_kernel(int32_t kind) {
