@@ -73,6 +73,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-op", action="store_true")
     ap.add_argument("--part-tokens", type=int, default=0, help="split-K partition size (0 = automatic)")
+    ap.add_argument("--queries", type=int, default=1,
+                    help="query rows per request: 1 = decode (pa_decode); Q > 1 = the last Q tokens of every "
+                         "request are its rows (speculative decode / prefill chunk; pa_attention)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="KV cache element type (fp8 = OCP E4M3 codes with per-tensor scales)")
     return ap.parse_args()
@@ -192,8 +195,9 @@ def profiled_traffic(config: str):
 
 
 # --------------------------------------------------------------------------- bytes
-def algorithmic_bytes(st) -> dict:
-    """Bytes the step must move, per layer."""
+def algorithmic_bytes(st, rows_per_seq: int = 1) -> dict:
+    """Bytes the step must move, per layer (rows_per_seq new K/V rows and
+    query rows per sequence)."""
     H, D, B = st.num_kv_heads, st.head_dim, st.block_size
     esz = 1 if st.kv_dtype == "fp8" else 2
     row = H * D * esz  # one token's K (or V) row in the cache
@@ -204,14 +208,14 @@ def algorithmic_bytes(st) -> dict:
         slots.append(st.block_tables_np[s, pos // B].astype(np.int64) * B + pos % B)
     uniq = np.unique(np.concatenate(slots)).size if slots else 0
     logical = int(st.seq_lens_np.sum())
-    T = st.slot_mapping_np.size
+    T = st.slot_mapping_np.size * rows_per_seq
     P = st.cow_pairs_np.shape[0]
     return {
         "decode_kv": uniq * row * 2,  # K and V, each unique slot once
         "decode_kv_logical": logical * row * 2,
         "write": T * H * D * 2 * 2 + T * row * 2,  # bf16 K and V rows read, cache rows written
         "copy": P * B * row * 2 * 2,  # K and V blocks read and written
-        "q_out": 2 * st.q.numel() * 2,
+        "q_out": 2 * st.q.numel() * rows_per_seq * 2,
         "table": int(sum(-(-int(n) // B) for n in st.seq_lens_np)) * 4,
     }
 
@@ -230,12 +234,37 @@ def run_ours(args, world, rank, local):
     fp8 = args.kv_dtype == "fp8"
     st = stage(w, dev, layers=args.layers, kv_dtype=args.kv_dtype)
     L = args.layers
-    nbytes = algorithmic_bytes(st)
+    Q = args.queries
+    if Q > 1 and (fp8 or st.cow_pairs.shape[0] > 0):
+        raise SystemExit("--queries > 1 is measured on bf16 caches of workloads without copy-on-write pairs")
+    S = len(st.ids)
+    # The step's inputs.  Decode: one new token per sequence.  --queries Q: the
+    # last Q tokens of every sequence are its query rows; their K/V rows are
+    # written again (same values, same slots) and pa_attention reads them.
+    inp = {"q": st.q, "k": st.k_new, "v": st.v_new, "slots": st.slot_mapping, "bt": st.block_tables,
+           "lens": st.seq_lens, "out": st.out, "ws": st.workspace}
+    if Q > 1:
+        lens_np = st.seq_lens_np.astype(np.int64)
+        if int(lens_np.min()) < Q:
+            raise SystemExit("--queries exceeds a sequence length")
+        pos = np.concatenate([np.arange(n - Q, n) for n in lens_np])
+        req = np.repeat(np.arange(S), Q)
+        slots_np = st.block_tables_np[req, pos // st.block_size].astype(np.int64) * st.block_size + pos % st.block_size
+        k_rows = np.concatenate([w.rows("k", sid, int(n) - Q, int(n)) for sid, n in zip(st.ids, lens_np)])
+        v_rows = np.concatenate([w.rows("v", sid, int(n) - Q, int(n)) for sid, n in zip(st.ids, lens_np)])
+        q_rows = synth.bf16_normal(synth.make_rng(900 + Q), (S * Q, st.num_q_heads, st.head_dim))
+        to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).to(dev).view(
+            torch.bfloat16)
+        inp.update(q=to_dev(q_rows), k=to_dev(k_rows), v=to_dev(v_rows), slots=torch.from_numpy(slots_np).to(dev),
+                   qsl=torch.arange(0, S * Q + 1, Q, dtype=torch.int32, device=dev))
+        inp["out"] = torch.empty_like(inp["q"])
+        need = pa.pa_attention_workspace_bytes(S, S * Q, Q, st.num_q_heads, st.max_seq_len, *st.caches[0])
+        inp["ws"] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
+    nbytes = algorithmic_bytes(st, rows_per_seq=Q)
     step_bytes = L * (nbytes["decode_kv"] + nbytes["write"] + nbytes["copy"])
     stream = torch.cuda.current_stream(dev)
-    S = len(st.ids)
     has_pairs = st.cow_pairs.shape[0] > 0
-    split = st.workspace is not None
+    split = inp["ws"] is not None
     launches_per_layer = 2 + (1 if split else 0) + (1 if has_pairs else 0)
 
     def write_op(k, v, slots, kc, vc):
@@ -244,8 +273,11 @@ def run_ours(args, world, rank, local):
         else:
             pa.pa_write_kv(k, v, slots, kc, vc)
 
-    def decode_op(q, kc, vc, bt, lens):
-        if fp8:
+    def decode_op(q, kc, vc, bt, lens, qsl=None):
+        if Q > 1:
+            pa.pa_attention(q, qsl, kc, vc, bt, lens, st.scale, max_query_len=Q, out=inp["out"],
+                            max_seq_len=st.max_seq_len, workspace=inp["ws"])
+        elif fp8:
             pa.pa_decode_fp8(q, kc, vc, st.k_scale, st.v_scale, bt, lens, st.scale, out=st.out,
                              max_seq_len=st.max_seq_len, workspace=st.workspace)
         else:
@@ -257,9 +289,9 @@ def run_ours(args, world, rank, local):
         if with_write:
             if has_pairs:
                 pa.pa_copy_blocks(kc, vc, st.cow_pairs)
-            write_op(st.k_new, st.v_new, st.slot_mapping, kc, vc)
+            write_op(inp["k"], inp["v"], inp["slots"], kc, vc)
         if with_decode:
-            decode_op(st.q, kc, vc, st.block_tables, st.seq_lens)
+            decode_op(inp["q"], kc, vc, inp["bt"], inp["lens"], inp.get("qsl"))
 
     def barrier():
         if world > 1:
@@ -315,7 +347,10 @@ def run_ours(args, world, rank, local):
 
     # ---- per-op times (graphs of one launch per layer) -------------------------
     per_op = {}
-    if not args.no_per_op and not fp8:
+    if Q > 1:
+        per_op["attention"] = {"us": round(dec_mean_ms * 1e3, 3), "GB/s": round(achieved, 2),
+                               "rows_per_s": round(S * Q / (dec_mean_ms * 1e-3), 1)}
+    if not args.no_per_op and not fp8 and Q == 1:
         row = st.num_kv_heads * st.head_dim * 2
         T = st.slot_mapping.numel()
         pos = st.seq_lens.to(torch.int64) - 1  # decode step: the new token is the last
@@ -351,14 +386,16 @@ def run_ours(args, world, rank, local):
     # ---- end to end: the same step from pinned host buffers -------------------
     e2e = None
     if not args.no_e2e:
-        q_h = st.q.cpu().pin_memory()
-        k_h, v_h = st.k_new.cpu().pin_memory(), st.v_new.cpu().pin_memory()
-        sm_h = st.slot_mapping.cpu().pin_memory()
-        bt_h, sl_h = st.block_tables.cpu().pin_memory(), st.seq_lens.cpu().pin_memory()
-        out_h = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-        q_d, k_d, v_d = torch.empty_like(st.q), torch.empty_like(st.k_new), torch.empty_like(st.v_new)
-        sm_d, bt_d, sl_d = (torch.empty_like(st.slot_mapping), torch.empty_like(st.block_tables),
-                            torch.empty_like(st.seq_lens))
+        q_h = inp["q"].cpu().pin_memory()
+        k_h, v_h = inp["k"].cpu().pin_memory(), inp["v"].cpu().pin_memory()
+        sm_h = inp["slots"].cpu().pin_memory()
+        bt_h, sl_h = inp["bt"].cpu().pin_memory(), inp["lens"].cpu().pin_memory()
+        qsl_h = inp["qsl"].cpu().pin_memory() if Q > 1 else None
+        out_h = torch.empty(inp["out"].shape, dtype=inp["out"].dtype).pin_memory()
+        q_d, k_d, v_d = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
+        sm_d, bt_d, sl_d = (torch.empty_like(inp["slots"]), torch.empty_like(inp["bt"]),
+                            torch.empty_like(inp["lens"]))
+        qsl_d = torch.empty_like(inp["qsl"]) if Q > 1 else None
         pairs_h = st.cow_pairs.cpu().pin_memory() if has_pairs else None
         pairs_d = torch.empty_like(st.cow_pairs) if has_pairs else None
 
@@ -366,6 +403,8 @@ def run_ours(args, world, rank, local):
             sm_d.copy_(sm_h, non_blocking=True)
             bt_d.copy_(bt_h, non_blocking=True)
             sl_d.copy_(sl_h, non_blocking=True)
+            if Q > 1:
+                qsl_d.copy_(qsl_h, non_blocking=True)
             if has_pairs:
                 pairs_d.copy_(pairs_h, non_blocking=True)
             for l in range(L):
@@ -376,8 +415,8 @@ def run_ours(args, world, rank, local):
                 if has_pairs:
                     pa.pa_copy_blocks(kc, vc, pairs_d)
                 write_op(k_d, v_d, sm_d, kc, vc)
-                decode_op(q_d, kc, vc, bt_d, sl_d)
-                out_h.copy_(st.out, non_blocking=True)
+                decode_op(q_d, kc, vc, bt_d, sl_d, qsl_d)
+                out_h.copy_(inp["out"], non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -386,6 +425,7 @@ def run_ours(args, world, rank, local):
             g_e2e.replay()
         e_ms = timed(g_e2e, K)
         h2d = (sm_h.numel() * 8 + bt_h.numel() * 4 + sl_h.numel() * 4 + (pairs_h.numel() * 8 if has_pairs else 0)
+               + (qsl_h.numel() * 4 if Q > 1 else 0)
                + L * (q_h.numel() + k_h.numel() + v_h.numel()) * 2)
         d2h = L * out_h.numel() * 2
         e2e = {"value": round(whole_job_rate(world, step_bytes, e_ms / K * 1e-3), 2), "unit": "GB/s",
@@ -408,7 +448,10 @@ def run_ours(args, world, rank, local):
         "dtype": "bf16 (fp8 e4m3 KV cache)" if fp8 else "bf16",
         "data": "synthetic (seeded N(0,1) bf16 K/V/q; seeded shuffled free list)",
         "config": {
-            "workload": WORKLOAD_TEXT.get(args.config, args.config),
+            "workload": WORKLOAD_TEXT.get(args.config, args.config)
+                        + (f"; {Q} query rows per sequence (its last {Q} tokens, causal), pa_attention" if Q > 1
+                           else ""),
+            "query_rows_per_seq": Q,
             "layers_per_step": L,
             "batch": S,
             "block_size": st.block_size,
@@ -425,23 +468,25 @@ def run_ours(args, world, rank, local):
         },
         "pct_of_peak": {"measured": round(100 * value / world / peak, 2),
                         "nominal_8tbs": round(100 * value / world / NOMINAL_HBM_GBS, 2)},
-        "decode_tokens_per_s_per_layer": round(world * S / (ms_step / L * 1e-3), 1),
+        "decode_tokens_per_s_per_layer": round(world * S * Q / (ms_step / L * 1e-3), 1),
         "per_op_bytes_per_layer": nbytes,
         "per_op": per_op,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(args.config) if not (args.part_tokens or fp8) else None,
-                     "kernel": ("pa_decode_fp8" if fp8 else "pa_decode") + " (partition kernel"
+                     "traffic": profiled_traffic(args.config) if not (args.part_tokens or fp8 or Q > 1) else None,
+                     "kernel": ("pa_attention" if Q > 1 else "pa_decode_fp8" if fp8 else "pa_decode")
+                               + " (partition kernel"
                                + (" + LSE merge)" if split else ")"),
                      "mean_launch_us": round(dec_mean_ms * 1e3, 3),
-                     "how": f"CUDA graph of {L} back-to-back pa_decode calls (one per layer cache), "
+                     "how": f"CUDA graph of {L} back-to-back {'pa_attention' if Q > 1 else 'pa_decode'} calls "
+                            f"(one per layer cache), "
                             f"{K} replays timed with CUDA events on the replay stream; mean per call",
                      "bytes_per_launch": nbytes["decode_kv"], "peak_source": peak_src},
         "e2e": e2e,
         "gpu_launches": K * L * launches_per_layer,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and Q == 1:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(result), flush=True)

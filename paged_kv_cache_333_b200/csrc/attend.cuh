@@ -8,17 +8,25 @@
 //
 // Work decomposition.  A "column" is one (query row, query head of the KV
 // group) pair of a request: column c = i * G + g.  One CTA handles one
-// (split-K partition, KV head, request, chunk of kAttendCols columns); each
-// of its kAttendWarps consumer warps owns 8 consecutive columns, which are
+// (split-K partition, KV head, request, chunk of 8W columns); each of its W
+// consumer warps owns 8 consecutive columns, which are
 // the N = 8 side of the same tensor-core tiles the decode kernel uses:
 //   S^T(16 tokens x 8 columns) = K(16x128) Q^T, mma.m16n8k16 bf16;
 //   O^T(128 x 8) += V^T(128x16) P^T, with P^T from movmatrix.trans.
-// Every consumer warp reads every K/V tile of the CTA's token range from the
-// shared-memory ring (the tile is fetched from HBM once per CTA and read by
-// up to four warps), so the ring's "empty" barrier counts all consumer warps
-// and a warp never runs a phase ahead of another.  The token range of a CTA
-// ends at the last position its last row may see; a warp skips the math
-// (still releasing the stage) for tiles past its own rows' range.
+// The chunk's columns form c = ceil(columns / 8) groups of 8 (c <= W).  With
+// fewer groups than warps, the s = W / c' warps of a group (c' = c rounded up
+// to a power of two, at most W) split its tiles round-robin, as the decode
+// kernel's two consumer warps do, and their (max, sum, acc) are merged
+// through shared memory at the end; with c' = W each warp owns one group and
+// reads every tile.  Every tile of the CTA's token range is fetched from HBM once
+// and read by one warp of each group, so the ring's "empty" barrier counts
+// c' arrivals per phase (set once the request's row count is known).  Tile t
+// is read by the warps with t % s == their split index and lives in stage
+// t % kStagesA; kStagesA is a multiple of every s, so a stage is only ever
+// read by the warps of one split index, each of which has read the stage's
+// previous phase before it waits on the next.  The token range of a CTA ends
+// at the last position its last row may see; a warp skips the math (still
+// releasing the stage) for tiles past its own rows' range.
 //
 // Masking is per column: token t is seen by column c iff t <= n - q_len +
 // c / G.  A column can see no token of a whole tile (or of a whole split-K
@@ -45,11 +53,30 @@
 
 namespace pa {
 
-constexpr int kAttendWarps = 4;                        // consumer warps per CTA
-constexpr int kAttendThreads = (kAttendWarps + 1) * 32;
-constexpr int kAttendCols = 8 * kAttendWarps;          // (row, head) columns per CTA
-constexpr int kStagesA = 8;
-constexpr int kAttendCtasPerSm = 2;
+// Two shapes of CTA, chosen per call from the columns a request has
+// (max_query_len * G): W = 2 consumer warps (16 columns, 96 threads, 4 CTAs
+// per SM, as the decode kernel) for up to 16 columns, W = 4 (32 columns, 160
+// threads, 2 CTAs per SM) above.  Four CTAs per SM keep a chat-sized batch
+// (512 CTAs) in one wave: measured on B200 (64 requests of 512..612
+// tokens, Llama-3-8B heads), 4 query rows per request took 32.6 us with
+// W = 2 against 57 us with W = 4, while 8 rows took 57 us with W = 4 against
+// 70 us with W = 2.  When each warp owns a whole group (no split) its
+// columns are written from registers; a shared-memory round trip there cost
+// 20-30% on B200.
+template <int W>
+struct AttendCfg;
+template <>
+struct AttendCfg<2> {
+    static constexpr int kStages = 6, kCtasPerSm = 4;
+};
+template <>
+struct AttendCfg<4> {
+    static constexpr int kStages = 8, kCtasPerSm = 2;
+};
+template <int W>
+constexpr int attend_threads() { return (W + 1) * 32; }
+template <int W>
+constexpr int attend_cols() { return 8 * W; }  // (row, head) columns per CTA
 
 struct AttendParams {
     DecodeParams d;  // q / out rows are query rows; seq_lens, block_tables per request (num_seqs = requests)
@@ -60,27 +87,37 @@ struct AttendParams {
     int32_t chunks;                  // column chunks per request
 };
 
+template <int W>
 struct AttendSmem {
-    uint16_t kv[kStagesA][4][kHalfElems];  // [stage][K lo, K hi, V lo, V hi][16 x 64], 128B-swizzled rows
-    uint64_t full[kStagesA];
-    uint64_t empty[kStagesA];
+    static constexpr int kStages = AttendCfg<W>::kStages;
+    static_assert(kStages % W == 0, "stages must be a multiple of every split");
+    uint16_t kv[kStages][4][kHalfElems];  // [stage][K lo, K hi, V lo, V hi][16 x 64], 128B-swizzled rows
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    float wm[W][8];  // per warp and column: running max, sum (for the split merge)
+    float wl[W][8];
     int32_t blocks[kMaxPartBlocksM];
 };
-constexpr size_t kAttendSmemBytes = sizeof(AttendSmem) + 1024;
+template <int W>
+constexpr size_t attend_smem_bytes() { return sizeof(AttendSmem<W>) + 1024; }
 
 __device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-template <int G>
-__global__ void __launch_bounds__(kAttendThreads, kAttendCtasPerSm)
+template <int G, int W>
+__global__ void __launch_bounds__(attend_threads<W>(), AttendCfg<W>::kCtasPerSm)
 attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const AttendParams ap) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     constexpr unsigned FULL = 0xffffffffu;
+    constexpr int kAttendWarps = W;
+    constexpr int kAttendCols = attend_cols<W>();
+    constexpr int kStagesA = AttendCfg<W>::kStages;
+    static_assert(sizeof(float) * W * 8 * kD <= sizeof(AttendSmem<W>::kv), "merge scratch must fit in the KV ring");
     const DecodeParams &p = ap.d;
     extern __shared__ uint8_t smem_raw[];
-    AttendSmem &sm = *reinterpret_cast<AttendSmem *>(
+    AttendSmem<W> &sm = *reinterpret_cast<AttendSmem<W> *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
     const int part = blockIdx.x;
@@ -92,13 +129,6 @@ attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const int B = p.block_size;
     const bool use_tma = B >= 8;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kStagesA; ++i) {
-            mbar_init(&sm.full[i], use_tma ? 1 : 32);
-            mbar_init(&sm.empty[i], kAttendWarps);
-        }
-        mbar_init_fence();
-    }
     if (use_tma && warp == kAttendWarps && lane == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -129,6 +159,18 @@ attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const int t_end = min(lim_max + 1, t_begin + p.part_tokens);
     const int num_tiles = (t_end - t_begin + kTile - 1) / kTile;
     const int Hkv = gridDim.y;
+    // column groups (rounded up to a power of two) and the tile split
+    const int groups_used = (last_col - col0) / 8 + 1;
+    const int ngroups = groups_used == 1 ? 1 : groups_used == 2 ? 2 : kAttendWarps;
+    const int split = kAttendWarps / ngroups;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStagesA; ++i) {
+            mbar_init(&sm.full[i], use_tma ? 1 : 32);
+            mbar_init(&sm.empty[i], ngroups);
+        }
+        mbar_init_fence();
+    }
 
     if (p.num_parts > 1 && part == 0 && h == 0 && warp == 0) {
         for (int i = col0 / G + lane; i <= last_col / G; i += 32)
@@ -211,7 +253,9 @@ attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     }
 
     // =================================================================== consumers
-    const int wcol0 = col0 + 8 * warp;         // this warp's first column
+    const int grp = warp % ngroups;            // this warp's column group
+    const int sub = warp / ngroups;            // its split index: tiles t with t % split == sub
+    const int wcol0 = col0 + 8 * grp;          // the group's first column
     const bool active = wcol0 <= last_col;
     // q as the B operand: column n = lane / 4 is row (wcol0 + n) / G, head
     // h*G + (wcol0 + n) % G; zero for columns past the chunk.
@@ -248,7 +292,7 @@ attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const int v_chk = (lane >> 3) & 1;
     const int tok0 = lane >> 2;  // C-fragment token rows tok0, tok0 + 8
 
-    for (int it = 0; it < num_tiles; ++it) {
+    for (int it = sub; it < num_tiles; it += split) {
         const int slot = it % kStagesA;
         bool ok = true;
         if (lane == 0)
@@ -335,38 +379,102 @@ attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     }
     if (threadIdx.x == 0)
         grid_launch_dependents();
-    if (!active)
-        return;
 #pragma unroll
     for (int off = 4; off <= 16; off <<= 1) {
         lA += __shfl_xor_sync(FULL, lA, off);
         lB += __shfl_xor_sync(FULL, lB, off);
     }
-    // ---- this lane's two columns: dims 16mt + tok0 (acc 0/1) and + 8 (acc 2/3)
+    // ---- one warp per group: its lane's two columns go straight out ---------
+    // (dims 16mt + tok0 in acc 0/1 and 16mt + tok0 + 8 in acc 2/3)
+    if (split == 1) {
+        if (!active)
+            return;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int col = u ? cB : cA;
-        if ((u ? limB : limA) < 0)
-            continue;
-        const float M = u ? mB : mA, L = u ? lB : lA;
-        const int64_t qrow = q0 + col / G;
-        const int j = h * G + col % G;
-        if (p.num_parts == 1) {
-            __nv_bfloat16 *o = p.out + (qrow * p.num_q_heads + j) * kD;
+        for (int u = 0; u < 2; ++u) {
+            const int col = u ? cB : cA;
+            if ((u ? limB : limA) < 0)
+                continue;
+            const float M = u ? mB : mA, L = u ? lB : lA;
+            const int64_t qrow = q0 + col / G;
+            const int j = h * G + col % G;
+            if (p.num_parts == 1) {
+                __nv_bfloat16 *o = p.out + (qrow * p.num_q_heads + j) * kD;
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                o[16 * mt + tok0] = __float2bfloat16_rn(L > 0.f ? acc[mt][u] / L : 0.f);
-                o[16 * mt + tok0 + 8] = __float2bfloat16_rn(L > 0.f ? acc[mt][2 + u] / L : 0.f);
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[16 * mt + tok0] = __float2bfloat16_rn(L > 0.f ? acc[mt][u] / L : 0.f);
+                    o[16 * mt + tok0 + 8] = __float2bfloat16_rn(L > 0.f ? acc[mt][2 + u] / L : 0.f);
+                }
+            } else {
+                const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + part;
+                float *o = p.part_acc + idx * kD;
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[16 * mt + tok0] = acc[mt][u];
+                    o[16 * mt + tok0 + 8] = acc[mt][2 + u];
+                }
+                if (tok0 == 0)
+                    p.part_ml[idx] = make_float2(M, L);
             }
-        } else {
+        }
+        return;
+    }
+    // ---- several warps per group: merge them through shared memory ---------
+    // Every tile has been waited for by some consumer warp before this
+    // barrier, so no copy into the ring is still in flight.
+    asm volatile("bar.sync 1, %0;" ::"n"(kAttendWarps * 32) : "memory");
+    float *wacc = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [warp][8 columns][D]
+    {
+        const int ca = 2 * (lane & 3);
+        float *wa = wacc + (warp * 8 + ca) * kD;
+        float *wb = wa + kD;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            const int d = mt * 16 + tok0;
+            wa[d] = acc[mt][0];
+            wb[d] = acc[mt][1];
+            wa[d + 8] = acc[mt][2];
+            wb[d + 8] = acc[mt][3];
+        }
+        if (lane < 4) {
+            sm.wm[warp][ca] = mA;
+            sm.wm[warp][ca + 1] = mB;
+            sm.wl[warp][ca] = lA;
+            sm.wl[warp][ca + 1] = lB;
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kAttendWarps * 32) : "memory");
+    // the W*32 consumer threads finish every column, thread t dims t, t + 32W, ...
+    for (int gi = 0; gi < ngroups; ++gi) {
+        for (int c = 0; c < 8; ++c) {
+            const int col = col0 + 8 * gi + c;
+            if (col > last_col)
+                break;
+            float M = -INFINITY;
+            for (int si = 0; si < split; ++si)
+                M = fmaxf(M, sm.wm[si * ngroups + gi][c]);
+            float L = 0.f;
+            for (int si = 0; si < split && M != -INFINITY; ++si) {
+                const float mw = sm.wm[si * ngroups + gi][c];
+                if (mw != -INFINITY)
+                    L = fmaf(sm.wl[si * ngroups + gi][c], exp2f(mw - M), L);
+            }
+            const int64_t qrow = q0 + col / G;
+            const int j = h * G + col % G;
             const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + part;
-            float *o = p.part_acc + idx * kD;
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                o[16 * mt + tok0] = acc[mt][u];
-                o[16 * mt + tok0 + 8] = acc[mt][2 + u];
+            for (int d = threadIdx.x; d < kD; d += kAttendWarps * 32) {
+                float o = 0.f;
+                for (int si = 0; si < split && M != -INFINITY; ++si) {
+                    const int w = si * ngroups + gi;
+                    const float mw = sm.wm[w][c];
+                    if (mw != -INFINITY)
+                        o = fmaf(wacc[(w * 8 + c) * kD + d], exp2f(mw - M), o);
+                }
+                if (p.num_parts == 1)
+                    p.out[(qrow * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(L > 0.f ? o / L : 0.f);
+                else
+                    p.part_acc[idx * kD + d] = o;
             }
-            if (tok0 == 0)
+            if (p.num_parts > 1 && threadIdx.x == 0)
                 p.part_ml[idx] = make_float2(M, L);
         }
     }

@@ -247,7 +247,7 @@ namespace {
 // (m, l), acc and per-row length arrays when there is more than one
 // partition.
 struct AttendLayout {
-    int32_t chunks, part_tokens, num_parts;
+    int32_t warps, chunks, part_tokens, num_parts;
     size_t acc_offset, len_offset, total;
 };
 
@@ -255,8 +255,10 @@ AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_que
                            int32_t num_kv_heads, int32_t max_seq_len, int32_t block_size) {
     AttendLayout a{};
     const int64_t G = num_q_heads / num_kv_heads;
-    a.chunks = static_cast<int32_t>(std::max<int64_t>(1, (static_cast<int64_t>(max_query_len) * G +
-                                                          pa::kAttendCols - 1) / pa::kAttendCols));
+    const int64_t cols = static_cast<int64_t>(max_query_len) * G;
+    a.warps = cols <= 16 ? 2 : 4;  // CTA shape: 16 columns x 4 CTAs/SM, or 32 columns x 2 CTAs/SM
+    const int64_t per_cta = 8 * a.warps;
+    a.chunks = static_cast<int32_t>(std::max<int64_t>(1, (cols + per_cta - 1) / per_cta));
     const int64_t units = std::min<int64_t>(INT32_MAX, static_cast<int64_t>(num_reqs) * a.chunks);
     a.part_tokens = choose_part_tokens(static_cast<int32_t>(units), num_kv_heads, max_seq_len, block_size, true);
     a.num_parts = max_seq_len > 0 ? (max_seq_len + a.part_tokens - 1) / a.part_tokens : 1;
@@ -271,15 +273,16 @@ AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_que
     return a;
 }
 
-template <int G>
+template <int G, int W>
 int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap, int32_t num_kv_heads,
                     cudaStream_t stream) {
     static bool done[64] = {};
-    int rc = prepare_kernel(pa::attend_partition_kernel<G>, pa::kAttendSmemBytes, done);
+    constexpr size_t smem = pa::attend_smem_bytes<W>();
+    int rc = prepare_kernel(pa::attend_partition_kernel<G, W>, smem, done);
     if (rc)
         return rc;
     const dim3 grid(ap.d.num_parts, num_kv_heads, ap.d.num_seqs * ap.chunks);
-    cudaError_t e = launch_pdl(pa::attend_partition_kernel<G>, grid, dim3(pa::kAttendThreads), pa::kAttendSmemBytes,
+    cudaError_t e = launch_pdl(pa::attend_partition_kernel<G, W>, grid, dim3(pa::attend_threads<W>()), smem,
                                stream, tk, tv, ap);
     if (e != cudaSuccess)
         return cuda_fail(e, "attend_partition_kernel launch");
@@ -646,11 +649,16 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     ap.max_query_len = max_query_len;
     ap.chunks = a.chunks;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool w2 = a.warps == 2;
     switch (G) {
-    case 1: return launch_attend_g<1>(tk, tv, ap, cache->num_kv_heads, st);
-    case 2: return launch_attend_g<2>(tk, tv, ap, cache->num_kv_heads, st);
-    case 4: return launch_attend_g<4>(tk, tv, ap, cache->num_kv_heads, st);
-    default: return launch_attend_g<8>(tk, tv, ap, cache->num_kv_heads, st);
+    case 1: return w2 ? launch_attend_g<1, 2>(tk, tv, ap, cache->num_kv_heads, st)
+                      : launch_attend_g<1, 4>(tk, tv, ap, cache->num_kv_heads, st);
+    case 2: return w2 ? launch_attend_g<2, 2>(tk, tv, ap, cache->num_kv_heads, st)
+                      : launch_attend_g<2, 4>(tk, tv, ap, cache->num_kv_heads, st);
+    case 4: return w2 ? launch_attend_g<4, 2>(tk, tv, ap, cache->num_kv_heads, st)
+                      : launch_attend_g<4, 4>(tk, tv, ap, cache->num_kv_heads, st);
+    default: return w2 ? launch_attend_g<8, 2>(tk, tv, ap, cache->num_kv_heads, st)
+                       : launch_attend_g<8, 4>(tk, tv, ap, cache->num_kv_heads, st);
     }
 }
 

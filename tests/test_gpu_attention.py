@@ -82,6 +82,20 @@ def test_attention_block_and_group_sizes(pa, G, B):
     assert pa.pa_get_device_error(clear=True) == 0
 
 
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("B", [1, 4, 16, 64])
+def test_attention_small_queries(pa, G, B):
+    """At most 16 (row, head) columns per request: the two-warp CTA shape,
+    whose warps split the tiles of a group when it has 8 columns or fewer."""
+    rmax = 16 // G
+    lens = [1, 9, 40, 130, 700, 3]
+    q_lens = [min(q, n) for q, n in zip([1, rmax, max(1, rmax - 1), rmax, max(1, rmax // 2), 0], lens)]
+    q, kc, vc, bt, qsl, n = _case(600 + 10 * G + B, lens, q_lens, B, 2 * G, 2)
+    ref = oracle.attention(q, kc, vc, bt, qsl, n, SCALE)
+    _check(_run(pa, q, kc, vc, bt, qsl, n), ref, f"G={G} B={B}")
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
 @pytest.mark.parametrize("part", [64, 256, 1024])
 def test_attention_split_k(pa, part):
     lens = [1, 300, 1000, 2049, 3000]
