@@ -137,6 +137,29 @@ def slot_mapping(table_rows, positions, block_size: int) -> np.ndarray:
     return out
 
 
+def map_to_kernel_blocks(block_table, blocks_per_alloc: int) -> np.ndarray:
+    """Block table of allocation blocks -> block table of kernel blocks, m =
+    blocks_per_alloc kernel blocks per allocation block ("PagedAttention:
+    fragmentation, blocks, block tables": section 2 "The block table", where
+    append_row maps the ids through map_to_kernel_blocks when the kernel's
+    block is smaller, and the decoupling passage: a 32-token allocation block
+    can feed a kernel that wants 16-token pages).  Storage is block-major, so
+    allocation block a owns the bytes of kernel blocks a*m .. a*m + m - 1:
+    entry i of a row becomes entries i*m .. i*m + m - 1.  Negative entries
+    (padding) become m entries of -1."""
+    t = np.asarray(block_table, dtype=np.int64)
+    rows, width = t.shape
+    out = np.full((rows, width * blocks_per_alloc), -1, dtype=np.int64)
+    for r in range(rows):
+        for i in range(width):
+            a = int(t[r, i])
+            if a < 0:
+                continue
+            for j in range(blocks_per_alloc):
+                out[r, i * blocks_per_alloc + j] = a * blocks_per_alloc + j
+    return out.astype(np.int32)
+
+
 # ----------------------------------------------------------------------------
 # Device operations, on host arrays
 # ----------------------------------------------------------------------------

@@ -85,3 +85,73 @@ def test_partial_hit_and_prefix(golden):
     assert p["prefix_tokens"] // p["block_size"] == p["shared_full_blocks"]
     assert p["prefix_tokens"] % p["block_size"] == p["partial_tail_tokens"]
     assert oracle.blocks_for(p["prefix_tokens"], p["block_size"]) == p["shared_full_blocks"] + 1
+
+
+# ---- kernel block != allocation block ("PagedAttention: fragmentation,
+# blocks, block tables", section 2 and the decoupling passage)
+
+def test_kernel_blocks_page_example():
+    """A 32-token allocation block feeding 16-token kernel pages: block 7
+    becomes kernel blocks 14 and 15; padding stays padding."""
+    got = oracle.map_to_kernel_blocks(np.array([[7, 0, -1]], np.int32), 2)
+    assert got.tolist() == [[14, 15, 0, 1, -1, -1]]
+
+
+def test_kernel_blocks_cover_the_same_bytes():
+    """Block-major storage: allocation block a of a pages of P_a bytes is the
+    byte range [a*P_a, (a+1)*P_a); the kernel blocks it maps to must tile
+    exactly that range with pages of P_a / m."""
+    gen = np.random.default_rng(3)
+    for m in (1, 2, 4, 8, 16):
+        page_a = 4096 * m
+        t = gen.integers(-1, 200, size=(5, 7)).astype(np.int32)
+        k = oracle.map_to_kernel_blocks(t, m)
+        page_k = page_a // m
+        for r in range(5):
+            for i in range(7):
+                ids = k[r, i * m:(i + 1) * m]
+                if t[r, i] < 0:
+                    assert np.all(ids == -1)
+                    continue
+                starts = ids.astype(np.int64) * page_k
+                assert starts[0] == int(t[r, i]) * page_a
+                assert np.all(np.diff(starts) == page_k)
+                assert starts[-1] + page_k == (int(t[r, i]) + 1) * page_a
+
+
+def test_kernel_blocks_preserve_every_slot():
+    """Every position maps to the same flat slot through (allocation table,
+    B_a) and through (kernel table, B_a / m)."""
+    gen = np.random.default_rng(4)
+    for m, B_a in ((2, 32), (4, 16), (8, 64), (16, 16)):
+        t = gen.permutation(300)[:40].reshape(4, 10).astype(np.int32)
+        k = oracle.map_to_kernel_blocks(t, m)
+        B_k = B_a // m
+        for r in range(4):
+            for pos in range(10 * B_a):
+                assert oracle.slot_of(t[r], pos, B_a) == oracle.slot_of(k[r], pos, B_k)
+
+
+def test_kernel_blocks_decode_invariance():
+    """Decode through the kernel table over the cache viewed with kernel
+    blocks equals decode through the allocation table (bit-identical)."""
+    import synth
+    gen = synth.make_rng(41)
+    H_q, H_kv, D, B_a, m = 8, 2, 128, 32, 4
+    NB = 16
+    lens = [1, 33, 100, 250]
+    kc = synth.bf16_normal(gen, (NB, B_a, H_kv, D))
+    vc = synth.bf16_normal(gen, (NB, B_a, H_kv, D))
+    t = np.full((4, 8), -1, np.int32)
+    perm = gen.permutation(NB)
+    used = 0
+    for r, n in enumerate(lens):
+        nb = oracle.blocks_for(n, B_a)
+        t[r, :nb] = perm[used:used + nb]
+        used += nb
+    q = synth.bf16_normal(gen, (4, H_q, D))
+    n = np.array(lens, np.int32)
+    a = oracle.decode(q, kc, vc, t, n, 0.088)
+    b = oracle.decode(q, kc.reshape(NB * m, B_a // m, H_kv, D), vc.reshape(NB * m, B_a // m, H_kv, D),
+                      oracle.map_to_kernel_blocks(t, m), n, 0.088)
+    assert np.array_equal(a, b)
