@@ -124,6 +124,30 @@ PA_API int pa_write_kv_positions(const void *k, const void *v, const int64_t *po
                                  void *stream);
 
 /*
+ * pa_map_to_kernel_blocks -- expand block tables of allocation blocks into
+ * block tables of smaller kernel blocks.
+ * Defined by: "PagedAttention: fragmentation, blocks, block tables",
+ * section 2 "The block table" (append_row maps the ids through
+ * map_to_kernel_blocks when the kernel's block is smaller) and the passage
+ * on decoupling the allocation block from the kernel's page (a 32-token
+ * allocation block can feed a kernel that wants 16-token pages).  The cache
+ * is block-major, so allocation block a (pages of block_size tokens) owns the
+ * bytes of kernel blocks a*m .. a*m + m - 1 (pages of block_size / m tokens),
+ * m = blocks_per_alloc: the same memory is a pa_cache_t with num_blocks * m
+ * blocks of block_size / m tokens, addressed by the expanded tables.
+ *   block_tables   [num_rows][width] int32 on the device; negative = padding.
+ *   kernel_tables  [num_rows][kernel_width] int32 on the device, kernel_width
+ *                  >= width * m: entry i*m + j of row r is tables[r][i]*m + j,
+ *                  -1 for padding and for the columns past width * m.
+ * Returns PA_EINVAL for blocks_per_alloc < 1 or kernel_width < width * m.  An
+ * id whose kernel ids exceed INT32_MAX is written as -1 and sets
+ * PA_DEVERR_BLOCK_ID.
+ */
+PA_API int pa_map_to_kernel_blocks(const int32_t *block_tables, int32_t num_rows, int32_t width,
+                                   int32_t blocks_per_alloc, int32_t *kernel_tables, int32_t kernel_width,
+                                   void *stream);
+
+/*
  * pa_copy_blocks -- copy-on-write block copies.
  * Defined by: "PagedAttention: fragmentation, blocks, block tables",
  * copy-on-write passage (a list of (src_block_id, dst_block_id) pairs runs

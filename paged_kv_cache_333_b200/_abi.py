@@ -26,7 +26,7 @@ PA_DEVERR_QUERY_LOC = 32
 
 EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
             "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
+            "pa_map_to_kernel_blocks", "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
             "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
@@ -65,6 +65,8 @@ lib.pa_decode.restype = ctypes.c_int
 lib.pa_decode_static_ws.argtypes = [_P, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
                                     _P, _P]
 lib.pa_decode_static_ws.restype = ctypes.c_int
+lib.pa_map_to_kernel_blocks.argtypes = [_P, _i32, _i32, _i32, _P, _i32, _P]
+lib.pa_map_to_kernel_blocks.restype = ctypes.c_int
 lib.pa_attention_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32, ctypes.POINTER(PaCache)]
 lib.pa_attention_workspace_bytes.restype = ctypes.c_size_t
 lib.pa_attention.argtypes = [_P, _i32, _P, _i32, _i32, ctypes.POINTER(PaCache), _P, _i32, _P, _i32, _i32,
@@ -282,6 +284,20 @@ def pa_decode(q, k_cache, v_cache, block_tables, seq_lens, scale: float, out=Non
                          _dev(seq_lens, "seq_lens", torch.int32), S, int(max_seq_len), Hq,
                          float(scale), _dev(out, "out", torch.bfloat16), ws_ptr, ws_bytes,
                          _stream_ptr(stream)), "pa_decode")
+    return out
+
+
+def pa_map_to_kernel_blocks(block_tables, blocks_per_alloc: int, out=None, stream=None) -> torch.Tensor:
+    """[R, W] int32 allocation-block table -> [R, W * m] kernel-block table
+    (entry i*m + j = table[i]*m + j; padding stays -1)."""
+    if block_tables.dim() != 2:
+        raise ValueError("block_tables must be [num_rows, width]")
+    R, W = block_tables.shape
+    if out is None:
+        out = torch.empty((R, W * blocks_per_alloc), dtype=torch.int32, device=block_tables.device)
+    _check(lib.pa_map_to_kernel_blocks(_dev(block_tables, "block_tables", torch.int32), R, W, int(blocks_per_alloc),
+                                       _dev(out, "out", torch.int32), out.shape[1], _stream_ptr(stream)),
+           "pa_map_to_kernel_blocks")
     return out
 
 

@@ -104,6 +104,37 @@ slot_mapping_kernel(const int64_t *__restrict__ positions, const int32_t *__rest
     slot_mapping[i] = slot;
 }
 
+// pa_map_to_kernel_blocks: one thread per output entry.  Allocation block a
+// of a block-major cache owns the bytes of kernel blocks a*m .. a*m + m - 1,
+// so entry i of a row becomes entries i*m .. i*m + m - 1 ("PagedAttention:
+// fragmentation, blocks, block tables", section 2 "The block table",
+// map_to_kernel_blocks; a 32-token allocation block feeding 16-token kernel
+// pages).  Padding (< 0) and the columns past width * m become -1; an id
+// whose kernel ids overflow int32 is flagged and written as -1.
+__global__ void __launch_bounds__(kSlotThreads)
+map_to_kernel_blocks_kernel(const int32_t *__restrict__ tables, int32_t num_rows, int32_t width,
+                            int32_t blocks_per_alloc, int32_t *__restrict__ kernel_tables, int32_t kernel_width) {
+    grid_launch_dependents();
+    grid_dependency_wait();
+    const int64_t e = static_cast<int64_t>(blockIdx.x) * kSlotThreads + threadIdx.x;
+    if (e >= static_cast<int64_t>(num_rows) * kernel_width)
+        return;
+    const int64_t r = e / kernel_width;
+    const int64_t c = e % kernel_width;
+    int32_t id = -1;
+    if (c < static_cast<int64_t>(width) * blocks_per_alloc) {
+        const int32_t a = tables[r * width + c / blocks_per_alloc];
+        if (a >= 0) {
+            const int64_t k = static_cast<int64_t>(a) * blocks_per_alloc + c % blocks_per_alloc;
+            if (k <= INT32_MAX)
+                id = static_cast<int32_t>(k);
+            else
+                flag_error(PA_DEVERR_BLOCK_ID);
+        }
+    }
+    kernel_tables[e] = id;
+}
+
 // pa_write_kv_positions: the KV write with the slot computed in-kernel from
 // the token's request row and position (one warp per (token, K|V)).
 __global__ void __launch_bounds__(kWriteThreads)

@@ -387,6 +387,25 @@ int pa_compute_slot_mapping(const int64_t *positions, const int32_t *req_indices
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "slot_mapping_kernel launch");
 }
 
+int pa_map_to_kernel_blocks(const int32_t *block_tables, int32_t num_rows, int32_t width, int32_t blocks_per_alloc,
+                            int32_t *kernel_tables, int32_t kernel_width, void *stream) {
+    if (num_rows < 0 || width < 0 || blocks_per_alloc < 1 || kernel_width < 0)
+        return PA_EINVAL;
+    if (static_cast<int64_t>(width) * blocks_per_alloc > kernel_width)
+        return PA_EINVAL;
+    if (num_rows == 0 || kernel_width == 0)
+        return PA_OK;
+    if (!kernel_tables || (width > 0 && !block_tables))
+        return PA_EINVAL;
+    const int64_t blocks = (static_cast<int64_t>(num_rows) * kernel_width + pa::kSlotThreads - 1) / pa::kSlotThreads;
+    if (blocks > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::map_to_kernel_blocks_kernel, dim3(static_cast<unsigned>(blocks)),
+                               dim3(pa::kSlotThreads), 0, static_cast<cudaStream_t>(stream), block_tables, num_rows,
+                               width, blocks_per_alloc, kernel_tables, kernel_width);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "map_to_kernel_blocks_kernel launch");
+}
+
 int pa_write_kv_positions(const void *k, const void *v, const int64_t *positions, const int32_t *req_indices,
                           int64_t num_tokens, const int32_t *block_tables, int32_t max_blocks_per_seq,
                           int32_t num_reqs, const pa_cache_t *cache, void *stream) {

@@ -130,3 +130,53 @@ def test_copy_blocks_for_all_layers_in_one_launch(pa):
     for (k, v), (dk, dv) in zip(host, dev):
         assert np.array_equal(_bits(dk), k) and np.array_equal(_bits(dv), v)
     assert pa.pa_get_device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("m", [1, 2, 4, 8, 16])
+def test_map_to_kernel_blocks_bit_exact(pa, m):
+    """Allocation-block tables expanded to kernel-block tables on the device
+    equal the oracle's definition, padding and the extra columns included."""
+    gen = synth.make_rng(60 + m)
+    t = gen.integers(-1, 5000, size=(33, 41)).astype(np.int32)
+    expect = np.full((33, 41 * m + 7), -1, np.int32)
+    expect[:, :41 * m] = oracle.map_to_kernel_blocks(t, m)
+    out = torch.full((33, 41 * m + 7), 12345, dtype=torch.int32, device="cuda")
+    pa.pa_map_to_kernel_blocks(torch.from_numpy(t).cuda(), m, out=out)
+    assert np.array_equal(out.cpu().numpy(), expect)
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("B_a,m", [(32, 2), (64, 4), (16, 16), (8, 8)])
+def test_kernel_block_view_decodes_and_maps_slots_the_same(pa, B_a, m):
+    """The cache allocated in B_a-token blocks, seen as kernel blocks of B_a/m
+    tokens through the expanded tables: the device slot mapping gives the same
+    slots and decode the same outputs (within the tolerance of the oracle)."""
+    gen, pool, lens, bt = _layout(70 + m, B_a, R=10, max_len=400)
+    NB, H_kv, H_q, D = pool.num_blocks, 2, 8, 128
+    kc = synth.bf16_normal(gen, (NB, B_a, H_kv, D))
+    vc = synth.bf16_normal(gen, (NB, B_a, H_kv, D))
+    q = synth.bf16_normal(gen, (len(lens), H_q, D))
+    n = lens.astype(np.int32)
+    dkc, dvc = _to_dev(kc), _to_dev(vc)
+    kt = pa.pa_map_to_kernel_blocks(torch.from_numpy(bt).cuda(), m)
+    # slots: every position of every request, through both tables
+    req = np.repeat(np.arange(len(lens)), lens).astype(np.int32)
+    pos = np.concatenate([np.arange(x) for x in lens]).astype(np.int64)
+    s_a = pa.pa_compute_slot_mapping(torch.from_numpy(pos).cuda(), torch.from_numpy(req).cuda(),
+                                     torch.from_numpy(bt).cuda(), B_a, NB)
+    s_k = pa.pa_compute_slot_mapping(torch.from_numpy(pos).cuda(), torch.from_numpy(req).cuda(), kt, B_a // m,
+                                     NB * m)
+    assert torch.equal(s_a, s_k)
+    # decode through both views of the same memory
+    ref = oracle.decode(q, kc, vc, bt, n, 0.088)
+    out_a = pa.pa_decode(_to_dev(q), dkc, dvc, torch.from_numpy(bt).cuda(), torch.from_numpy(n).cuda(), 0.088,
+                         max_seq_len=int(n.max()))
+    shape_k = (NB * m, B_a // m, H_kv, D)
+    out_k = pa.pa_decode(_to_dev(q), dkc.view(shape_k), dvc.view(shape_k), kt, torch.from_numpy(n).cuda(), 0.088,
+                         max_seq_len=int(n.max()))
+    torch.cuda.synchronize()
+    for out in (out_a, out_k):
+        got = synth.bf16_bits_to_f32(_bits(out)).astype(np.float64)
+        err = np.abs(got - ref)
+        assert err.max() <= 1.5e-2 and err.mean() <= 1e-3
+    assert pa.pa_get_device_error(clear=True) == 0
