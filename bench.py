@@ -167,12 +167,19 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- ncu traffic
-def profiled_traffic(config: str):
-    """DRAM bytes (read + write) per decode launch from the committed ncu
-    capture, if that capture was of this workload and of the kernel sources
-    as they are now; otherwise None."""
+PROFILE_FOR = {"bf16": "decode_mma_chat_full.md", "fp8": "decode_fp8_chat_full.md",
+               "rows4": "attention_q4_chat_full.md"}
+
+
+def profiled_traffic(config: str, kind: str = "bf16"):
+    """DRAM bytes (read + write) per launch of the timed kernel from the
+    committed ncu capture of that kernel (kind: "bf16" decode, "fp8" decode,
+    "rows4" = pa_attention with 4 rows per sequence), if that capture was of
+    this workload and of the kernel sources as they are now; otherwise None."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "decode_mma_chat_full.md")
+    if kind not in PROFILE_FOR:
+        return None
+    prof = os.path.join(ROOT, "profiles", PROFILE_FOR[kind])
     try:
         text = open(prof).read()
     except OSError:
@@ -473,7 +480,8 @@ def run_ours(args, world, rank, local):
         "per_op": per_op,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(args.config) if not (args.part_tokens or fp8 or Q > 1) else None,
+                     "traffic": None if args.part_tokens else profiled_traffic(
+                         args.config, "fp8" if fp8 else "bf16" if Q == 1 else f"rows{Q}"),
                      "kernel": ("pa_attention" if Q > 1 else "pa_decode_fp8" if fp8 else "pa_decode")
                                + " (partition kernel"
                                + (" + LSE merge)" if split else ")"),
