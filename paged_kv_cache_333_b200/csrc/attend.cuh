@@ -358,11 +358,11 @@ attend_partition_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
         const float sA = nA == -INFINITY ? 0.f : nA;  // a column that has seen nothing yet
         const float sB = nB == -INFINITY ? 0.f : nB;
-        const float aA = exp2f(mA - sA), aB = exp2f(mB - sB);
+        const float aA = exp2_approx(mA - sA), aB = exp2_approx(mB - sB);
         mA = nA;
         mB = nB;
-        const float p0 = exp2f(x0 - sA), p1 = exp2f(x1 - sB);
-        const float p2 = exp2f(x2 - sA), p3 = exp2f(x3 - sB);
+        const float p0 = exp2_approx(x0 - sA), p1 = exp2_approx(x1 - sB);
+        const float p2 = exp2_approx(x2 - sA), p3 = exp2_approx(x3 - sB);
         lA = fmaf(lA, aA, p0 + p2);
         lB = fmaf(lB, aB, p1 + p3);
         const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));  // tokens 0..7

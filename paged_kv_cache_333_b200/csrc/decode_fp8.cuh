@@ -81,19 +81,19 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 // Two f16 (low half first) -> two e4m3 codes (low byte first), nearest even,
-// saturating.
+// saturating: one cvt.rn.satfinite.e4m3x2.f16x2.
 __device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t h2) {
-    __half2_raw r;
-    r.x = static_cast<unsigned short>(h2 & 0xffffu);
-    r.y = static_cast<unsigned short>(h2 >> 16);
-    return __nv_cvt_halfraw2_to_fp8x2(r, __NV_SATFINITE, __NV_E4M3);
+    uint16_t c;
+    asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(c) : "r"(h2));
+    return c;
 }
 
-// Two e4m3 codes (low byte first) -> two f16 values (exact), low half first.
+// Two e4m3 codes (low byte first) -> two f16 values (exact), low half first:
+// one cvt.rn.f16x2.e4m3x2.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu),
-                                                     __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(two_codes & 0xffffu)));
+    return h2;
 }
 
 // f16x2 value v -> (hi, lo) e4m3x2 code pairs with v ~ hi + lo (hi nearest to
@@ -335,7 +335,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
             tB = fmaxf(tB, __shfl_xor_sync(FULL, tB, off));
         }
         const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
-        const float aA = exp2f(mA - nA), aB = exp2f(mB - nB);
+        const float aA = exp2_approx(mA - nA), aB = exp2_approx(mB - nB);
         mA = nA;
         mB = nB;
         // 256 * 2^(x - m): p in [0, 256], clear of the e4m3 subnormals
@@ -343,10 +343,10 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         float pr[2][4];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-            pr[mt][0] = exp2f(x[mt][0] - oA);
-            pr[mt][1] = exp2f(x[mt][1] - oB);
-            pr[mt][2] = exp2f(x[mt][2] - oA);
-            pr[mt][3] = exp2f(x[mt][3] - oB);
+            pr[mt][0] = exp2_approx(x[mt][0] - oA);
+            pr[mt][1] = exp2_approx(x[mt][1] - oB);
+            pr[mt][2] = exp2_approx(x[mt][2] - oA);
+            pr[mt][3] = exp2_approx(x[mt][3] - oB);
         }
         lA = fmaf(lA, aA, (pr[0][0] + pr[0][2]) + (pr[1][0] + pr[1][2]));
         lB = fmaf(lB, aB, (pr[0][1] + pr[0][3]) + (pr[1][1] + pr[1][3]));

@@ -299,11 +299,11 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             tB = fmaxf(tB, __shfl_xor_sync(FULL, tB, off));
         }
         const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
-        const float aA = exp2f(mA - nA), aB = exp2f(mB - nB);
+        const float aA = exp2_approx(mA - nA), aB = exp2_approx(mB - nB);
         mA = nA;
         mB = nB;
-        const float p0 = exp2f(x0 - nA), p1 = exp2f(x1 - nB);
-        const float p2 = exp2f(x2 - nA), p3 = exp2f(x3 - nB);
+        const float p0 = exp2_approx(x0 - nA), p1 = exp2_approx(x1 - nB);
+        const float p2 = exp2_approx(x2 - nA), p3 = exp2_approx(x3 - nB);
         lA = fmaf(lA, aA, p0 + p2);
         lB = fmaf(lB, aB, p1 + p3);
         const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));  // tokens 0..7

@@ -82,6 +82,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// 2^x by the SFU instruction ex2.approx.ftz (relative error about 2^-22;
+// -inf gives +0, results below 2^-126 flush to 0).  Used for the softmax
+// weights and rescale factors of the decode loops, whose arguments are <= 0
+// and whose results lie in [0, 1]: nothing there needs exp2f's subnormal
+// handling.
+__device__ __forceinline__ float exp2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *tm) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
