@@ -52,3 +52,45 @@ def test_host_side_validation_without_gpu():
     assert lib.pa_decode_workspace_bytes(64, 32, 0, ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))) == 0
     assert lib.pa_decode_workspace_bytes(8, 32, 32768, ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))) > 0
     assert lib.pa_status_str(-3) == b"workspace too small"
+
+
+def test_host_side_validation_of_the_widened_entry_points():
+    """pa_attention, the FP8 entry points and pa_map_to_kernel_blocks reject
+    bad arguments on the host (and treat empty work as a no-op) without
+    touching the device."""
+    from paged_kv_cache_333_b200._abi import (PA_EINVAL, PA_EUNSUPPORTED, PA_EWORKSPACE, PaCache, PaCacheFp8,
+                                              lib)
+    ok = PaCache(16, 16, 26785, 16, 8, 128)  # fake, aligned pointers: never dereferenced
+    c = ctypes.byref(ok)
+
+    def attn(q=16, T=4, qsl=16, R=1, maxq=4, cache=c, W=64, maxlen=600, Hq=32, scale=0.1, out=16, ws=None,
+             ws_bytes=0):
+        return lib.pa_attention(q, T, qsl, R, maxq, cache, 16, W, 16, maxlen, Hq, scale, out, ws, ws_bytes, None)
+
+    assert attn(T=-1) == PA_EINVAL
+    assert attn(R=0) == 0 and attn(T=0) == 0 and attn(maxq=0) == 0  # nothing to do
+    assert attn(q=None) == PA_EINVAL and attn(qsl=None) == PA_EINVAL
+    assert attn(Hq=30) == PA_EINVAL                       # not a multiple of the KV heads
+    assert attn(Hq=24) == PA_EUNSUPPORTED                 # group size 3
+    assert attn(q=18) == PA_EUNSUPPORTED                  # q not 16-byte aligned
+    assert attn(scale=float("nan")) == PA_EINVAL
+    assert attn(R=40000, T=40000, maxq=16) == PA_EUNSUPPORTED  # requests x column chunks > 65535
+    assert attn(maxlen=32768) == PA_EWORKSPACE            # split-K needs scratch, none given
+    assert lib.pa_attention_workspace_bytes(64, 256, 4, 32, 600, c) == 0
+    assert lib.pa_attention_workspace_bytes(8, 32, 4, 32, 32768, c) > 0
+    assert lib.pa_attention_workspace_bytes(8, 32, 4, 32, 32768, ctypes.byref(PaCache(16, 16, 8, 16, 8, 64))) == 0
+
+    f8 = PaCacheFp8(16, 16, 64, 16, 2, 128, 1.0 / 64, 1.0 / 64)
+    assert lib.pa_write_kv_fp8(16, 16, 16, -1, ctypes.byref(f8), None) == PA_EINVAL
+    assert lib.pa_write_kv_fp8(None, None, None, 0, ctypes.byref(f8), None) == 0
+    for k_scale in (0.0, -1.0, float("inf"), float("nan")):
+        bad = PaCacheFp8(16, 16, 64, 16, 2, 128, k_scale, 1.0)
+        assert lib.pa_write_kv_fp8(16, 16, 16, 1, ctypes.byref(bad), None) == PA_EINVAL
+    bad_d = PaCacheFp8(16, 16, 64, 16, 2, 96, 1.0, 1.0)
+    assert lib.pa_decode_fp8(16, ctypes.byref(bad_d), 16, 4, 16, 1, 64, 4, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
+    assert lib.pa_decode_fp8(16, ctypes.byref(f8), 16, 4, 16, 1, 64, 6, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
+
+    assert lib.pa_map_to_kernel_blocks(16, 4, 10, 0, 16, 40, None) == PA_EINVAL    # m < 1
+    assert lib.pa_map_to_kernel_blocks(16, 4, 10, 4, 16, 39, None) == PA_EINVAL    # too narrow
+    assert lib.pa_map_to_kernel_blocks(16, 4, 10, 4, None, 40, None) == PA_EINVAL
+    assert lib.pa_map_to_kernel_blocks(None, 0, 10, 4, None, 40, None) == 0       # no rows
