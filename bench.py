@@ -227,6 +227,37 @@ def algorithmic_bytes(st, rows_per_seq: int = 1) -> dict:
     }
 
 
+def host_pool_step_us(w, steps: int = 200) -> dict:
+    """Host time of the scheduler-side step (the block table and slot
+    mapping build) on the C++ pool: append one token to every sequence in one
+    call, take the queued copy pairs, and build the step's slot mapping,
+    block table and lengths.  Timed on a fresh pool laid out as the workload
+    (the timed device step uses its own)."""
+    from paged_kv_cache_333_b200.pool import BlockPool
+    sh = w.shape
+    pool = BlockPool(sh.num_blocks, sh.block_size, w.free_order, "shared")
+    w.ops(pool)
+    if w.suffix_ops is not None:
+        w.suffix_ops(pool)
+    pool.take_cow_pairs()
+    ids = np.asarray(w.seq_ids, dtype=np.int64)
+    width = max(pool.num_blocks_of(int(i)) for i in ids) + steps // sh.block_size + 2
+    done = 0
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        if not pool.append_batch(ids, 1):
+            break
+        pool.take_cow_pairs()
+        pool.step_slots(ids, 1)
+        pool.block_table(ids, width)
+        pool.seq_lens(ids)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"us": round(dt / max(done, 1) * 1e6, 2), "steps": done, "sequences": int(len(ids)),
+            "what": "append_batch (1 token per sequence) + copy pairs + slot mapping + block table + lengths, "
+                    "C++ pool through ctypes, one host thread"}
+
+
 # --------------------------------------------------------------------------- ours
 def run_ours(args, world, rank, local):
     import synth
@@ -354,7 +385,7 @@ def run_ours(args, world, rank, local):
     achieved = nbytes["decode_kv"] / (dec_mean_ms * 1e-3) / 1e9
 
     # ---- per-op times (graphs of one launch per layer) -------------------------
-    per_op = {}
+    per_op = {"pool_step_host": host_pool_step_us(w)}
     if Q > 1:
         per_op["attention"] = {"us": round(dec_mean_ms * 1e3, 3), "GB/s": round(achieved, 2),
                                "rows_per_s": round(S * Q / (dec_mean_ms * 1e-3), 1)}

@@ -75,6 +75,13 @@ int pa_pool_seq_create(pa_pool_t *pool, int64_t seq_id);
  * copy-on-write redirect of a shared partial tail (queued as a (src, dst)
  * pair).  PA_POOL_ENOSPACE leaves everything unchanged. */
 int pa_pool_append(pa_pool_t *pool, int64_t seq_id, int64_t n_tokens);
+/* One scheduler step: pa_pool_append(seq_ids[i], n_tokens) for every listed
+ * sequence, in order, as one call.  Either every append is done or, when the
+ * free queue cannot hold them all (copy-on-write redirects included, each
+ * decided with the earlier appends of the call applied), none is:
+ * PA_POOL_ENOSPACE and nothing changed.  PA_POOL_EINVAL for a sequence listed
+ * twice; PA_POOL_ENOSEQ for an unknown one (nothing changed). */
+int pa_pool_append_batch(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens);
 /* dst becomes a new sequence sharing every block of src (refcount + 1). */
 int pa_pool_fork(pa_pool_t *pool, int64_t src, int64_t dst);
 /* Drop the sequence; its blocks are freed in reverse order. */

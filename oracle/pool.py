@@ -34,6 +34,7 @@ check the product's C++ pool operation by operation:
 """
 from __future__ import annotations
 
+import copy
 from collections import deque
 
 from . import blocks_for, slot_of
@@ -116,6 +117,24 @@ class RefPool:
             table.extend(self._take(needed))
             self.tail_owned[seq_id] = True
         self.lens[seq_id] = length + n
+        return True
+
+    def append_batch(self, seq_ids, n: int) -> bool:
+        """One scheduler step: append(seq, n) for every listed sequence in
+        order, all or nothing (a failed call leaves the state unchanged,
+        "PagedAttention: fragmentation, blocks, block tables", the allocator
+        invariants).  Written as snapshot, sequential appends, restore."""
+        if len(set(seq_ids)) != len(seq_ids):
+            raise ValueError("a sequence listed twice")
+        for sid in seq_ids:
+            if sid not in self.tables:
+                raise KeyError(sid)
+        saved = copy.deepcopy(self.__dict__)
+        for sid in seq_ids:
+            if not self.append(sid, n):
+                self.__dict__.clear()
+                self.__dict__.update(saved)
+                return False
         return True
 
     def fork(self, src: int, dst: int) -> None:

@@ -174,6 +174,46 @@ int pa_pool_append(pa_pool_t *pool, int64_t seq_id, int64_t n_tokens) {
     return PA_POOL_OK;
 }
 
+int pa_pool_append_batch(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens) {
+    if (!pool || n_tokens < 0 || num_seqs < 0 || (num_seqs > 0 && !seq_ids))
+        return PA_POOL_EINVAL;
+    // Dry run in call order: the blocks each append needs, with the copy-on-
+    // write decisions of the earlier ones applied (a copy takes the sequence
+    // off its shared tail, which a later sharer may then own alone).
+    const int64_t B = pool->block_size;
+    std::unordered_map<int32_t, int32_t> dropped;  // owner refs earlier copies removed
+    std::unordered_map<int64_t, bool> seen;
+    int64_t total = 0;
+    for (int32_t i = 0; i < num_seqs; ++i) {
+        if (!seen.emplace(seq_ids[i], true).second)
+            return PA_POOL_EINVAL;  // a sequence listed twice
+        auto it = pool->seqs.find(seq_ids[i]);
+        if (it == pool->seqs.end())
+            return PA_POOL_ENOSEQ;
+        const Seq &s = it->second;
+        const int64_t needed = cdiv(s.len + n_tokens, B) - static_cast<int64_t>(s.blocks.size());
+        const bool partial = !s.blocks.empty() && s.len % B != 0 && n_tokens > 0;
+        bool cow;
+        if (pool->rule == PA_COW_SHARED) {
+            const int32_t tail = partial ? s.blocks.back() : -1;
+            cow = partial && pool->ref[static_cast<size_t>(tail)] - dropped[tail] > 1;
+            if (cow)
+                dropped[tail] += 1;
+        } else {
+            cow = partial && !s.tail_owned;
+        }
+        total += needed + (cow ? 1 : 0);
+    }
+    if (total > pool->free_q.size())
+        return PA_POOL_ENOSPACE;
+    for (int32_t i = 0; i < num_seqs; ++i) {
+        const int rc = pa_pool_append(pool, seq_ids[i], n_tokens);
+        if (rc != PA_POOL_OK)
+            return rc;  // not reached: the dry run counted every block
+    }
+    return PA_POOL_OK;
+}
+
 int pa_pool_fork(pa_pool_t *pool, int64_t src, int64_t dst) {
     if (!pool)
         return PA_POOL_EINVAL;

@@ -16,7 +16,8 @@ PA_POOL_OK, PA_POOL_EINVAL, PA_POOL_ENOSPACE, PA_POOL_ENOSEQ, PA_POOL_EEXIST, PA
     PA_POOL_ERANGE = 0, -1, -2, -3, -4, -5, -6
 PA_COW_SHARED, PA_COW_INHERITED = 0, 1
 
-EXPORTED = ("pa_pool_create", "pa_pool_destroy", "pa_pool_seq_create", "pa_pool_append", "pa_pool_fork",
+EXPORTED = ("pa_pool_create", "pa_pool_destroy", "pa_pool_seq_create", "pa_pool_append", "pa_pool_append_batch",
+            "pa_pool_fork",
             "pa_pool_release", "pa_pool_num_pending_copies", "pa_pool_take_copies", "pa_pool_num_blocks",
             "pa_pool_block_size", "pa_pool_num_free", "pa_pool_seq_len", "pa_pool_seq_num_blocks",
             "pa_pool_refcount", "pa_pool_pins", "pa_pool_free_list", "pa_pool_block_table", "pa_pool_seq_lens",
@@ -30,6 +31,7 @@ lib.pa_pool_destroy.restype = None
 for _name, _args, _res in [
     ("pa_pool_seq_create", [_P, _i64], ctypes.c_int),
     ("pa_pool_append", [_P, _i64, _i64], ctypes.c_int),
+    ("pa_pool_append_batch", [_P, _P, _i32, _i64], ctypes.c_int),
     ("pa_pool_fork", [_P, _i64, _i64], ctypes.c_int),
     ("pa_pool_release", [_P, _i64], ctypes.c_int),
     ("pa_pool_num_pending_copies", [_P], _i64),
@@ -104,6 +106,16 @@ class BlockPool:
         if rc == PA_POOL_ENOSPACE:
             return False
         _ok(rc, "append")
+        return True
+
+    def append_batch(self, seq_ids, n: int) -> bool:
+        """append(seq, n) for every listed sequence, all or nothing; False
+        (and nothing changed) when the pool cannot hold them all."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        rc = lib.pa_pool_append_batch(self._h, _ptr(ids), len(ids), n)
+        if rc == PA_POOL_ENOSPACE:
+            return False
+        _ok(rc, "append_batch")
         return True
 
     def fork(self, src: int, dst: int) -> None:

@@ -266,3 +266,74 @@ def test_step_slots_and_padding():
     bt = pool.block_table([1, 2], 3, pad=-7)
     assert bt[0, 2] == -7 and bt[1, 2] == -7
     assert oracle.slot_of(bt[1], 7, 4) == sl[1]
+
+
+def _snapshot(p, ids, NB=40):
+    return (np.asarray(p.block_table(ids, 64)).tolist(), [p.seq_len(i) for i in ids], list(p.free_list()),
+            [p.refcount(b) for b in range(NB)], [p.pins(b) for b in range(NB)])
+
+
+@pytest.mark.parametrize("rule", ["shared", "inherited"])
+def test_append_batch_matches_sequential_appends(rule):
+    """One call per scheduler step: the C++ batch equals the oracle pool's
+    sequential appends, including copy-on-write of a tail several forks
+    share (the first sharer copies, the last one may own the tail alone)."""
+    for seed in range(8):
+        gen = np.random.default_rng(seed)
+        NB, B = 40, 4
+        order = gen.permutation(NB).astype(np.int32)
+        c, r = BlockPool(NB, B, order, rule), RefPool(NB, B, order, rule)
+        for p in (c, r):
+            p.create(0)
+            assert p.append(0, 6)  # partial tail (6 % 4)
+            for k in (1, 2, 3):
+                p.fork(0, k)
+        ids = [3, 0, 2, 1]
+        for step in range(6):
+            n = int(gen.integers(0, 5))
+            ok_c, ok_r = c.append_batch(ids, n), r.append_batch(ids, n)
+            assert ok_c == ok_r
+            assert _snapshot(c, ids) == _snapshot(r, ids)
+            c.check()
+            r.check()
+            assert np.asarray(c.take_cow_pairs()).reshape(-1, 2).tolist() == \
+                np.asarray(r.take_cow_pairs()).reshape(-1, 2).tolist()
+
+
+def test_append_batch_is_all_or_nothing():
+    """When the pool cannot hold every append of the batch, nothing changes
+    (and a batch that fits after a smaller step succeeds)."""
+    for cls in (BlockPool, RefPool):
+        p = cls(10, 4, np.arange(10, dtype=np.int32))
+        for k in range(3):
+            p.create(k)
+            assert p.append(k, 8)  # 2 blocks each -> 6 used, 4 free
+        ids = [0, 1, 2]
+        before = _snapshot(p, ids, 10)
+        assert not p.append_batch(ids, 8)  # needs 6 blocks
+        assert _snapshot(p, ids, 10) == before
+        assert p.append_batch(ids, 4)  # needs 3 blocks
+        p.check()
+        with pytest.raises(Exception):
+            p.append_batch([0, 0], 1)  # listed twice
+        with pytest.raises(Exception):
+            p.append_batch([0, 99], 1)  # unknown sequence
+        assert _snapshot(p, ids, 10)[1] == [12, 12, 12]
+
+
+@pytest.mark.parametrize("rule", ["shared", "inherited"])
+def test_append_batch_counts_copies_exactly_at_capacity(rule):
+    """Four sequences share a partial tail and the pool has room for exactly
+    three copies: under either rule three sharers copy and one writes in
+    place, so the batch fits (counting a copy for every sharer would refuse)."""
+    for cls in (BlockPool, RefPool):
+        p = cls(5, 4, np.arange(5, dtype=np.int32), rule)
+        p.create(0)
+        assert p.append(0, 6)  # blocks 0, 1; tail partial
+        for k in (1, 2, 3):
+            p.fork(0, k)
+        assert p.num_free() == 3
+        assert p.append_batch([3, 0, 2, 1], 1)
+        assert p.num_free() == 0
+        assert len(np.asarray(p.take_cow_pairs()).reshape(-1, 2)) == 3
+        p.check()
