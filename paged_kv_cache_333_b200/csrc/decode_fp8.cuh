@@ -50,18 +50,29 @@ namespace pa {
 
 constexpr int kTileF = 32;
 constexpr int kStagesF = 6;
+// Consumer warps per CTA, CW = 2 or 3, chosen per call: the FP8 consumer
+// does twice the tensor and byte-permute work per byte of the bf16 one.
+// When the grid fits in one wave (at most 4 CTAs per SM) every CTA is
+// resident from the start and two consumer warps at up to 168 registers do
+// best (chat on B200: 21.2 us against 22.8 us with three); when it takes
+// several waves, CTAs finish faster with three consumer warps at 128
+// registers (B=16 and B=1 sweeps on B200: 15% and 21% more bandwidth).
+template <int CW>
+constexpr int fp8_threads() { return (CW + 1) * 32; }
+constexpr int kFp8CtasPerSm = 4;
+constexpr int kMaxConsumerWarpsF = 3;
 constexpr int kTileBytesF = kTileF * kD;  // 32 tokens x 128 one-byte codes
-static_assert(kStagesF % kConsumerWarpsM == 0, "stages must be a multiple of the consumer warps");
+static_assert(kStagesF % 2 == 0 && kStagesF % 3 == 0, "stages must be a multiple of the consumer warps");
 
 struct DecodeSmemF {
     uint8_t kv[kStagesF][2][kTileBytesF];  // [stage][K, V][32 x 128], 128B-swizzled rows
     uint64_t full[kStagesF];
     uint64_t empty[kStagesF];
-    float wm[kConsumerWarpsM][8];
-    float wl[kConsumerWarpsM][8];
+    float wm[kMaxConsumerWarpsF][8];
+    float wl[kMaxConsumerWarpsF][8];
     int32_t blocks[kMaxPartBlocksM];
 };
-static_assert(sizeof(float) * kConsumerWarpsM * 8 * kD <= sizeof(uint8_t) * kStagesF * 2 * kTileBytesF,
+static_assert(sizeof(float) * kMaxConsumerWarpsF * 8 * kD <= sizeof(uint8_t) * kStagesF * 2 * kTileBytesF,
               "merge scratch must fit in the KV ring");
 constexpr size_t kDecodeSmemBytesF = sizeof(DecodeSmemF) + 1024;
 
@@ -122,11 +133,13 @@ __device__ __forceinline__ void split_f32x4(const float (&x)[4], uint32_t &hi, u
     lo = lc[0] | (lc[1] << 16);
 }
 
-template <int G>
-__global__ void __launch_bounds__(kDecodeThreadsM, kMmaCtasPerSm)
+template <int G, int CW>
+__global__ void __launch_bounds__(fp8_threads<CW>(), kFp8CtasPerSm)
 decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+    static_assert(CW == 2 || CW == 3, "consumer warps");
+    constexpr int kConsumerWarpsF = CW;
     constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ uint8_t smem_raw[];
     DecodeSmemF &sm = *reinterpret_cast<DecodeSmemF *>(
@@ -147,7 +160,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         mbar_init_fence();
     }
-    if (use_tma && warp == kConsumerWarpsM && lane == 0) {
+    if (use_tma && warp == kConsumerWarpsF && lane == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -157,7 +170,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int first_blk = t_begin / B;
     const int32_t *row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + first_blk;
     int32_t first_ids = 0;
-    if (warp == kConsumerWarpsM && lane < p.max_blocks_per_seq - first_blk)
+    if (warp == kConsumerWarpsF && lane < p.max_blocks_per_seq - first_blk)
         first_ids = __ldg(row + lane);
     const int n = clamp_seq_len(p, s);
     if (part > 0 && t_begin >= n)
@@ -165,7 +178,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int t_end = min(n, t_begin + p.part_tokens);
     const int num_tiles = t_end > t_begin ? (t_end - t_begin + kTileF - 1) / kTileF : 0;
     const int Hkv = gridDim.y;
-    if (warp == kConsumerWarpsM && num_tiles > 0) {
+    if (warp == kConsumerWarpsF && num_tiles > 0) {
         const int nblk = (t_end - 1) / B - first_blk + 1;
         for (int i = lane; i < nblk; i += 32) {
             int32_t b = i < 32 ? first_ids : __ldg(row + i);
@@ -179,7 +192,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     __syncthreads();
 
     // =================================================================== producer
-    if (warp == kConsumerWarpsM) {
+    if (warp == kConsumerWarpsF) {
         if (num_tiles == 0 || !use_tma)
             return;
         const uint64_t pol = l2_evict_first_policy();
@@ -307,13 +320,14 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                 mma_16832_e4m3(slo[mt], kf, ql[kk][0], ql[kk][1]);
             }
         }
-        // V^T fragments: matrix i of load c = tokens 8i..8i+7, dims 16c..16c+15;
-        // the stage is released once they are in registers.
-        uint32_t vf[8][4];
+        // V^T fragments, in two halves of four 16-dim tiles (fewer live
+        // registers): matrix i of load c = tokens 8i..8i+7, dims 16c..16c+15.
+        // The first half is loaded now, the second after the first half's
+        // MMAs; the stage is released once both are in registers.
+        uint32_t vf[4][4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < 4; ++c)
             ldmatrix_x4_trans(vf[c], vb + swz(lane, c));
-        loaded();
         // ---- online softmax (log2 domain) -------------------------------
         float x[2][4];
 #pragma unroll
@@ -367,24 +381,34 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         // running sum in fp32 outside the MMA, so the sum over thousands of
         // tiles does not depend on how the FP8 MMA rounds its accumulator.
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint32_t a[4] = {__byte_perm(vf[c][0], vf[c][1], 0x6420),   // dim 2g, tokens 2t,2t+1,8+2t,9+2t
-                                   __byte_perm(vf[c][0], vf[c][1], 0x7531),   // dim 2g+1
-                                   __byte_perm(vf[c][2], vf[c][3], 0x6420),   // dim 2g, tokens +16
-                                   __byte_perm(vf[c][2], vf[c][3], 0x7531)};  // dim 2g+1, tokens +16
-            float o[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_16832_e4m3(o, a, pbh0, pbh1);
-            mma_16832_e4m3(o, a, pbl0, pbl1);
-            acc[c][0] = fmaf(acc[c][0], aA, o[0]);
-            acc[c][1] = fmaf(acc[c][1], aB, o[1]);
-            acc[c][2] = fmaf(acc[c][2], aA, o[2]);
-            acc[c][3] = fmaf(acc[c][3], aB, o[3]);
+        for (int half = 0; half < 2; ++half) {
+            if (half == 1) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    ldmatrix_x4_trans(vf[c], vb + swz(lane, 4 + c));
+                loaded();
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int c = 4 * half + c4;
+                const uint32_t a[4] = {__byte_perm(vf[c4][0], vf[c4][1], 0x6420),   // dim 2g, tokens 2t,2t+1,8+2t,9+2t
+                                       __byte_perm(vf[c4][0], vf[c4][1], 0x7531),   // dim 2g+1
+                                       __byte_perm(vf[c4][2], vf[c4][3], 0x6420),   // dim 2g, tokens +16
+                                       __byte_perm(vf[c4][2], vf[c4][3], 0x7531)};  // dim 2g+1, tokens +16
+                float o[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_16832_e4m3(o, a, pbh0, pbh1);
+                mma_16832_e4m3(o, a, pbl0, pbl1);
+                acc[c][0] = fmaf(acc[c][0], aA, o[0]);
+                acc[c][1] = fmaf(acc[c][1], aB, o[1]);
+                acc[c][2] = fmaf(acc[c][2], aA, o[2]);
+                acc[c][3] = fmaf(acc[c][3], aB, o[3]);
+            }
         }
     };
     auto tile_tokens = [&](int it) { return min(kTileF, t_end - (t_begin + it * kTileF)); };
 
     if (use_tma) {
-        for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
+        for (int it = warp; it < num_tiles; it += kConsumerWarpsF) {
             const int slot = it % kStagesF;
             bool ok = true;
             if (lane == 0)
@@ -403,7 +427,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     } else {
         // Blocks of 1, 2 or 4 tokens: each consumer warp gathers its own tiles
         // (lane = token parity, tensor, 16-byte chunk of the 128-byte row).
-        constexpr int kAhead = kStagesF / kConsumerWarpsM;
+        constexpr int kAhead = kStagesF / kConsumerWarpsF;
         const int par = lane >> 4, tensor = (lane >> 3) & 1, ch = lane & 7;
         const uint8_t *cache = static_cast<const uint8_t *>(tensor ? p.v_cache : p.k_cache);
         auto gather = [&](int it) {
@@ -428,13 +452,13 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         };
 #pragma unroll
         for (int k = 0; k < kAhead; ++k)
-            gather(warp + k * kConsumerWarpsM);
-        for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
+            gather(warp + k * kConsumerWarpsF);
+        for (int it = warp; it < num_tiles; it += kConsumerWarpsF) {
             asm volatile("cp.async.wait_group %0;" ::"n"(kAhead - 1) : "memory");
             __syncwarp();
             consume(it % kStagesF, tile_tokens(it), [] {});
             __syncwarp();
-            gather(it + kAhead * kConsumerWarpsM);
+            gather(it + kAhead * kConsumerWarpsF);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     }
@@ -447,7 +471,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     }
     if (threadIdx.x == 0)
         grid_launch_dependents();
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsF * 32) : "memory");
     float *wacc = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [warp][8 heads][D]
     {
         const int hA = t4 * 2;
@@ -468,31 +492,40 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
             sm.wl[warp][hA + 1] = lB;
         }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsF * 32) : "memory");
 #pragma unroll
     for (int gq = 0; gq < G; ++gq) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarpsM; ++w)
+        for (int w = 0; w < kConsumerWarpsF; ++w)
             M = fmaxf(M, sm.wm[w][gq]);
-        float L = 0.f, o[2] = {0.f, 0.f};
+        // the consumer threads finish dims t, t + 32 * kConsumerWarpsF, ...
+        constexpr int kStride = kConsumerWarpsF * 32;
+        constexpr int kPer = (kD + kStride - 1) / kStride;
+        float L = 0.f, o[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u)
+            o[u] = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kConsumerWarpsM; ++w) {
+            for (int w = 0; w < kConsumerWarpsF; ++w) {
                 const float mw = sm.wm[w][gq];
                 if (mw == -INFINITY)
                     continue;
                 const float sc = exp2f(mw - M);
                 L = fmaf(sm.wl[w][gq], sc, L);
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    o[u] = fmaf(wacc[(w * 8 + gq) * kD + threadIdx.x + 64 * u], sc, o[u]);
+                for (int u = 0; u < kPer; ++u)
+                    if (threadIdx.x + kStride * u < kD)
+                        o[u] = fmaf(wacc[(w * 8 + gq) * kD + threadIdx.x + kStride * u], sc, o[u]);
             }
         }
         const int jq = h * G + gq;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int d = threadIdx.x + 64 * u;
+        for (int u = 0; u < kPer; ++u) {
+            const int d = threadIdx.x + kStride * u;
+            if (d >= kD)
+                break;
             const float ov = o[u] * p.v_scale;
             if (p.num_parts == 1) {
                 const float r = L > 0.f ? ov / L : 0.f;

@@ -321,17 +321,31 @@ int check_cache_fp8(const pa_cache_fp8_t *c) {
     return PA_OK;
 }
 
+template <int G, int CW>
+int launch_decode_fp8_cw(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
+                         int32_t num_kv_heads, cudaStream_t stream) {
+    static bool done[64] = {};
+    int rc = prepare_kernel(pa::decode_partition_fp8_kernel<G, CW>, pa::kDecodeSmemBytesF, done);
+    if (rc)
+        return rc;
+    const cudaError_t e = launch_pdl(pa::decode_partition_fp8_kernel<G, CW>,
+                                     dim3(p.num_parts, num_kv_heads, p.num_seqs), dim3(pa::fp8_threads<CW>()),
+                                     pa::kDecodeSmemBytesF, stream, tk, tv, p);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_partition_fp8_kernel launch");
+}
+
+// Two consumer warps when the grid fits in one wave of 4 CTAs per SM, three
+// otherwise (see decode_fp8.cuh).
 template <int G>
 int launch_decode_fp8_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
                         int32_t num_kv_heads, cudaStream_t stream) {
-    static bool done[64] = {};
-    int rc = prepare_kernel(pa::decode_partition_fp8_kernel<G>, pa::kDecodeSmemBytesF, done);
+    const int64_t ctas = static_cast<int64_t>(p.num_parts) * num_kv_heads * p.num_seqs;
+    const bool one_wave = ctas <= static_cast<int64_t>(sm_count()) * pa::kFp8CtasPerSm;
+    int rc = one_wave ? launch_decode_fp8_cw<G, 2>(tk, tv, p, num_kv_heads, stream)
+                      : launch_decode_fp8_cw<G, 3>(tk, tv, p, num_kv_heads, stream);
     if (rc)
         return rc;
-    cudaError_t e = launch_pdl(pa::decode_partition_fp8_kernel<G>, dim3(p.num_parts, num_kv_heads, p.num_seqs),
-                               dim3(pa::kDecodeThreadsM), pa::kDecodeSmemBytesF, stream, tk, tv, p);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "decode_partition_fp8_kernel launch");
+    cudaError_t e;
     if (p.num_parts > 1) {
         e = launch_pdl(pa::decode_merge_kernel, dim3(p.num_q_heads, p.num_seqs, 1), dim3(pa::kD), 0, stream, p);
         if (e != cudaSuccess)

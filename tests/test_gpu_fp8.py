@@ -93,6 +93,20 @@ def test_fp8_decode_block_and_group_sizes(pa, G, B):
     assert pa.pa_get_device_error(clear=True) == 0
 
 
+@pytest.mark.parametrize("G", [1, 8])
+def test_fp8_multi_wave_grid(pa, G):
+    """A grid of more than 4 CTAs per SM (160 sequences x 2 KV heads x 5
+    partitions) runs the three-consumer-warp kernel."""
+    q, kc, vc, bt, n = _case(90 + G, [300] * 150 + [1, 17, 64, 250, 299, 33, 31, 32, 2, 5], 16, 2 * G, 2)
+    ref = oracle.decode_fp8(q, kc, vc, bt, n, 0.08838834764831845, KS, VS)
+    prev = pa.pa_decode_set_partition_tokens(64)
+    try:
+        _close(_run(pa, q, kc, vc, bt, n), ref, f"multi-wave G={G}")
+    finally:
+        pa.pa_decode_set_partition_tokens(prev)
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
 @pytest.mark.parametrize("part", [64, 256, 1024])
 def test_fp8_split_k(pa, part):
     q, kc, vc, bt, n = _case(77, [1, 100, 777, 2049, 5000], 16, 32, 8)
