@@ -58,7 +58,9 @@ enum {
     PA_DEVERR_TIMEOUT = 16,   /* a pipeline wait gave up after its time limit */
     PA_DEVERR_QUERY_LOC = 32  /* pa_attention: query_start_loc not a non-decreasing split of
                                  [0, num_tokens), or a request with more rows than tokens or
-                                 than max_query_len (its rows are left unwritten) */
+                                 than max_query_len (the outputs of that request's rows are
+                                 undefined: not written with one partition, merged from
+                                 unset partials with split-K; every access stays in bounds) */
 };
 
 /* One layer's paged KV cache.  k_cache and v_cache are separate tensors of

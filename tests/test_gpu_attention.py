@@ -147,8 +147,9 @@ def test_attention_spec_decode_full_size(pa):
 
 
 def test_attention_rejects_bad_query_start_loc(pa):
-    """A request with more rows than tokens is flagged on the device and its
-    rows are left unwritten; the other requests are still computed."""
+    """A request with more rows than tokens is flagged on the device; with a
+    single partition its rows are not written, and the other requests are
+    still computed."""
     lens = [3, 50]
     q, kc, vc, bt, qsl, n = _case(82, lens, [2, 5], 16, 8, 2)
     bad_lens = np.array([1, 50], np.int32)  # request 0: 2 rows but 1 token
