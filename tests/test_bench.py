@@ -1,0 +1,59 @@
+"""bench.py's measurement helpers on the CPU: the algorithmic bytes it
+divides by, the ncu traffic it reports (only while the captured kernel
+sources are unchanged), and the host timing of the scheduler step."""
+import os
+import shutil
+import types
+
+import numpy as np
+
+import bench
+import synth
+
+
+def _step(tables, lens, B=4, H=2, D=128, dtype="bf16", T=2, P=0):
+    return types.SimpleNamespace(
+        num_kv_heads=H, head_dim=D, block_size=B, kv_dtype=dtype, ids=list(range(len(lens))),
+        seq_lens_np=np.array(lens, np.int32), block_tables_np=np.array(tables, np.int32),
+        slot_mapping_np=np.zeros(T, np.int64), cow_pairs_np=np.zeros((P, 2), np.int64),
+        q=types.SimpleNamespace(numel=lambda: len(lens) * 8 * D))
+
+
+def test_algorithmic_bytes_count_shared_blocks_once():
+    # sequence 1 shares block 7 (positions 0..3) with sequence 0
+    st = _step([[7, 2, -1], [7, 9, -1]], [6, 5])
+    b = bench.algorithmic_bytes(st)
+    row = 2 * 128 * 2
+    unique = 4 + 2 + 1  # block 7 (4 slots), block 2 (2 of its slots), block 9 (1 slot)
+    assert b["decode_kv"] == unique * row * 2
+    assert b["decode_kv_logical"] == 11 * row * 2
+    assert b["table"] == (2 + 2) * 4
+    assert b["write"] == 2 * 2 * 128 * 2 * 2 + 2 * row * 2
+    fp8 = bench.algorithmic_bytes(_step([[7, 2, -1], [7, 9, -1]], [6, 5], dtype="fp8"))
+    assert fp8["decode_kv"] == b["decode_kv"] // 2
+    rows4 = bench.algorithmic_bytes(st, rows_per_seq=4)
+    assert rows4["q_out"] == 4 * b["q_out"] and rows4["decode_kv"] == b["decode_kv"]
+
+
+def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    for kind in ("bf16", "fp8", "rows4"):
+        t = bench.profiled_traffic("chat", kind)
+        assert isinstance(t, int) and t > 0, kind
+    assert bench.profiled_traffic("long", "bf16") is None  # captured on chat only
+    assert bench.profiled_traffic("chat", "rows8") is None
+    # a copy of the tree with one kernel source edited: no traffic reported
+    root = tmp_path / "tree"
+    shutil.copytree(os.path.join(bench.ROOT, "profiles"), root / "profiles")
+    shutil.copytree(os.path.join(bench.ROOT, "paged_kv_cache_333_b200", "csrc"),
+                    root / "paged_kv_cache_333_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.profiled_traffic("chat", "bf16") is not None
+    with open(root / "paged_kv_cache_333_b200" / "csrc" / "decode_mma.cuh", "a") as f:
+        f.write("\n")
+    assert bench.profiled_traffic("chat", "bf16") is None
+    assert bench.profiled_traffic("chat", "fp8") is None  # also hashes decode_mma.cuh
+
+
+def test_host_pool_step_timing_runs_the_step():
+    r = bench.host_pool_step_us(synth.tiny(), steps=20)
+    assert r["steps"] == 20 and r["sequences"] == 4 and r["us"] > 0
