@@ -318,7 +318,12 @@ PA_API int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_map
                            const pa_cache_fp8_t *cache, void *stream);
 /* pa_decode over an FP8 cache: same contract and output as pa_decode, with
  * K = value(code) * k_scale and V = value(code) * v_scale.  q and out stay
- * bf16.  Scratch per pa_decode_fp8_workspace_bytes. */
+ * bf16.  Scratch per pa_decode_fp8_workspace_bytes.  The codes go into e4m3
+ * tensor-core MMAs as they are; q (scaled per head by a power of two) and the
+ * softmax weights enter as sums of two e4m3 numbers (exact for bf16 q, 8
+ * significant bits for the weights, as bf16 weights have in pa_decode), so
+ * the result is within pa_decode's tolerance of the exact one.  A scale that
+ * is not positive and finite gives PA_EINVAL. */
 PA_API size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
                                             const pa_cache_fp8_t *cache);
 PA_API int pa_decode_fp8(const void *q, const pa_cache_fp8_t *cache, const int32_t *block_tables,
