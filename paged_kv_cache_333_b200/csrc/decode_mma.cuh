@@ -62,15 +62,25 @@ constexpr int kHalfElems = kTile * 64;  // one 64-dim half of a 16-token tile
 // streaming into its other stages while it computes on one.
 static_assert(kStagesM % kConsumerWarpsM == 0, "stages must be a multiple of the consumer warps");
 
+// Multi-wave grids of ragged work (the host decides: more CTAs than 4 per SM
+// and at most 16 partitions per sequence) run a variant with three consumer
+// warps, so that each short CTA finishes sooner; it keeps within 128
+// registers per thread (4 CTAs per SM) by loading the V^T fragments of a tile
+// in two halves.  Other grids keep two consumer warps.
+constexpr int kMaxConsumerWarpsM = 3;
+static_assert(kStagesM % 3 == 0, "stages must be a multiple of every consumer-warp count");
+template <int CW>
+constexpr int mma_threads() { return (CW + 1) * 32; }
+
 struct DecodeSmemM {
     uint16_t kv[kStagesM][4][kHalfElems];  // [stage][K lo, K hi, V lo, V hi][16 x 64]
     uint64_t full[kStagesM];
     uint64_t empty[kStagesM];
-    float wm[kConsumerWarpsM][8];
-    float wl[kConsumerWarpsM][8];
+    float wm[kMaxConsumerWarpsM][8];
+    float wl[kMaxConsumerWarpsM][8];
     int32_t blocks[kMaxPartBlocksM];
 };
-static_assert(sizeof(float) * kConsumerWarpsM * 8 * kD <= sizeof(uint16_t) * kStagesM * 4 * kHalfElems,
+static_assert(sizeof(float) * kMaxConsumerWarpsM * 8 * kD <= sizeof(uint16_t) * kStagesM * 4 * kHalfElems,
               "merge scratch must fit in the KV ring");
 constexpr size_t kDecodeSmemBytesM = sizeof(DecodeSmemM) + 1024;
 
@@ -115,11 +125,13 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int G>
-__global__ void __launch_bounds__(kDecodeThreadsM, kMmaCtasPerSm)
+template <int G, int CW>
+__global__ void __launch_bounds__(mma_threads<CW>(), kMmaCtasPerSm)
 decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+    static_assert(CW == 2 || CW == 3, "consumer warps");
+    constexpr int kCW = CW;
     constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ uint8_t smem_raw[];
     DecodeSmemM &sm = *reinterpret_cast<DecodeSmemM *>(
@@ -142,7 +154,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         }
         mbar_init_fence();
     }
-    if (use_tma && warp == kConsumerWarpsM && lane == 0) {
+    if (use_tma && warp == kCW && lane == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -155,7 +167,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int first_blk = t_begin / B;
     const int32_t *row = p.block_tables + static_cast<int64_t>(s) * p.max_blocks_per_seq + first_blk;
     int32_t first_ids = 0;
-    if (warp == kConsumerWarpsM && lane < p.max_blocks_per_seq - first_blk)
+    if (warp == kCW && lane < p.max_blocks_per_seq - first_blk)
         first_ids = __ldg(row + lane);
     const int n = clamp_seq_len(p, s);
     if (part > 0 && t_begin >= n)
@@ -165,7 +177,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int Hkv = gridDim.y;
     // The producer warp copies the partition's slice of the block table into
     // shared memory (read once, bounds-checked) before the CTA barrier.
-    if (warp == kConsumerWarpsM && num_tiles > 0) {
+    if (warp == kCW && num_tiles > 0) {
         const int nblk = (t_end - 1) / B - first_blk + 1;
         for (int i = lane; i < nblk; i += 32) {
             int32_t b = i < 32 ? first_ids : __ldg(row + i);
@@ -179,7 +191,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     __syncthreads();
 
     // =================================================================== producer
-    if (warp == kConsumerWarpsM) {
+    if (warp == kCW) {
         if (num_tiles == 0 || !use_tma)
             return;  // with blocks < 8 tokens each consumer warp gathers its own tiles
         const uint64_t pol = l2_evict_first_policy();
@@ -270,16 +282,22 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             }
             __syncwarp();
         }
-        uint32_t ka[8][4], va[8][4];
+        // two consumer warps: all V^T fragments now; three: the first half now
+        constexpr int kVa = kCW == 2 ? 8 : 4;
+        uint32_t ka[8][4], va[kVa][4];
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
             ldmatrix_x4(ka[ks], ((ks < 4) ? kb0 : kb1) + swz(k_row, (ks & 3) * 2 + k_chk));
+        auto load_va = [&](int mt0) {
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            const int chunk = 2 * mt + v_chk;  // 16-byte chunk of the 128-dim row
-            ldmatrix_x4_trans(va[mt], ((chunk < 8) ? vb0 : vb1) + swz(v_row, chunk & 7));
-        }
-        loaded();
+            for (int i = 0; i < kVa; ++i) {
+                const int chunk = 2 * (mt0 + i) + v_chk;  // 16-byte chunk of the 128-dim row
+                ldmatrix_x4_trans(va[i], ((chunk < 8) ? vb0 : vb1) + swz(v_row, chunk & 7));
+            }
+        };
+        load_va(0);
+        if constexpr (kCW == 2)
+            loaded();
 
         // ---- S^T = K Q^T ------------------------------------------------
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -310,12 +328,20 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));  // tokens 8..15
         // ---- O^T = alpha O^T + V^T P^T ----------------------------------
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-            acc[mt][0] *= aA;
-            acc[mt][1] *= aB;
-            acc[mt][2] *= aA;
-            acc[mt][3] *= aB;
-            mma_16816(acc[mt], va[mt], pb0, pb1);
+        for (int half = 0; half < 8 / kVa; ++half) {
+            if (half == 1) {  // three consumer warps: second half of V^T, then hand the stage back
+                load_va(kVa);
+                loaded();
+            }
+#pragma unroll
+            for (int i = 0; i < kVa; ++i) {
+                const int mt = half * kVa + i;
+                acc[mt][0] *= aA;
+                acc[mt][1] *= aB;
+                acc[mt][2] *= aA;
+                acc[mt][3] *= aB;
+                mma_16816(acc[mt], va[i], pb0, pb1);
+            }
         }
     };
     auto tile_tokens = [&](int it) { return min(kTile, t_end - (t_begin + it * kTile)); };
@@ -323,7 +349,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (use_tma) {
         // Fed by the producer warp: wait for the stage, release it as soon as
         // the fragments are in registers.
-        for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
+        for (int it = warp; it < num_tiles; it += kCW) {
             const int slot = it % kStagesM;
             bool ok = true;
             if (lane == 0)
@@ -346,7 +372,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         // in stage t % kStagesM, always this warp's).  Lane i < 16 computes the
         // cache row of token i once; the row is broadcast by shuffle to the
         // lanes that copy its 16 chunks (lanes 0-15 K, 16-31 V).
-        constexpr int kAhead = kStagesM / kConsumerWarpsM;
+        constexpr int kAhead = kStagesM / kCW;
         const int tensor = lane >> 4;
         const int ch = lane & 15;
         const uint16_t *cache = static_cast<const uint16_t *>(tensor ? p.v_cache : p.k_cache);
@@ -370,13 +396,13 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
         };
 #pragma unroll
         for (int k = 0; k < kAhead; ++k)
-            gather(warp + k * kConsumerWarpsM);
-        for (int it = warp; it < num_tiles; it += kConsumerWarpsM) {
+            gather(warp + k * kCW);
+        for (int it = warp; it < num_tiles; it += kCW) {
             asm volatile("cp.async.wait_group %0;" ::"n"(kAhead - 1) : "memory");
             __syncwarp();
             consume(it % kStagesM, tile_tokens(it), [] {});
             __syncwarp();  // every lane is done with this stage before it is refilled
-            gather(it + kAhead * kConsumerWarpsM);
+            gather(it + kAhead * kCW);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
     }
@@ -390,7 +416,7 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (threadIdx.x == 0)
         grid_launch_dependents();
 
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
     float *wacc = reinterpret_cast<float *>(&sm.kv[0][0][0]);  // [warp][8 heads][D]
     {
         const int hA = (lane & 3) * 2;
@@ -411,33 +437,41 @@ decode_partition_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
             sm.wl[warp][hA + 1] = lB;
         }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarpsM * 32) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
 
-    // thread t finishes dims t and t + 64 of every real head
+    // the consumer threads finish dims t, t + 32 * kCW, ... of every real head
+    constexpr int kStride = kCW * 32;
+    constexpr int kPer = (kD + kStride - 1) / kStride;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kConsumerWarpsM; ++w)
+        for (int w = 0; w < kCW; ++w)
             M = fmaxf(M, sm.wm[w][g]);
-        float L = 0.f, o[2] = {0.f, 0.f};
+        float L = 0.f, o[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u)
+            o[u] = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kConsumerWarpsM; ++w) {
+            for (int w = 0; w < kCW; ++w) {
                 const float mw = sm.wm[w][g];
                 if (mw == -INFINITY)
                     continue;
                 const float sc = exp2f(mw - M);
                 L = fmaf(sm.wl[w][g], sc, L);
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    o[u] = fmaf(wacc[(w * 8 + g) * kD + threadIdx.x + 64 * u], sc, o[u]);
+                for (int u = 0; u < kPer; ++u)
+                    if (threadIdx.x + kStride * u < kD)
+                        o[u] = fmaf(wacc[(w * 8 + g) * kD + threadIdx.x + kStride * u], sc, o[u]);
             }
         }
         const int j = h * G + g;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int d = threadIdx.x + 64 * u;
+        for (int u = 0; u < kPer; ++u) {
+            const int d = threadIdx.x + kStride * u;
+            if (d >= kD)
+                break;
             if (p.num_parts == 1) {
                 const float r = L > 0.f ? o[u] / L : 0.f;
                 p.out[(static_cast<int64_t>(s) * p.num_q_heads + j) * kD + d] = __float2bfloat16_rn(r);

@@ -212,12 +212,25 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
                     int32_t num_kv_heads, cudaStream_t stream) {
     dim3 grid(p.num_parts, num_kv_heads, p.num_seqs);
     if (g_decode_kernel == PA_DECODE_KERNEL_MMA) {
-        static bool done[64] = {};
-        int rc = prepare_kernel(pa::decode_partition_mma_kernel<G>, pa::kDecodeSmemBytesM, done);
+        // Three consumer warps for multi-wave grids of ragged work, two
+        // otherwise (see decode_mma.cuh).  With at most 16 partitions per
+        // sequence, sequences of varied length leave many short CTAs whose
+        // latency sets the waves (block-size sweeps on B200: +9-11% with
+        // three); with more, nearly every CTA is a full partition and two
+        // warps stream best (32K context on B200: 3% slower with three).  A
+        // one-wave grid has every CTA resident from the start: two warps.
+        const int64_t ctas = static_cast<int64_t>(grid.x) * grid.y * grid.z;
+        const bool one_wave = ctas <= static_cast<int64_t>(sm_count()) * pa::kMmaCtasPerSm;
+        const bool two = one_wave || p.num_parts > 16;
+        static bool done2[64] = {}, done3[64] = {};
+        int rc = two ? prepare_kernel(pa::decode_partition_mma_kernel<G, 2>, pa::kDecodeSmemBytesM, done2)
+                     : prepare_kernel(pa::decode_partition_mma_kernel<G, 3>, pa::kDecodeSmemBytesM, done3);
         if (rc)
             return rc;
-        cudaError_t e = launch_pdl(pa::decode_partition_mma_kernel<G>, grid, dim3(pa::kDecodeThreadsM),
-                                   pa::kDecodeSmemBytesM, stream, tk, tv, p);
+        cudaError_t e = two ? launch_pdl(pa::decode_partition_mma_kernel<G, 2>, grid, dim3(pa::mma_threads<2>()),
+                                         pa::kDecodeSmemBytesM, stream, tk, tv, p)
+                            : launch_pdl(pa::decode_partition_mma_kernel<G, 3>, grid, dim3(pa::mma_threads<3>()),
+                                         pa::kDecodeSmemBytesM, stream, tk, tv, p);
         if (e != cudaSuccess)
             return cuda_fail(e, "decode_partition_mma_kernel launch");
     } else {
