@@ -16,7 +16,7 @@
 //     largest |element| into [128, 256), then split as q' = hi + lo with
 //     hi = e4m3(q'), lo = e4m3(q' - hi).  For a bf16 q this is exact (the
 //     residual of rounding 8 significant bits to 4 has at most 4) except for
-//     elements below 2^-10 of the head's largest, whose error is under 2^-18
+//     elements below 2^-10 of the head's largest, whose error is under 2^-17
 //     of it.  S = K.hi + K.lo (two MMAs), and 2^-s_j joins the score scale.
 //   * P: probabilities are formed as 256 * 2^(x - m) (the factor cancels in
 //     acc / l and in the split-K merge), rounded to f16 for the movmatrix
