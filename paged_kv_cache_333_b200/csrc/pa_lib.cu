@@ -7,6 +7,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -24,8 +25,10 @@
 namespace {
 
 thread_local char g_last_cuda_error[256] = "";
-int32_t g_part_tokens_override = 0;
-int32_t g_decode_kernel = PA_DECODE_KERNEL_MMA;
+// Process-wide knobs (pa_decode_set_*); atomics so that a setter on one host
+// thread and a call on another do not race.  A call reads each knob once.
+std::atomic<int32_t> g_part_tokens_override{0};
+std::atomic<int32_t> g_decode_kernel{PA_DECODE_KERNEL_MMA};
 
 
 
@@ -79,8 +82,9 @@ int32_t choose_part_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t max_s
     const int64_t max_blocks = tensor_core_kernel ? pa::kMaxPartBlocksM : pa::kMaxPartBlocks;
     const int64_t cap = max_blocks * block_size;
     int64_t part;
-    if (g_part_tokens_override > 0) {
-        part = g_part_tokens_override;
+    const int32_t override_tokens = g_part_tokens_override.load(std::memory_order_relaxed);
+    if (override_tokens > 0) {
+        part = override_tokens;
     } else {
         const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
         const int64_t slots = static_cast<int64_t>(sm_count()) *
@@ -101,9 +105,10 @@ struct WorkspaceLayout {
     size_t ml_bytes, acc_offset, total;
 };
 
+bool decode_kernel_is_mma() { return g_decode_kernel.load(std::memory_order_relaxed) == PA_DECODE_KERNEL_MMA; }
+
 WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
-                                 int32_t max_seq_len, int32_t block_size,
-                                 bool tensor_core_kernel = g_decode_kernel == PA_DECODE_KERNEL_MMA) {
+                                 int32_t max_seq_len, int32_t block_size, bool tensor_core_kernel) {
     WorkspaceLayout w{};
     w.part_tokens = choose_part_tokens(num_seqs, num_kv_heads, max_seq_len, block_size, tensor_core_kernel);
     w.num_parts = max_seq_len > 0 ? static_cast<int32_t>((max_seq_len + w.part_tokens - 1) / w.part_tokens) : 1;
@@ -189,10 +194,10 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Opt a kernel into its dynamic shared memory and the all-shared carveout
 // (so that its CTAs-per-SM target fits), once per device.
 template <typename K>
-int prepare_kernel(K kernel, size_t smem, bool (&done)[64]) {
+int prepare_kernel(K kernel, size_t smem, std::atomic<bool> (&done)[64]) {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && done[dev])
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire))
         return PA_OK;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -203,15 +208,15 @@ int prepare_kernel(K kernel, size_t smem, bool (&done)[64]) {
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
     if (dev >= 0 && dev < 64)
-        done[dev] = true;
+        done[dev].store(true, std::memory_order_release);  // setting the attributes twice is harmless
     return PA_OK;
 }
 
 template <int G>
 int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
-                    int32_t num_kv_heads, cudaStream_t stream) {
+                    int32_t num_kv_heads, bool mma, cudaStream_t stream) {
     dim3 grid(p.num_parts, num_kv_heads, p.num_seqs);
-    if (g_decode_kernel == PA_DECODE_KERNEL_MMA) {
+    if (mma) {
         // Three consumer warps for multi-wave grids of ragged work, two
         // otherwise (see decode_mma.cuh).  With at most 16 partitions per
         // sequence, sequences of varied length leave many short CTAs whose
@@ -222,7 +227,7 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
         const int64_t ctas = static_cast<int64_t>(grid.x) * grid.y * grid.z;
         const bool one_wave = ctas <= static_cast<int64_t>(sm_count()) * pa::kMmaCtasPerSm;
         const bool two = one_wave || p.num_parts > 16;
-        static bool done2[64] = {}, done3[64] = {};
+        static std::atomic<bool> done2[64] = {}, done3[64] = {};
         int rc = two ? prepare_kernel(pa::decode_partition_mma_kernel<G, 2>, pa::kDecodeSmemBytesM, done2)
                      : prepare_kernel(pa::decode_partition_mma_kernel<G, 3>, pa::kDecodeSmemBytesM, done3);
         if (rc)
@@ -234,7 +239,7 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
         if (e != cudaSuccess)
             return cuda_fail(e, "decode_partition_mma_kernel launch");
     } else {
-        static bool done[64] = {};
+        static std::atomic<bool> done[64] = {};
         int rc = prepare_kernel(pa::decode_partition_kernel<G>, pa::kDecodeSmemBytes, done);
         if (rc)
             return rc;
@@ -289,7 +294,7 @@ AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_que
 template <int G, int W>
 int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap, int32_t num_kv_heads,
                     cudaStream_t stream) {
-    static bool done[64] = {};
+    static std::atomic<bool> done[64] = {};
     constexpr size_t smem = pa::attend_smem_bytes<W>();
     int rc = prepare_kernel(pa::attend_partition_kernel<G, W>, smem, done);
     if (rc)
@@ -337,7 +342,7 @@ int check_cache_fp8(const pa_cache_fp8_t *c) {
 template <int G, int CW>
 int launch_decode_fp8_cw(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
                          int32_t num_kv_heads, cudaStream_t stream) {
-    static bool done[64] = {};
+    static std::atomic<bool> done[64] = {};
     int rc = prepare_kernel(pa::decode_partition_fp8_kernel<G, CW>, pa::kDecodeSmemBytesF, done);
     if (rc)
         return rc;
@@ -617,7 +622,9 @@ size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t 
                                  const pa_cache_t *cache) {
     if (check_cache(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)
         return 0;
-    return workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size).total;
+    return workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size,
+                            decode_kernel_is_mma())
+        .total;
 }
 
 size_t pa_attention_workspace_bytes(int32_t num_reqs, int32_t num_tokens, int32_t max_query_len,
@@ -709,16 +716,13 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
 }
 
 int32_t pa_decode_set_kernel(int32_t kind) {
-    const int32_t prev = g_decode_kernel;
     if (kind == PA_DECODE_KERNEL_MMA || kind == PA_DECODE_KERNEL_SIMT)
-        g_decode_kernel = kind;
-    return prev;
+        return g_decode_kernel.exchange(kind);
+    return g_decode_kernel.load();
 }
 
 int32_t pa_decode_set_partition_tokens(int32_t tokens) {
-    const int32_t prev = g_part_tokens_override;
-    g_part_tokens_override = tokens > 0 ? tokens : 0;
-    return prev;
+    return g_part_tokens_override.exchange(tokens > 0 ? tokens : 0);
 }
 
 int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
@@ -746,18 +750,18 @@ int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_table
     if (!std::isfinite(scale))
         return PA_EINVAL;
 
+    const bool mma = decode_kernel_is_mma();  // the knob, read once for the whole call
     const WorkspaceLayout w =
-        workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size);
+        workspace_layout(num_seqs, num_q_heads, cache->num_kv_heads, max_seq_len, cache->block_size, mma);
     if (w.total > 0 && (workspace == nullptr || workspace_bytes < w.total))
         return PA_EWORKSPACE;
     if (w.total > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return PA_EUNSUPPORTED;
 
-    const bool swizzled = g_decode_kernel == PA_DECODE_KERNEL_MMA;
     CUtensorMap tk, tv;
-    if ((rc = encode_cache_map(&tk, cache->k_cache, cache, swizzled)) != PA_OK)
+    if ((rc = encode_cache_map(&tk, cache->k_cache, cache, mma)) != PA_OK)
         return rc;
-    if ((rc = encode_cache_map(&tv, cache->v_cache, cache, swizzled)) != PA_OK)
+    if ((rc = encode_cache_map(&tv, cache->v_cache, cache, mma)) != PA_OK)
         return rc;
 
     pa::DecodeParams p{};
@@ -783,10 +787,10 @@ int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_table
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     switch (G) {
-    case 1: return launch_decode_g<1>(tk, tv, p, cache->num_kv_heads, st);
-    case 2: return launch_decode_g<2>(tk, tv, p, cache->num_kv_heads, st);
-    case 4: return launch_decode_g<4>(tk, tv, p, cache->num_kv_heads, st);
-    default: return launch_decode_g<8>(tk, tv, p, cache->num_kv_heads, st);
+    case 1: return launch_decode_g<1>(tk, tv, p, cache->num_kv_heads, mma, st);
+    case 2: return launch_decode_g<2>(tk, tv, p, cache->num_kv_heads, mma, st);
+    case 4: return launch_decode_g<4>(tk, tv, p, cache->num_kv_heads, mma, st);
+    default: return launch_decode_g<8>(tk, tv, p, cache->num_kv_heads, mma, st);
     }
 }
 
