@@ -230,8 +230,8 @@ def algorithmic_bytes(st, rows_per_seq: int = 1) -> dict:
 def host_pool_step_us(w, steps: int = 200) -> dict:
     """Host time of the scheduler-side step (the block table and slot
     mapping build) on the C++ pool: append one token to every sequence in one
-    call, take the queued copy pairs, and build the step's slot mapping,
-    block table and lengths.  Timed on a fresh pool laid out as the workload
+    call, take the queued copy pairs, and build the step's slot mapping and
+    lengths, with the block table kept across steps and updated append-only.  Timed on a fresh pool laid out as the workload
     (the timed device step uses its own)."""
     from paged_kv_cache_333_b200.pool import BlockPool
     sh = w.shape
@@ -242,6 +242,9 @@ def host_pool_step_us(w, steps: int = 200) -> dict:
     pool.take_cow_pairs()
     ids = np.asarray(w.seq_ids, dtype=np.int64)
     width = max(pool.num_blocks_of(int(i)) for i in ids) + steps // sh.block_size + 2
+    table = np.full((len(ids), width), -1, dtype=np.int32)  # kept across steps, updated append-only
+    synced = np.zeros(len(ids), dtype=np.int32)
+    pool.block_table_update(ids, table, synced)
     done = 0
     t0 = time.perf_counter()
     for _ in range(steps):
@@ -249,13 +252,13 @@ def host_pool_step_us(w, steps: int = 200) -> dict:
             break
         pool.take_cow_pairs()
         pool.step_slots(ids, 1)
-        pool.block_table(ids, width)
+        pool.block_table_update(ids, table, synced)
         pool.seq_lens(ids)
         done += 1
     dt = time.perf_counter() - t0
     return {"us": round(dt / max(done, 1) * 1e6, 2), "steps": done, "sequences": int(len(ids)),
-            "what": "append_batch (1 token per sequence) + copy pairs + slot mapping + block table + lengths, "
-                    "C++ pool through ctypes, one host thread"}
+            "what": "append_batch (1 token per sequence) + copy pairs + slot mapping + block table (updated "
+                    "append-only) + lengths, C++ pool through ctypes, one host thread"}
 
 
 # --------------------------------------------------------------------------- ours

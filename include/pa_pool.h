@@ -114,6 +114,20 @@ int64_t pa_pool_free_list(const pa_pool_t *pool, int32_t *out, int64_t capacity)
  * PA_POOL_ERANGE if a sequence holds more than width blocks. */
 int pa_pool_block_table(const pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs,
                         int32_t width, int32_t pad, int32_t *out);
+/* The same rows kept up to date in place, append-only ("PagedAttention:
+ * fragmentation, blocks, block tables", section 2 "The block table": a
+ * request's new block ids are appended to its row).  synced[r] is the number
+ * of entries of row r written by earlier calls for the same sequence; a row
+ * with synced[r] = 0 must hold `pad` everywhere (a fresh row, or one the
+ * caller reset because it now names another sequence or a re-created id).  A
+ * call writes only the old tail entry (a copy-on-write may have redirected
+ * it) and the new entries, and sets synced[r] to the row's block count; the
+ * rows then equal pa_pool_block_table's.  PA_POOL_ERANGE if a sequence holds
+ * more than width blocks or synced[r] is outside [0, width]; PA_POOL_EINVAL
+ * if synced[r] exceeds the sequence's block count (a sequence never loses
+ * blocks, so the row was not reset); nothing is written on an error. */
+int pa_pool_block_table_update(const pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int32_t width,
+                               int32_t pad, int32_t *out, int32_t *synced);
 /* int32 lengths of num_seqs sequences. */
 int pa_pool_seq_lens(const pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs,
                      int32_t *out);

@@ -334,6 +334,34 @@ int pa_pool_block_table(const pa_pool_t *pool, const int64_t *seq_ids, int32_t n
     return PA_POOL_OK;
 }
 
+int pa_pool_block_table_update(const pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int32_t width,
+                               int32_t /* pad: rows past their count already hold it */, int32_t *out,
+                               int32_t *synced) {
+    if (!pool || num_seqs < 0 || width < 0 || (num_seqs > 0 && (!seq_ids || !out || !synced)))
+        return PA_POOL_EINVAL;
+    for (int32_t r = 0; r < num_seqs; ++r) {
+        auto it = pool->seqs.find(seq_ids[r]);
+        if (it == pool->seqs.end())
+            return PA_POOL_ENOSEQ;
+        const int64_t n = static_cast<int64_t>(it->second.blocks.size());
+        if (n > width || synced[r] < 0 || synced[r] > width)
+            return PA_POOL_ERANGE;
+        if (synced[r] > n)  // a sequence never loses blocks: the row names another one now
+            return PA_POOL_EINVAL;
+    }
+    for (int32_t r = 0; r < num_seqs; ++r) {
+        const std::vector<int32_t> &bl = pool->seqs.find(seq_ids[r])->second.blocks;
+        const int32_t n = static_cast<int32_t>(bl.size());
+        int32_t *row = out + static_cast<int64_t>(r) * width;
+        // Entries before the old tail never change; the old tail may have been
+        // redirected by a copy-on-write, and the entries after it are new.
+        const int32_t from = synced[r] > 0 ? synced[r] - 1 : 0;
+        std::copy(bl.begin() + from, bl.end(), row + from);
+        synced[r] = n;
+    }
+    return PA_POOL_OK;
+}
+
 int pa_pool_seq_lens(const pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int32_t *out) {
     if (!pool || num_seqs < 0 || (num_seqs > 0 && (!seq_ids || !out)))
         return PA_POOL_EINVAL;

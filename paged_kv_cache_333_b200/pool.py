@@ -20,7 +20,8 @@ EXPORTED = ("pa_pool_create", "pa_pool_destroy", "pa_pool_seq_create", "pa_pool_
             "pa_pool_fork",
             "pa_pool_release", "pa_pool_num_pending_copies", "pa_pool_take_copies", "pa_pool_num_blocks",
             "pa_pool_block_size", "pa_pool_num_free", "pa_pool_seq_len", "pa_pool_seq_num_blocks",
-            "pa_pool_refcount", "pa_pool_pins", "pa_pool_free_list", "pa_pool_block_table", "pa_pool_seq_lens",
+            "pa_pool_refcount", "pa_pool_pins", "pa_pool_free_list", "pa_pool_block_table",
+            "pa_pool_block_table_update", "pa_pool_seq_lens",
             "pa_pool_slots", "pa_pool_step_slots", "pa_pool_check", "pa_pool_status_str")
 
 _P, _i32, _i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
@@ -45,6 +46,7 @@ for _name, _args, _res in [
     ("pa_pool_pins", [_P, _i64], _i32),
     ("pa_pool_free_list", [_P, _P, _i64], _i64),
     ("pa_pool_block_table", [_P, _P, _i32, _i32, _i32, _P], ctypes.c_int),
+    ("pa_pool_block_table_update", [_P, _P, _i32, _i32, _i32, _P, _P], ctypes.c_int),
     ("pa_pool_seq_lens", [_P, _P, _i32, _P], ctypes.c_int),
     ("pa_pool_slots", [_P, _i64, _i64, _i64, _P], ctypes.c_int),
     ("pa_pool_step_slots", [_P, _P, _i32, _i64, _P], ctypes.c_int),
@@ -161,6 +163,18 @@ class BlockPool:
         out = np.empty((len(ids), width), dtype=np.int32)
         _ok(lib.pa_pool_block_table(self._h, _ptr(ids), len(ids), width, pad, _ptr(out)), "block_table")
         return out
+
+    def block_table_update(self, seq_ids, table: np.ndarray, synced: np.ndarray, pad: int = -1) -> None:
+        """Bring `table` ([num_seqs, width] int32, C-contiguous) up to date in
+        place, writing only the entries that can have changed since `synced`
+        (int32 [num_seqs], entries already written per row; updated)."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        if table.dtype != np.int32 or not table.flags.c_contiguous or table.shape[0] != len(ids):
+            raise ValueError("table must be a C-contiguous int32 [num_seqs, width] array")
+        if synced.dtype != np.int32 or synced.shape != (len(ids),):
+            raise ValueError("synced must be int32 [num_seqs]")
+        _ok(lib.pa_pool_block_table_update(self._h, _ptr(ids), len(ids), table.shape[1], pad, _ptr(table),
+                                           _ptr(synced)), "block_table_update")
 
     def seq_lens(self, seq_ids) -> np.ndarray:
         ids = np.ascontiguousarray(seq_ids, dtype=np.int64)

@@ -337,3 +337,71 @@ def test_append_batch_counts_copies_exactly_at_capacity(rule):
         assert p.num_free() == 0
         assert len(np.asarray(p.take_cow_pairs()).reshape(-1, 2)) == 3
         p.check()
+
+
+@pytest.mark.parametrize("rule", ["shared", "inherited"])
+def test_incremental_block_table_equals_full_rebuild(rule):
+    """Rows kept up to date append-only (only the old tail, which a copy-on-
+    write may redirect, and the new entries are written) equal a full
+    rebuild after every step, including rows reused for another sequence."""
+    for seed in range(10):
+        gen = np.random.default_rng(100 + seed)
+        NB, B, W = 120, 4, 40
+        p = BlockPool(NB, B, gen.permutation(NB).astype(np.int32), rule)
+        live = []
+        next_id = 0
+        for _ in range(4):
+            p.create(next_id)
+            assert p.append(next_id, int(gen.integers(1, 9)))
+            live.append(next_id)
+            next_id += 1
+        rows = list(live)
+        table = np.full((len(rows), W), -1, np.int32)
+        synced = np.zeros(len(rows), np.int32)
+        for step in range(60):
+            op = gen.integers(0, 10)
+            if op < 5:
+                p.append_batch(rows, int(gen.integers(0, 6)))
+            elif op < 7 and len(live) < 8:  # fork a row's sequence into a fresh one (shares its tail)
+                src = rows[int(gen.integers(0, len(rows)))]
+                p.fork(src, next_id)
+                live.append(next_id)
+                next_id += 1
+            elif op < 9:  # a row starts naming another live sequence: the caller resets it
+                free = [i for i in live if i not in rows]
+                if free:
+                    r = int(gen.integers(0, len(rows)))
+                    rows[r] = free[int(gen.integers(0, len(free)))]
+                    table[r, :] = -1
+                    synced[r] = 0
+            else:  # append to one sequence only (copy-on-write of a shared tail)
+                p.append(rows[int(gen.integers(0, len(rows)))], int(gen.integers(1, 4)))
+            p.take_cow_pairs()
+            if max(p.num_blocks_of(i) for i in rows) > W:
+                break
+            p.block_table_update(rows, table, synced)
+            assert np.array_equal(table, p.block_table(rows, W)), (seed, step)
+            assert synced.tolist() == [p.num_blocks_of(i) for i in rows]
+        p.check()
+
+
+def test_incremental_block_table_refuses_a_row_that_was_not_reset():
+    """A row whose count exceeds its sequence's blocks names another sequence
+    now: refused with nothing written (silently keeping the other sequence's
+    leading entries would give a wrong table)."""
+    p = BlockPool(20, 4, np.arange(20, dtype=np.int32))
+    for k, n in ((0, 14), (1, 3)):
+        p.create(k)
+        assert p.append(k, n)
+    table = np.full((1, 6), -1, np.int32)
+    synced = np.zeros(1, np.int32)
+    p.block_table_update([0], table, synced)
+    assert synced.tolist() == [4]
+    before = table.copy()
+    with pytest.raises(Exception):
+        p.block_table_update([1], table, synced)  # same row, other sequence, count not reset
+    assert np.array_equal(table, before) and synced.tolist() == [4]
+    table[:] = -1
+    synced[:] = 0
+    p.block_table_update([1], table, synced)
+    assert np.array_equal(table, p.block_table([1], 6)) and synced.tolist() == [1]
