@@ -94,3 +94,20 @@ def test_host_side_validation_of_the_widened_entry_points():
     assert lib.pa_map_to_kernel_blocks(16, 4, 10, 4, 16, 39, None) == PA_EINVAL    # too narrow
     assert lib.pa_map_to_kernel_blocks(16, 4, 10, 4, None, 40, None) == PA_EINVAL
     assert lib.pa_map_to_kernel_blocks(None, 0, 10, 4, None, 40, None) == 0       # no rows
+
+
+@pytest.mark.parametrize("missing", ["libpa.so", "libpa_pool.so"])
+def test_package_refuses_to_import_without_its_libraries(tmp_path, missing):
+    """No fallback path: a copy of the package without one of its built
+    libraries fails at import, naming the library."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = tmp_path / "paged_kv_cache_333_b200"
+    shutil.copytree(os.path.join(ROOT, "paged_kv_cache_333_b200"), pkg,
+                    ignore=shutil.ignore_patterns("csrc", "__pycache__"))
+    os.remove(pkg / missing)
+    r = subprocess.run([sys.executable, "-c", "import paged_kv_cache_333_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert missing in r.stderr
