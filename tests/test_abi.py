@@ -111,3 +111,24 @@ def test_package_refuses_to_import_without_its_libraries(tmp_path, missing):
                        capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert missing in r.stderr
+
+
+def test_split_k_partition_choice_through_the_workspace_sizes():
+    """The partition heuristic, seen through the public workspace sizes (no
+    device: the SM count falls back to B200's 148).  Chat lengths (<= 612
+    tokens) take one partition, so no scratch; 32K context takes 640-token
+    partitions: 52 per sequence, (m, l) float2 + 128 fp32 per (sequence,
+    query head, partition)."""
+    from paged_kv_cache_333_b200._abi import PaCache, lib
+    c = ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))
+    assert lib.pa_decode_workspace_bytes(64, 32, 612, c) == 0
+    units = 8 * 32 * 52
+    ml = units * 8
+    expect = -(-ml // 256) * 256 + units * 128 * 4
+    assert lib.pa_decode_workspace_bytes(8, 32, 32768, c) == expect
+    # pa_attention over the same sequences, 4 rows each: per (row, head, partition)
+    rows = 8 * 4
+    cells = rows * 32 * 52
+    acc_off = -(-cells * 8 // 256) * 256
+    len_off = -(-(acc_off + cells * 128 * 4) // 256) * 256
+    assert lib.pa_attention_workspace_bytes(8, rows, 4, 32, 32768, c) == len_off + rows * 4
