@@ -251,7 +251,7 @@ def sweep(block_size: int, seed: int = 337, batch: int = 128, mean_len: int = 10
           cap: int = 8192, events: int = 10_000, occupancy: float = 0.9,
           slots: int = LLAMA3_8B_POOL_SLOTS) -> Workload:
     """Block-size sweep under fragmentation.  The pool keeps the same token
-    capacity for every block size (num_blocks = 428,560 / block_size, the
+    capacity for every block size (num_blocks = floor(428,560 / block_size), the
     "block count halved" rule of page 1's experiment list).  Churn: ``events``
     seeded events on background sequences, each either a create with a
     Geometric(1/mean_len) length capped at ``cap`` tokens or the release of a
