@@ -280,7 +280,10 @@ PA_API int32_t pa_decode_set_partition_tokens(int32_t tokens);
  *   nothing.  The call allocates nothing.
  *   Set-up: the first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current and caches it; make that
- *   first call before any stream capture.
+ *   first call before any stream capture.  A call with num_seqs = 0 does only
+ *   this set-up and enqueues nothing.
+ *   Errors: the argument checks of pa_decode, then the scratch size check,
+ *   run on the host before any CUDA call.
  *   Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents (nothing in it needs to start at zero).  Calls that may
  *   overlap on the GPU (other streams, other host threads) race on it:

@@ -371,6 +371,34 @@ int launch_decode_fp8_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::
     }
     return PA_OK;
 }
+
+// The host-side argument checks of pa_decode (and pa_decode_static_ws, which
+// runs them before it touches the CUDA runtime).  An empty batch passes.
+int check_decode_args(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
+                      int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                      int32_t max_seq_len, int32_t num_q_heads, float scale, const void *out) {
+    int rc = check_cache(cache);
+    if (rc)
+        return rc;
+    if (num_seqs < 0 || max_seq_len < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
+        return PA_EINVAL;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (!q || !block_tables || !seq_lens || !out)
+        return PA_EINVAL;
+    if (num_q_heads % cache->num_kv_heads != 0)
+        return PA_EINVAL;
+    const int32_t G = num_q_heads / cache->num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return PA_EUNSUPPORTED;
+    if (!aligned16(q) || !aligned16(out))
+        return PA_EUNSUPPORTED;
+    if (num_seqs > 65535 || cache->num_kv_heads > 65535)
+        return PA_EUNSUPPORTED;
+    if (!std::isfinite(scale))
+        return PA_EINVAL;
+    return PA_OK;
+}
 }  // namespace
 
 extern "C" {
@@ -729,26 +757,11 @@ int pa_decode(const void *q, const pa_cache_t *cache, const int32_t *block_table
               int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
               int32_t max_seq_len, int32_t num_q_heads, float scale, void *out, void *workspace,
               size_t workspace_bytes, void *stream) {
-    int rc = check_cache(cache);
-    if (rc)
+    int rc = check_decode_args(q, cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, max_seq_len,
+                               num_q_heads, scale, out);
+    if (rc || num_seqs == 0)
         return rc;
-    if (num_seqs < 0 || max_seq_len < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
-        return PA_EINVAL;
-    if (num_seqs == 0)
-        return PA_OK;
-    if (!q || !block_tables || !seq_lens || !out)
-        return PA_EINVAL;
-    if (num_q_heads % cache->num_kv_heads != 0)
-        return PA_EINVAL;
     const int32_t G = num_q_heads / cache->num_kv_heads;
-    if (G != 1 && G != 2 && G != 4 && G != 8)
-        return PA_EUNSUPPORTED;
-    if (!aligned16(q) || !aligned16(out))
-        return PA_EUNSUPPORTED;
-    if (num_seqs > 65535 || cache->num_kv_heads > 65535)
-        return PA_EUNSUPPORTED;
-    if (!std::isfinite(scale))
-        return PA_EINVAL;
 
     const bool mma = decode_kernel_is_mma();  // the knob, read once for the whole call
     const WorkspaceLayout w =
@@ -834,10 +847,13 @@ int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int32_t *b
                         int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
                         int32_t max_seq_len, int32_t num_q_heads, float scale, void *out,
                         void *stream) {
-    int rc = check_cache(cache);
+    // Argument errors and a too-large shape are reported before any CUDA
+    // call; an empty batch still does the one-time address lookup below.
+    int rc = check_decode_args(q, cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, max_seq_len,
+                               num_q_heads, scale, out);
     if (rc)
         return rc;
-    if (num_seqs > 0 && num_q_heads > 0 && max_seq_len >= 0) {
+    if (num_seqs > 0) {
         const size_t need = pa_decode_workspace_bytes(num_seqs, num_q_heads, max_seq_len, cache);
         if (need > PA_DECODE_STATIC_WS_BYTES) {
             std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error,

@@ -132,3 +132,70 @@ def test_split_k_partition_choice_through_the_workspace_sizes():
     acc_off = -(-cells * 8 // 256) * 256
     len_off = -(-(acc_off + cells * 128 * 4) // 256) * 256
     assert lib.pa_attention_workspace_bytes(8, rows, 4, 32, 32768, c) == len_off + rows * 4
+
+
+def test_host_side_validation_of_the_remaining_entry_points():
+    """Slot mapping, the fused positions write, the all-layer copy, the
+    static-scratch decode and the process-wide knobs: every rejection below
+    happens on the host, before any CUDA call (this machine has no device)."""
+    from paged_kv_cache_333_b200._abi import (PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT,
+                                              PA_DECODE_STATIC_WS_BYTES, PA_EINVAL, PA_EUNSUPPORTED,
+                                              PA_EWORKSPACE, PaCache, lib)
+    ok = PaCache(16, 16, 26785, 16, 8, 128)  # fake, aligned pointers: never dereferenced
+    c = ctypes.byref(ok)
+
+    def slots(pos=16, req=16, T=4, bt=16, W=8, R=2, B=16, NB=64, out=16):
+        return lib.pa_compute_slot_mapping(pos, req, T, bt, W, R, B, NB, out, None)
+
+    assert slots(T=-1) == PA_EINVAL and slots(W=-1) == PA_EINVAL and slots(R=-1) == PA_EINVAL
+    assert slots(B=0) == PA_EINVAL and slots(NB=0) == PA_EINVAL
+    assert slots(T=0) == 0
+    assert slots(pos=None) == PA_EINVAL and slots(req=None) == PA_EINVAL and slots(out=None) == PA_EINVAL
+    assert slots(bt=None) == PA_EINVAL        # requests but no tables
+
+    def wpos(k=16, v=16, pos=16, req=16, T=4, bt=16, W=8, R=2, cache=c):
+        return lib.pa_write_kv_positions(k, v, pos, req, T, bt, W, R, cache, None)
+
+    assert wpos(T=-1) == PA_EINVAL and wpos(R=-1) == PA_EINVAL
+    assert wpos(T=0) == 0
+    assert wpos(k=None) == PA_EINVAL and wpos(req=None) == PA_EINVAL and wpos(bt=None) == PA_EINVAL
+    assert wpos(v=24) == PA_EUNSUPPORTED      # v not 16-byte aligned
+    assert wpos(cache=ctypes.byref(PaCache(16, 16, 64, 16, 2, 64))) == PA_EUNSUPPORTED
+    assert wpos(cache=ctypes.byref(PaCache(None, 16, 64, 16, 2, 128))) == PA_EINVAL
+
+    layers = (PaCache * 3)(ok, ok, ok)
+    assert lib.pa_copy_blocks_layers(layers, 3, None, 0, None) == 0
+    assert lib.pa_copy_blocks_layers(layers, 0, 16, 5, None) == 0
+    assert lib.pa_copy_blocks_layers(layers, 3, None, 5, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_layers(layers, 3, 16, -1, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_layers(None, 3, 16, 5, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_layers(layers, 129, 16, 5, None) == PA_EUNSUPPORTED
+    mixed = (PaCache * 2)(ok, PaCache(16, 16, 26784, 16, 8, 128))  # one pair list, two geometries
+    assert lib.pa_copy_blocks_layers(mixed, 2, 16, 5, None) == PA_EINVAL
+
+    def static(q=16, S=4, maxlen=600, Hq=32, scale=0.1, out=16):
+        return lib.pa_decode_static_ws(q, c, 16, 64, 16, S, maxlen, Hq, scale, out, None)
+
+    assert static(S=-1) == PA_EINVAL and static(Hq=30) == PA_EINVAL and static(q=None) == PA_EINVAL
+    assert static(Hq=24) == PA_EUNSUPPORTED and static(out=8) == PA_EUNSUPPORTED
+    assert static(scale=float("inf")) == PA_EINVAL
+    big = lib.pa_decode_workspace_bytes(64, 32, 32768, c)
+    assert big > PA_DECODE_STATIC_WS_BYTES
+    assert static(S=64, maxlen=32768) == PA_EWORKSPACE
+    assert b"static" in lib.pa_last_cuda_error()
+
+    prev = lib.pa_decode_set_kernel(PA_DECODE_KERNEL_SIMT)
+    try:
+        assert prev == PA_DECODE_KERNEL_MMA
+        assert lib.pa_decode_set_kernel(7) == PA_DECODE_KERNEL_SIMT   # ignored, reports the current
+        assert lib.pa_decode_set_kernel(PA_DECODE_KERNEL_MMA) == PA_DECODE_KERNEL_SIMT
+    finally:
+        lib.pa_decode_set_kernel(prev)
+    prev = lib.pa_decode_set_partition_tokens(256)
+    try:
+        assert lib.pa_decode_set_partition_tokens(-5) == 256
+        assert lib.pa_decode_set_partition_tokens(0) == 0            # negative means automatic
+    finally:
+        lib.pa_decode_set_partition_tokens(prev)
+    for code, text in ((0, b"ok"), (-1, b"invalid argument"), (-2, b"unsupported"), (-4, b"CUDA"), (9, b"unknown")):
+        assert text in lib.pa_status_str(code)
