@@ -260,6 +260,19 @@ PA_API int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_
 enum { PA_DECODE_KERNEL_MMA = 0, PA_DECODE_KERNEL_SIMT = 1 };
 PA_API int32_t pa_decode_set_kernel(int32_t kind);
 
+/* Which kernel pa_attention runs (process wide; returns the previous value;
+ * other values are ignored).  pa_attention_workspace_bytes() follows the
+ * setting, so query it after choosing.
+ *   PA_ATTENTION_KERNEL_MMA     (default) warps of 8 (row, head) columns on
+ *                               mma.m16n8k16, 16-token K/V tiles;
+ *   PA_ATTENTION_KERNEL_TCGEN05 128 columns per CTA on tcgen05.mma with the
+ *                               S and O accumulators in tensor memory, 64-token
+ *                               K/V tiles: for requests with many rows
+ *                               (prefill chunks).  Not yet validated on a
+ *                               GPU; the default stays the MMA kernel. */
+enum { PA_ATTENTION_KERNEL_MMA = 0, PA_ATTENTION_KERNEL_TCGEN05 = 1 };
+PA_API int32_t pa_attention_set_kernel(int32_t kind);
+
 /* Tokens per split-K partition used by pa_decode: 0 = automatic (the
  * default), otherwise a multiple of 64.  Host-side setting, process wide;
  * returns the previous value.  For tuning and tests. */

@@ -27,9 +27,10 @@ PA_DEVERR_QUERY_LOC = 32
 EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
             "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
             "pa_map_to_kernel_blocks", "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
-            "pa_decode_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
+            "pa_decode_set_kernel", "pa_attention_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
+PA_ATTENTION_KERNEL_MMA, PA_ATTENTION_KERNEL_TCGEN05 = 0, 1
 
 
 class PaCache(ctypes.Structure):
@@ -82,6 +83,8 @@ lib.pa_decode_fp8.argtypes = [_P, ctypes.POINTER(PaCacheFp8), _P, _i32, _P, _i32
 lib.pa_decode_fp8.restype = ctypes.c_int
 lib.pa_decode_set_kernel.argtypes = [_i32]
 lib.pa_decode_set_kernel.restype = _i32
+lib.pa_attention_set_kernel.argtypes = [_i32]
+lib.pa_attention_set_kernel.restype = _i32
 lib.pa_decode_set_partition_tokens.argtypes = [_i32]
 lib.pa_decode_set_partition_tokens.restype = _i32
 lib.pa_get_device_error.argtypes = [ctypes.POINTER(_i32), ctypes.c_int]
@@ -371,6 +374,13 @@ def pa_decode_set_kernel(kind: str) -> str:
     """Select the decode partition kernel: "mma" (default) or "simt"; returns the previous one."""
     prev = lib.pa_decode_set_kernel({"mma": PA_DECODE_KERNEL_MMA, "simt": PA_DECODE_KERNEL_SIMT}[kind])
     return "mma" if prev == PA_DECODE_KERNEL_MMA else "simt"
+
+
+def pa_attention_set_kernel(kind: str) -> str:
+    """Select the pa_attention kernel: "mma" (default) or "tcgen05" (128
+    columns per CTA, accumulators in tensor memory); returns the previous one."""
+    prev = lib.pa_attention_set_kernel({"mma": PA_ATTENTION_KERNEL_MMA, "tcgen05": PA_ATTENTION_KERNEL_TCGEN05}[kind])
+    return "mma" if prev == PA_ATTENTION_KERNEL_MMA else "tcgen05"
 
 
 def pa_decode_set_partition_tokens(tokens: int) -> int:

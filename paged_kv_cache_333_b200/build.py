@@ -21,7 +21,7 @@ LIBPA = os.path.join(PKG, "libpa.so")
 LIBPOOL = os.path.join(PKG, "libpa_pool.so")
 
 CUDA_SOURCES = ["pa_lib.cu"]
-CUDA_DEPS = ["pa_lib.cu", "attend.cuh", "decode.cuh", "decode_mma.cuh", "decode_fp8.cuh", "kv_ops.cuh", "pa_device.cuh"]
+CUDA_DEPS = ["pa_lib.cu", "attend.cuh", "attend_tc.cuh", "decode.cuh", "decode_mma.cuh", "decode_fp8.cuh", "kv_ops.cuh", "pa_device.cuh"]
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared",
               "--expt-relaxed-constexpr"]

@@ -1,0 +1,568 @@
+// Attention of several query tokens per request over the paged cache on the
+// fifth-generation tensor cores (tcgen05): the same operation as
+// attend_partition_kernel ("PagedAttention: fragmentation, blocks, block
+// tables", the attention-metadata passage: query_start_loc, seq_lens,
+// max_query_len; row i of a request with q_len rows and n tokens attends to
+// positions 0 .. n - q_len + i), for requests with many rows: chunks of a
+// prefill, long speculative runs.
+//
+// Work decomposition.  A column is one (query row, query head of the KV group)
+// pair, c = i * G + g, as in attend.cuh.  One CTA handles one (split-K
+// partition, KV head, request, chunk of 128 columns) and streams the chunk's
+// token range in 64-token tiles:
+//   S = Q K^T    M = 128 columns, N = 64 tokens, K = 128 dims: 8 MMAs of K = 16
+//   O += P V     M = 128 columns, N = 128 dims, K = 64 tokens: 4 MMAs of K = 16
+// (tcgen05.mma.cta_group::1.kind::f16, bf16 operands, fp32 accumulators in
+// tensor memory).  Q, K, P are K-major and V is MN-major, all in the 128-byte
+// swizzled layout the TMA loads write: rows of 128 bytes, 16-byte chunk j of
+// row r at position j ^ (r % 8), 8-row groups 1024 bytes apart.
+//
+// Roles (192 threads):
+//   warps 0-3  softmax: thread t owns column t of the chunk, which is tensor-
+//              memory lane t (a warp may only read lanes 32 * (warp % 4) ..
+//              + 31).  Per tile: read its S row (64 fp32), mask, online
+//              softmax with a lazily moved reference max, write its P row
+//              (bf16) to shared memory; at the end read its O row and write
+//              the output (or the split-K partials);
+//   warp 4     producer: 64-token K/V tiles into a 4-stage ring, by TMA for
+//              whole tiles of blocks >= 8 tokens, else by a cp.async gather
+//              that zero-fills the rows past the range;
+//   warp 5     allocates tensor memory; one thread issues the MMAs.
+// Tensor memory: S double-buffered in columns [0, 64) and [64, 128), O in
+// [128, 256); 256 columns per CTA, one CTA per SM (shared memory).
+//
+// Lazy rescaling.  A column keeps a reference max m_ref (log2 domain) and
+// moves it only when a tile's max exceeds it by more than 8; the weights
+// 2^(x - m_ref) then stay <= 256, exact enough in bf16 for P and far from
+// fp32 overflow in O and l.  Moving m_ref multiplies that column's O row in
+// tensor memory by 2^(old - new), after the previous tile's P V has
+// completed.  (m_ref, l, O) is a consistent triple at any reference, which is
+// all the final division and the split-K merge need.
+//
+// Synchronisation (all mbarriers, every wait bounded):
+//   full[s]    producer -> MMA      stage s holds tile t (TMA bytes or cp.async)
+//   empty[s]   MMA commit -> producer  P V of tile t done: stage s reusable
+//   s_full[b]  MMA commit -> softmax   S of tile t in buffer b = t % 2
+//   s_free[b]  softmax (4 warps) -> MMA  S buffer b read
+//   p_full[b]  softmax (4 warps) -> MMA  P buffer b written, O rescaled
+//   pv_done[b] MMA commit -> softmax   P V of tile t done: P buffer b free, O current
+// The MMA thread issues S(t + 1) before P V(t), so the tensor pipe computes
+// the next scores while the softmax warps work on the current tile.  No
+// waiter can fall two phases behind a barrier: each phase it waits for is
+// the latest one that the other side can have completed.
+#pragma once
+
+#include "attend.cuh"
+
+namespace pa {
+
+constexpr int kTokTc = 64;      // tokens per tile
+constexpr int kStagesTc = 4;    // K/V ring depth
+constexpr int kColsTc = 128;    // columns per CTA (= MMA M = tensor-memory lanes)
+constexpr int kTmemColsTc = 256;
+constexpr int kTcThreads = 192;
+constexpr int kTcSoftmaxThreads = 128;
+constexpr int kTcProducerWarp = 4;
+constexpr int kTcMmaWarp = 5;
+constexpr float kLazyRescaleLog2 = 8.f;
+
+// ---------------------------------------------------------------- descriptors
+// Instruction descriptor of tcgen05.mma.kind::f16 with bf16 A and B and an
+// fp32 accumulator (PTX ISA, "Instruction descriptor"): bits 4-5 D format
+// (1 = f32), 7-9 A format (1 = bf16), 10-12 B format (1 = bf16), 15 A
+// major-ness, 16 B major-ness (0 = K-major, 1 = MN-major), 17-22 N / 8,
+// 24-28 M / 16.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
+           (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
+}
+// Shared-memory matrix descriptor (PTX ISA, "Shared memory descriptor"):
+// bits 0-13 start address / 16, 16-29 leading-dimension byte offset / 16,
+// 32-45 stride-dimension byte offset / 16, 46-47 version (1), 49-51 base
+// offset (0: every swizzle atom here starts on a 1024-byte boundary), 61-63
+// layout (2 = 128-byte swizzle).
+__host__ __device__ constexpr uint64_t umma_sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// The two MMA shapes of this kernel, written out bit by bit.
+static_assert(umma_idesc_bf16(128, 64, false, false) == 0x08100490u, "S = Q K^T descriptor");
+static_assert(umma_idesc_bf16(128, 128, false, true) == 0x08210490u, "O += P V descriptor");
+static_assert(umma_sdesc_sw128(0x1000u, 16u, 1024u) == 0x4000404000010100ull, "K-major operand descriptor");
+static_assert(umma_sdesc_sw128(0x2000u, 8192u, 1024u) == 0x4000404002000200ull, "MN-major operand descriptor");
+
+constexpr uint32_t kIdescS = umma_idesc_bf16(kColsTc, kTokTc, false, false);
+constexpr uint32_t kIdescPV = umma_idesc_bf16(kColsTc, kD, false, true);
+
+// ---------------------------------------------------------------- tcgen05 PTX
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// D (tensor memory) = A B (+ D when accumulate != 0); A and B in shared memory.
+__device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive once on `bar` when every tcgen05.mma this thread issued so far is complete.
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+// 32 consecutive fp32 columns of this thread's tensor-memory lane, waited for
+// in the same statement (so no use of r can be scheduled before the wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+          "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+          "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 16-byte cp.async that writes zeros when src_bytes is 0.
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+// Arrive on `bar` when this thread's cp.async copies so far have landed; the
+// pending count is raised first, so the arrival does not count toward the
+// barrier's expected count.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+struct AttendTcSmem {
+    uint16_t kv[kStagesTc][4][kTokTc * 64];  // [stage][K lo, K hi, V lo, V hi][64 tokens x 64 dims], swizzled
+    uint16_t q[2][kColsTc * 64];             // [dims lo, dims hi][128 columns x 64 dims], swizzled
+    uint16_t p[2][kColsTc * kTokTc];         // [buffer][128 columns x 64 tokens], swizzled
+    uint64_t full[kStagesTc];
+    uint64_t empty[kStagesTc];
+    uint64_t s_full[2];
+    uint64_t s_free[2];
+    uint64_t p_full[2];
+    uint64_t pv_done[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int32_t blocks[kMaxPartBlocksM];
+};
+constexpr size_t kAttendTcSmemBytes = sizeof(AttendTcSmem) + 1024;
+static_assert(kAttendTcSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert(offsetof(AttendTcSmem, q) % 1024 == 0 && offsetof(AttendTcSmem, p) % 1024 == 0,
+              "swizzle atoms start on 1024-byte boundaries");
+
+template <int G>
+__global__ void __launch_bounds__(kTcThreads, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const AttendParams ap) {
+    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+    constexpr unsigned FULL = 0xffffffffu;
+    const DecodeParams &p = ap.d;
+    extern __shared__ uint8_t smem_raw[];
+    AttendTcSmem &sm = *reinterpret_cast<AttendTcSmem *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const int part = blockIdx.x;
+    const int h = blockIdx.y;
+    const int r = blockIdx.z / ap.chunks;
+    const int chunk = blockIdx.z % ap.chunks;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int B = p.block_size;
+    const int Hkv = gridDim.y;
+
+    if (warp == kTcProducerWarp && lane == 0 && B >= 8) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    grid_dependency_wait();
+
+    // ---- the request's rows, this CTA's columns and token range -------------
+    // (every exit before the tensor-memory allocation below is CTA-uniform)
+    const int q0 = ap.query_start_loc[r];
+    const int q1 = ap.query_start_loc[r + 1];
+    const int n = clamp_seq_len(p, r);
+    const int q_len = q1 - q0;
+    if (q_len < 0 || q_len > n || q_len > ap.max_query_len || q0 < 0 || q1 > ap.num_tokens ||
+        (r == 0 && q0 != 0) || (r == p.num_seqs - 1 && q1 != ap.num_tokens)) {
+        if (part == 0 && h == 0 && chunk == 0 && threadIdx.x == 0)
+            flag_error(PA_DEVERR_QUERY_LOC);
+        return;
+    }
+    const int cols = q_len * G;
+    const int col0 = chunk * kColsTc;
+    if (col0 >= cols)
+        return;
+    const int last_col = min(cols, col0 + kColsTc) - 1;
+    const int first_visible = n - q_len;               // row i sees positions <= first_visible + i
+    const int lim_max = first_visible + last_col / G;  // >= 0
+    const int t_begin = part * p.part_tokens;
+    if (t_begin > lim_max)
+        return;
+    const int t_end = min(lim_max + 1, t_begin + p.part_tokens);
+    const int num_tiles = (t_end - t_begin + kTokTc - 1) / kTokTc;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStagesTc; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.s_full[b], 1);
+            mbar_init(&sm.s_free[b], 4);
+            mbar_init(&sm.p_full[b], 4);
+            mbar_init(&sm.pv_done[b], 1);
+        }
+        mbar_init(&sm.mma_done, 1);
+        mbar_init_fence();
+    }
+    if (p.num_parts > 1 && part == 0 && h == 0 && warp == 0) {
+        for (int i = col0 / G + lane; i <= last_col / G; i += 32)
+            ap.row_len[q0 + i] = first_visible + i + 1;
+    }
+    const int first_blk = t_begin / B;
+    if (warp == kTcProducerWarp) {
+        const int32_t *row = p.block_tables + static_cast<int64_t>(r) * p.max_blocks_per_seq + first_blk;
+        const int nblk = (t_end - 1) / B - first_blk + 1;
+        for (int i = lane; i < nblk; i += 32) {
+            int32_t b = __ldg(row + i);
+            if (b < 0 || b >= p.num_blocks) {
+                flag_error(PA_DEVERR_BLOCK_ID);
+                b = 0;
+            }
+            sm.blocks[i] = b;
+        }
+    }
+    if (warp < 4) {
+        // Q rows of the chunk's columns into the swizzled K-major tile; zeros
+        // for columns past the chunk (their scores are masked anyway).
+        const int c = col0 + threadIdx.x;
+        const bool ok = c <= last_col;
+        const uint4 *qrow = p.q + ((static_cast<int64_t>(q0) + (ok ? c / G : 0)) * p.num_q_heads + h * G +
+                                   (ok ? c % G : 0)) *
+                                      (kD / 8);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const uint4 v = ok ? __ldg(qrow + k) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(&sm.q[k >> 3][0]) + swz(threadIdx.x, k & 7)) = v;
+        }
+        fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
+    }
+    if (warp == kTcMmaWarp) {
+        tmem_alloc(&sm.tmem_base, kTmemColsTc);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t tmem_o = tmem + 2 * kTokTc;
+
+    if (warp == kTcProducerWarp) {
+        // ============================================================ producer
+        const uint64_t pol = l2_evict_first_policy();
+        int issued = 0;
+        bool dead = false;
+        for (int it = 0; it < num_tiles && !dead; ++it) {
+            const int slot = it % kStagesTc;
+            if (it >= kStagesTc) {
+                bool ok = true;
+                if (lane == 0)
+                    ok = mbar_wait(&sm.empty[slot], ((it / kStagesTc) + 1) & 1);
+                if (!__shfl_sync(FULL, ok, 0)) {
+                    dead = true;
+                    break;
+                }
+            }
+            const int t0 = t_begin + it * kTokTc;
+            const int ntok = min(kTokTc, t_end - t0);
+            if (B >= 8 && ntok == kTokTc) {
+                // whole tile by TMA: boxes of min(B, 16) rows, 4 quarters each
+                const int rows = B < kTile ? B : kTile;
+                const int nbox = kTokTc / rows;  // 4 or 8
+                if (lane == 0)
+                    mbar_arrive_expect_tx(&sm.full[slot], static_cast<uint32_t>(kTokTc * 128 * 4));
+                __syncwarp();
+                const int j = lane >> 2, qd = lane & 3;  // box j of quarter qd (K lo, K hi, V lo, V hi)
+                if (j < nbox) {
+                    const int t = t0 + j * rows;
+                    const int32_t rr = sm.blocks[t / B - first_blk] * B + (t % B);
+                    tma_load_3d(&sm.kv[slot][qd][j * rows * 64], (qd < 2) ? &tm_k : &tm_v, (qd & 1) * 64, h, rr,
+                                &sm.full[slot], pol);
+                }
+            } else {
+                // gather: lane = (quarter, 16-byte chunk); rows past the range
+                // are zero-filled so that 0-weight V rows stay finite
+                const int qd = lane >> 3, ch = lane & 7;
+                const uint16_t *cache = static_cast<const uint16_t *>(qd < 2 ? p.k_cache : p.v_cache);
+                // cache rows of tokens lane and lane + 32, handed out by shuffle
+                int64_t row_lo = 0, row_hi = 0;
+                if (lane < ntok) {
+                    const int t = t0 + lane;
+                    row_lo = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + h;
+                }
+                if (lane + 32 < ntok) {
+                    const int t = t0 + lane + 32;
+                    row_hi = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + h;
+                }
+                const uint32_t base = smem_addr(&sm.kv[slot][qd][0]);
+                for (int i = 0; i < kTokTc; ++i) {
+                    const int64_t rr = __shfl_sync(FULL, i < 32 ? row_lo : row_hi, i & 31);
+                    const bool in = i < ntok;
+                    cp_async16_zfill(base + swz(i, ch), cache + (in ? rr * kD + (qd & 1) * 64 + ch * 8 : 0),
+                                     in ? 16u : 0u);
+                }
+                cp_async_mbar_arrive(&sm.full[slot]);
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.full[slot]);
+            }
+            issued = it + 1;
+        }
+        // nothing may still be copying into shared memory when the CTA ends
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        if (lane == 0) {
+            for (int sl = 0; sl < kStagesTc && sl < issued; ++sl) {
+                const int last = sl + ((issued - 1 - sl) / kStagesTc) * kStagesTc;
+                mbar_wait(&sm.full[sl], (last / kStagesTc) & 1);
+            }
+        }
+    } else if (warp == kTcMmaWarp) {
+        // ============================================================ MMA issue
+        if (lane == 0) {
+            const uint32_t q_base = smem_addr(&sm.q[0][0]);
+            auto pv = [&](int u) -> bool {
+                if (!mbar_wait(&sm.p_full[u & 1], (u >> 1) & 1))
+                    return false;
+                tc_fence_after();
+                const uint32_t p_base = smem_addr(&sm.p[u & 1][0]);
+                const uint32_t v_base = smem_addr(&sm.kv[u % kStagesTc][2][0]);
+#pragma unroll
+                for (int kk = 0; kk < kTokTc / 16; ++kk)
+                    umma_bf16_ss(tmem_o, umma_sdesc_sw128(p_base + kk * 32, 16, 1024),
+                                 umma_sdesc_sw128(v_base + kk * 2048, kTokTc * 128, 1024), kIdescPV,
+                                 (u > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&sm.pv_done[u & 1]);
+                umma_commit(&sm.empty[u % kStagesTc]);
+                return true;
+            };
+            bool ok = true;
+            for (int t = 0; t < num_tiles && ok; ++t) {
+                const int slot = t % kStagesTc;
+                ok = mbar_wait(&sm.full[slot], (t / kStagesTc) & 1);
+                if (ok && t >= 2)
+                    ok = mbar_wait(&sm.s_free[t & 1], ((t >> 1) - 1) & 1);
+                if (!ok)
+                    break;
+                // a gathered stage was written by cp.async (generic proxy);
+                // the tensor cores read it through the async proxy
+                fence_proxy_async_smem();
+                tc_fence_after();
+                const uint32_t k_base = smem_addr(&sm.kv[slot][0][0]);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    umma_bf16_ss(tmem + (t & 1) * kTokTc,
+                                 umma_sdesc_sw128(q_base + (kk >> 2) * (kColsTc * 128) + (kk & 3) * 32, 16, 1024),
+                                 umma_sdesc_sw128(k_base + (kk >> 2) * (kTokTc * 128) + (kk & 3) * 32, 16, 1024),
+                                 kIdescS, kk > 0 ? 1u : 0u);
+                umma_commit(&sm.s_full[t & 1]);
+                if (t >= 1)
+                    ok = pv(t - 1);
+            }
+            if (ok)
+                pv(num_tiles - 1);
+            // everything issued above has completed before the allocation is freed
+            umma_commit(&sm.mma_done);
+            mbar_wait(&sm.mma_done, 0);
+        }
+        __syncwarp();
+    } else {
+        // ============================================================ softmax
+        const int c = col0 + threadIdx.x;
+        const int lim = c <= last_col ? first_visible + c / G : -1;  // last position column c sees
+        const bool warp_live = __any_sync(FULL, lim >= t_begin);
+        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int t = 0; t < num_tiles; ++t) {
+            if (lane == 0)
+                ok = mbar_wait(&sm.s_full[t & 1], (t >> 1) & 1);
+            if (!__shfl_sync(FULL, ok, 0))
+                break;
+            tc_fence_after();
+            const int t0 = t_begin + t * kTokTc;
+            const int ntok = min(kTokTc, t_end - t0);
+            const int jcount = max(0, min(ntok, lim - t0 + 1));  // tokens of this tile column c sees
+            float x[kTokTc];
+            if (warp_live) {
+                uint32_t s[32];
+                tmem_ld32(tmem + lane_base + (t & 1) * kTokTc, s);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    x[j] = j < jcount ? __uint_as_float(s[j]) * sl2 : -INFINITY;
+                tmem_ld32(tmem + lane_base + (t & 1) * kTokTc + 32, s);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    x[32 + j] = 32 + j < jcount ? __uint_as_float(s[j]) * sl2 : -INFINITY;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.s_free[t & 1]);
+            // the P buffer of this tile was last read by P V of tile t - 2
+            if (t >= 2) {
+                if (lane == 0)
+                    ok = mbar_wait(&sm.pv_done[t & 1], ((t >> 1) - 1) & 1);
+                if (!__shfl_sync(FULL, ok, 0))
+                    break;
+            }
+            if (warp_live) {
+                float mt = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < kTokTc; ++j)
+                    mt = fmaxf(mt, x[j]);
+                float alpha = 1.f;
+                bool rescale = false;
+                if (mt > m_ref + kLazyRescaleLog2) {  // false while the column has seen nothing
+                    if (m_ref != -INFINITY) {
+                        alpha = exp2_approx(m_ref - mt);
+                        rescale = true;
+                    }
+                    m_ref = mt;
+                }
+                l *= alpha;
+                if (__any_sync(FULL, rescale)) {
+                    // O must hold P V of tile t - 1 before it is scaled
+                    if (lane == 0)
+                        ok = mbar_wait(&sm.pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1);
+                    if (!__shfl_sync(FULL, ok, 0))
+                        break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int cc = 0; cc < kD / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem_o + lane_base + cc * 32, o);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                        tmem_st32(tmem_o + lane_base + cc * 32, o);
+                    }
+                    tmem_st_wait();
+                }
+                // P row: 2^(x - m_ref), 0 where masked or while nothing is seen
+                const bool seen = m_ref != -INFINITY;
+                uint8_t *prow = reinterpret_cast<uint8_t *>(&sm.p[t & 1][0]);
+                float lsum = 0.f;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    float e[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        e[u] = seen ? exp2_approx(x[8 * k + u] - m_ref) : 0.f;
+                        lsum += e[u];
+                    }
+                    uint4 w;
+                    w.x = pack_bf16x2(e[0], e[1]);
+                    w.y = pack_bf16x2(e[2], e[3]);
+                    w.z = pack_bf16x2(e[4], e[5]);
+                    w.w = pack_bf16x2(e[6], e[7]);
+                    *reinterpret_cast<uint4 *>(prow + swz(threadIdx.x, k)) = w;
+                }
+                l += lsum;
+                fence_proxy_async_smem();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.p_full[t & 1]);
+        }
+        if (threadIdx.x == 0)
+            grid_launch_dependents();
+        // ---- epilogue: this column's O row -----------------------------------
+        if (ok && lane == 0)
+            ok = mbar_wait(&sm.pv_done[(num_tiles - 1) & 1], ((num_tiles - 1) >> 1) & 1);
+        ok = __shfl_sync(FULL, ok, 0);
+        if (ok && warp_live) {
+            tc_fence_after();
+            const bool valid = c <= last_col;
+            const int64_t qrow = valid ? q0 + c / G : 0;
+            const int j = h * G + c % G;
+#pragma unroll 1
+            for (int cc = 0; cc < kD / 32; ++cc) {
+                uint32_t o[32];
+                __syncwarp();  // the load is warp-collective
+                tmem_ld32(tmem_o + lane_base + cc * 32, o);
+                if (!valid) {
+                } else if (p.num_parts == 1) {
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qrow * p.num_q_heads + j) * kD + cc * 32);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+                        w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+                        w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+                        w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+                        dst[k] = w;
+                    }
+                } else {
+                    const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + part;
+                    float4 *dst = reinterpret_cast<float4 *>(p.part_acc + idx * kD + cc * 32);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
+                                             __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+                    if (cc == 0)
+                        p.part_ml[idx] = make_float2(m_ref, l);
+                }
+            }
+        }
+    }
+    // every role is done with tensor memory before it is freed
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kTcMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemColsTc);
+    }
+}
+
+}  // namespace pa

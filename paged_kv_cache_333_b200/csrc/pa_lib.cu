@@ -15,6 +15,7 @@
 #include <utility>
 
 #include "attend.cuh"
+#include "attend_tc.cuh"
 #include "decode.cuh"
 #include "decode_mma.cuh"
 #include "decode_fp8.cuh"
@@ -29,7 +30,7 @@ thread_local char g_last_cuda_error[256] = "";
 // thread and a call on another do not race.  A call reads each knob once.
 std::atomic<int32_t> g_part_tokens_override{0};
 std::atomic<int32_t> g_decode_kernel{PA_DECODE_KERNEL_MMA};
-
+std::atomic<int32_t> g_attention_kernel{PA_ATTENTION_KERNEL_MMA};
 
 
 int cuda_fail(cudaError_t e, const char *what) {
@@ -106,6 +107,9 @@ struct WorkspaceLayout {
 };
 
 bool decode_kernel_is_mma() { return g_decode_kernel.load(std::memory_order_relaxed) == PA_DECODE_KERNEL_MMA; }
+bool attention_kernel_is_tcgen05() {
+    return g_attention_kernel.load(std::memory_order_relaxed) == PA_ATTENTION_KERNEL_TCGEN05;
+}
 
 WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                  int32_t max_seq_len, int32_t block_size, bool tensor_core_kernel) {
@@ -265,17 +269,19 @@ namespace {
 // (m, l), acc and per-row length arrays when there is more than one
 // partition.
 struct AttendLayout {
+    bool tcgen05;  // attend_tc_kernel (128 columns per CTA), else attend_partition_kernel
     int32_t warps, chunks, part_tokens, num_parts;
     size_t acc_offset, len_offset, total;
 };
 
 AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_query_len, int32_t num_q_heads,
-                           int32_t num_kv_heads, int32_t max_seq_len, int32_t block_size) {
+                           int32_t num_kv_heads, int32_t max_seq_len, int32_t block_size, bool tcgen05) {
     AttendLayout a{};
+    a.tcgen05 = tcgen05;
     const int64_t G = num_q_heads / num_kv_heads;
     const int64_t cols = static_cast<int64_t>(max_query_len) * G;
     a.warps = cols <= 16 ? 2 : 4;  // CTA shape: 16 columns x 4 CTAs/SM, or 32 columns x 2 CTAs/SM
-    const int64_t per_cta = 8 * a.warps;
+    const int64_t per_cta = tcgen05 ? pa::kColsTc : 8 * a.warps;
     a.chunks = static_cast<int32_t>(std::max<int64_t>(1, (cols + per_cta - 1) / per_cta));
     const int64_t units = std::min<int64_t>(INT32_MAX, static_cast<int64_t>(num_reqs) * a.chunks);
     a.part_tokens = choose_part_tokens(static_cast<int32_t>(units), num_kv_heads, max_seq_len, block_size, true);
@@ -291,6 +297,19 @@ AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_que
     return a;
 }
 
+// Split-K: merge the partitions of each query row, with its visible length
+// as that row's sequence length.
+int launch_row_merge(const pa::AttendParams &ap, cudaStream_t stream) {
+    if (ap.d.num_parts <= 1)
+        return PA_OK;
+    pa::DecodeParams md = ap.d;
+    md.seq_lens = ap.row_len;
+    md.num_seqs = ap.num_tokens;
+    const cudaError_t e = launch_pdl(pa::decode_merge_kernel, dim3(md.num_q_heads, std::min(ap.num_tokens, 65535), 1),
+                                     dim3(pa::kD), 0, stream, md);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "decode_merge_kernel launch");
+}
+
 template <int G, int W>
 int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap, int32_t num_kv_heads,
                     cudaStream_t stream) {
@@ -304,16 +323,23 @@ int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Atte
                                stream, tk, tv, ap);
     if (e != cudaSuccess)
         return cuda_fail(e, "attend_partition_kernel launch");
-    if (ap.d.num_parts > 1) {
-        pa::DecodeParams md = ap.d;  // merge per query row, each with its visible length
-        md.seq_lens = ap.row_len;
-        md.num_seqs = ap.num_tokens;
-        e = launch_pdl(pa::decode_merge_kernel, dim3(md.num_q_heads, std::min(ap.num_tokens, 65535), 1),
-                       dim3(pa::kD), 0, stream, md);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "decode_merge_kernel launch");
-    }
-    return PA_OK;
+    return launch_row_merge(ap, stream);
+}
+
+// The tensor-memory variant (attend_tc.cuh): 128 columns per CTA, one CTA per SM.
+template <int G>
+int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap,
+                       int32_t num_kv_heads, cudaStream_t stream) {
+    static std::atomic<bool> done[64] = {};
+    int rc = prepare_kernel(pa::attend_tc_kernel<G>, pa::kAttendTcSmemBytes, done);
+    if (rc)
+        return rc;
+    const dim3 grid(ap.d.num_parts, num_kv_heads, ap.d.num_seqs * ap.chunks);
+    cudaError_t e = launch_pdl(pa::attend_tc_kernel<G>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
+                               stream, tk, tv, ap);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "attend_tc_kernel launch");
+    return launch_row_merge(ap, stream);
 }
 
 pa_cache_t as_cache(const pa_cache_fp8_t *c) {
@@ -661,7 +687,7 @@ size_t pa_attention_workspace_bytes(int32_t num_reqs, int32_t num_tokens, int32_
         num_q_heads <= 0 || max_seq_len < 0 || num_q_heads % cache->num_kv_heads != 0)
         return 0;
     return attend_layout(num_reqs, num_tokens, max_query_len, num_q_heads, cache->num_kv_heads, max_seq_len,
-                         cache->block_size)
+                         cache->block_size, attention_kernel_is_tcgen05())
         .total;
 }
 
@@ -689,7 +715,7 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     if (!std::isfinite(scale))
         return PA_EINVAL;
     const AttendLayout a = attend_layout(num_reqs, num_tokens, max_query_len, num_q_heads, cache->num_kv_heads,
-                                         max_seq_len, cache->block_size);
+                                         max_seq_len, cache->block_size, attention_kernel_is_tcgen05());
     if (static_cast<int64_t>(num_reqs) * a.chunks > 65535 || cache->num_kv_heads > 65535)
         return PA_EUNSUPPORTED;
     if (a.total > 0 && (workspace == nullptr || workspace_bytes < a.total))
@@ -730,6 +756,14 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     ap.max_query_len = max_query_len;
     ap.chunks = a.chunks;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (a.tcgen05) {
+        switch (G) {
+        case 1: return launch_attend_tc_g<1>(tk, tv, ap, cache->num_kv_heads, st);
+        case 2: return launch_attend_tc_g<2>(tk, tv, ap, cache->num_kv_heads, st);
+        case 4: return launch_attend_tc_g<4>(tk, tv, ap, cache->num_kv_heads, st);
+        default: return launch_attend_tc_g<8>(tk, tv, ap, cache->num_kv_heads, st);
+        }
+    }
     const bool w2 = a.warps == 2;
     switch (G) {
     case 1: return w2 ? launch_attend_g<1, 2>(tk, tv, ap, cache->num_kv_heads, st)
@@ -747,6 +781,12 @@ int32_t pa_decode_set_kernel(int32_t kind) {
     if (kind == PA_DECODE_KERNEL_MMA || kind == PA_DECODE_KERNEL_SIMT)
         return g_decode_kernel.exchange(kind);
     return g_decode_kernel.load();
+}
+
+int32_t pa_attention_set_kernel(int32_t kind) {
+    if (kind == PA_ATTENTION_KERNEL_MMA || kind == PA_ATTENTION_KERNEL_TCGEN05)
+        return g_attention_kernel.exchange(kind);
+    return g_attention_kernel.load();
 }
 
 int32_t pa_decode_set_partition_tokens(int32_t tokens) {

@@ -199,3 +199,41 @@ def test_host_side_validation_of_the_remaining_entry_points():
         lib.pa_decode_set_partition_tokens(prev)
     for code, text in ((0, b"ok"), (-1, b"invalid argument"), (-2, b"unsupported"), (-4, b"CUDA"), (9, b"unknown")):
         assert text in lib.pa_status_str(code)
+
+
+def test_attention_kernel_knob_and_the_tensor_memory_chunking():
+    """pa_attention_set_kernel is a process-wide host setting that returns the
+    previous choice; the tensor-memory kernel takes 128 (row, head) columns
+    per CTA instead of 32, which the workspace size shows through the split-K
+    partition heuristic (fewer column chunks -> fewer units -> more, shorter
+    partitions).  Only sizes are computed here: nothing is launched."""
+    from paged_kv_cache_333_b200._abi import (PA_ATTENTION_KERNEL_MMA, PA_ATTENTION_KERNEL_TCGEN05, PaCache,
+                                              lib)
+    c = ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))
+
+    def ws_bytes(rows, parts):
+        cells = rows * 32 * parts
+        acc_off = -(-cells * 8 // 256) * 256
+        len_off = -(-(acc_off + cells * 128 * 4) // 256) * 256
+        return len_off + rows * 4
+
+    R, maxq, L = 8, 64, 32768          # 8 requests of 32K tokens, 64 rows each, G = 4: 256 columns
+    slots = 148 * 4                    # no device: B200's SM count x the heuristic's 4 CTAs per SM
+
+    def parts(units):
+        part = max(640, -(-(L * units * 8) // (16 * slots)))
+        part = -(-part // 64) * 64
+        return -(-L // part)
+
+    prev = lib.pa_attention_set_kernel(PA_ATTENTION_KERNEL_MMA)
+    try:
+        assert lib.pa_attention_workspace_bytes(R, R * maxq, maxq, 32, L, c) == ws_bytes(R * maxq, parts(R * 8))
+        assert lib.pa_attention_set_kernel(PA_ATTENTION_KERNEL_TCGEN05) == PA_ATTENTION_KERNEL_MMA
+        assert lib.pa_attention_set_kernel(9) == PA_ATTENTION_KERNEL_TCGEN05   # ignored
+        assert lib.pa_attention_workspace_bytes(R, R * maxq, maxq, 32, L, c) == ws_bytes(R * maxq, parts(R * 2))
+        assert parts(R * 2) == 52 and parts(R * 8) == 19
+        # chat lengths stay one partition either way: no scratch
+        assert lib.pa_attention_workspace_bytes(64, 64 * 16, 16, 32, 612, c) == 0
+    finally:
+        lib.pa_attention_set_kernel(prev)
+    assert lib.pa_attention_set_kernel(prev) == prev == PA_ATTENTION_KERNEL_MMA
