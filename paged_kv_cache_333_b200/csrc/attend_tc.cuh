@@ -95,6 +95,64 @@ static_assert(umma_sdesc_sw128(0x2000u, 8192u, 1024u) == 0x4000404002000200ull, 
 constexpr uint32_t kIdescS = umma_idesc_bf16(kColsTc, kTokTc, false, false);
 constexpr uint32_t kIdescPV = umma_idesc_bf16(kColsTc, kD, false, true);
 
+// ---------------------------------------------------------------- operand views
+// Byte offsets (from 1024-aligned tile bases) and strides of the four MMA
+// operands, k-step kk covering 16 values of the reduction dimension.
+constexpr uint32_t kQHalfBytes = kColsTc * 128;  // Q: [dims 0-63 | 64-127][128 columns x 128 B]
+constexpr uint32_t kKvQuarterBytes = kTokTc * 128;  // K lo, K hi, V lo, V hi: [64 tokens x 128 B]
+constexpr uint32_t kSbo = 1024;                  // 8 rows of 128 B
+constexpr uint32_t kLboK = 16;                   // unused by swizzled K-major operands
+__host__ __device__ constexpr uint32_t q_step(int kk) { return (kk >> 2) * kQHalfBytes + (kk & 3) * 32; }
+__host__ __device__ constexpr uint32_t k_step(int kk) { return (kk >> 2) * kKvQuarterBytes + (kk & 3) * 32; }
+__host__ __device__ constexpr uint32_t p_step(int kk) { return kk * 32; }
+__host__ __device__ constexpr uint32_t v_step(int kk) { return kk * 16 * 128; }
+constexpr uint32_t kLboV = kKvQuarterBytes;      // V's dims 64-127 (V hi) after dims 0-63 (V lo)
+
+// Where the tensor cores read element (mn, k) of a bf16 operand given by a
+// 128-byte-swizzle descriptor, in the canonical layouts of the tcgen05
+// matrix descriptors (T = 8 bf16 = 16 bytes; CUTLASS cute/atom/
+// mma_traits_sm100.hpp, make_umma_desc):
+//   K-major  ((8, m), (T, 2)) : ((8T, SBO), (1, T))
+//   MN-major ((T, 8, m), (8, k)) : ((1, T, LBO), (8T, SBO))
+// followed by the 128-byte swizzle of the address (bits 4-6 ^= bits 7-9).
+__host__ __device__ constexpr uint32_t sw128_read(uint32_t start, uint32_t lbo, uint32_t sbo, bool mn_major,
+                                                  int mn, int k) {
+    const uint32_t off = mn_major ? 2u * (mn % 64) + (mn / 64) * lbo + (k % 8) * 128u + (k / 8) * sbo
+                                  : (mn % 8) * 128u + (mn / 8) * sbo + 2u * k;
+    const uint32_t a = start + off;
+    return a ^ (((a >> 7) & 7u) << 4);
+}
+// Where the TMA boxes (128-byte swizzle) and swz() put element (row, col) of
+// a tile stored as [col / 64][rows x 128 B], `half` bytes apart.
+__host__ __device__ constexpr uint32_t sw128_written(uint32_t half, int row, int col) {
+    return (col / 64) * half + static_cast<uint32_t>(row * 128 + ((((col % 64) / 8) ^ (row & 7)) << 4)) +
+           2u * (col % 8);
+}
+// Every element each k-step of the four operands reads is the element the
+// kernel wrote there: Q[column][dim], K[token][dim], P[column][token],
+// V[token][dim] (V read MN-major: mn = dim, k = token).
+__host__ __device__ constexpr bool operand_views_agree() {
+    for (int kk = 0; kk < kD / 16; ++kk)
+        for (int mn = 0; mn < kColsTc; ++mn)
+            for (int kl = 0; kl < 16; ++kl) {
+                if (sw128_read(q_step(kk), kLboK, kSbo, false, mn, kl) != sw128_written(kQHalfBytes, mn, 16 * kk + kl))
+                    return false;
+                if (mn < kTokTc &&
+                    sw128_read(k_step(kk), kLboK, kSbo, false, mn, kl) != sw128_written(kKvQuarterBytes, mn, 16 * kk + kl))
+                    return false;
+            }
+    for (int kk = 0; kk < kTokTc / 16; ++kk)
+        for (int mn = 0; mn < kColsTc; ++mn)
+            for (int kl = 0; kl < 16; ++kl) {
+                if (sw128_read(p_step(kk), kLboK, kSbo, false, mn, kl) != sw128_written(0, mn, 16 * kk + kl))
+                    return false;
+                if (sw128_read(v_step(kk), kLboV, kSbo, true, mn, kl) != sw128_written(kKvQuarterBytes, 16 * kk + kl, mn))
+                    return false;
+            }
+    return true;
+}
+static_assert(operand_views_agree(), "MMA operand descriptors must read what the tiles hold");
+
 // ---------------------------------------------------------------- tcgen05 PTX
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),
@@ -376,8 +434,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const uint32_t v_base = smem_addr(&sm.kv[u % kStagesTc][2][0]);
 #pragma unroll
                 for (int kk = 0; kk < kTokTc / 16; ++kk)
-                    umma_bf16_ss(tmem_o, umma_sdesc_sw128(p_base + kk * 32, 16, 1024),
-                                 umma_sdesc_sw128(v_base + kk * 2048, kTokTc * 128, 1024), kIdescPV,
+                    umma_bf16_ss(tmem_o, umma_sdesc_sw128(p_base + p_step(kk), kLboK, kSbo),
+                                 umma_sdesc_sw128(v_base + v_step(kk), kLboV, kSbo), kIdescPV,
                                  (u > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&sm.pv_done[u & 1]);
                 umma_commit(&sm.empty[u % kStagesTc]);
@@ -398,10 +456,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const uint32_t k_base = smem_addr(&sm.kv[slot][0][0]);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    umma_bf16_ss(tmem + (t & 1) * kTokTc,
-                                 umma_sdesc_sw128(q_base + (kk >> 2) * (kColsTc * 128) + (kk & 3) * 32, 16, 1024),
-                                 umma_sdesc_sw128(k_base + (kk >> 2) * (kTokTc * 128) + (kk & 3) * 32, 16, 1024),
-                                 kIdescS, kk > 0 ? 1u : 0u);
+                    umma_bf16_ss(tmem + (t & 1) * kTokTc, umma_sdesc_sw128(q_base + q_step(kk), kLboK, kSbo),
+                                 umma_sdesc_sw128(k_base + k_step(kk), kLboK, kSbo), kIdescS, kk > 0 ? 1u : 0u);
                 umma_commit(&sm.s_full[t & 1]);
                 if (t >= 1)
                     ok = pv(t - 1);
