@@ -112,16 +112,25 @@ def _check(rc: int, what: str) -> None:
 def _stream_ptr(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
+    dev = getattr(stream, "device", None)
+    if dev is not None and dev.index != torch.cuda.current_device():
+        raise ValueError(f"stream is on {dev}, but the current CUDA device is cuda:{torch.cuda.current_device()}")
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
 def _dev(t: torch.Tensor, name: str, dtype) -> int:
+    """Device pointer of a contiguous CUDA tensor of `dtype` on the current
+    device: the library launches on the current device, where a pointer into
+    another GPU's memory would be an illegal address."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}; call under torch.cuda.device({t.device})")
     return t.data_ptr()
 
 

@@ -237,3 +237,39 @@ def test_attention_kernel_knob_and_the_tensor_memory_chunking():
     finally:
         lib.pa_attention_set_kernel(prev)
     assert lib.pa_attention_set_kernel(prev) == prev == PA_ATTENTION_KERNEL_MMA
+
+
+def test_binding_refuses_tensors_of_another_device(monkeypatch):
+    """The library launches on the current device; the binding refuses a
+    tensor (or stream) that lives on another GPU instead of passing its
+    pointer.  Checked on CPU with a tensor that reports cuda:1 while the
+    current device is cuda:0 (nothing is launched)."""
+    import torch
+    from paged_kv_cache_333_b200 import _abi
+
+    class OnGpu1(torch.Tensor):
+        @property
+        def is_cuda(self):
+            return True
+
+        @property
+        def device(self):
+            return torch.device("cuda", 1)
+
+    t = torch.Tensor._make_subclass(OnGpu1, torch.zeros(8, dtype=torch.bfloat16))
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="current CUDA device is cuda:0"):
+        _abi._dev(t, "q", torch.bfloat16)
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 1)
+    assert _abi._dev(t, "q", torch.bfloat16) == t.data_ptr()
+    with pytest.raises(TypeError, match="must be torch.int32"):
+        _abi._dev(t, "q", torch.int32)
+
+    class Stream1:
+        device = torch.device("cuda", 1)
+        cuda_stream = 1234
+    assert _abi._stream_ptr(Stream1()) == 1234
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    with pytest.raises(ValueError, match="stream is on cuda:1"):
+        _abi._stream_ptr(Stream1())
+    assert _abi._stream_ptr(5678) == 5678      # a raw handle: nothing to check
