@@ -143,6 +143,8 @@ int pa_pool_append(pa_pool_t *pool, int64_t seq_id, int64_t n_tokens) {
         return PA_POOL_ENOSEQ;
     Seq &s = it->second;
     const int64_t B = pool->block_size;
+    if (n_tokens > pool->num_blocks * B - s.len)
+        return PA_POOL_ENOSPACE;  // more than the whole pool holds (and len + n_tokens cannot overflow)
     const int64_t needed = cdiv(s.len + n_tokens, B) - static_cast<int64_t>(s.blocks.size());
     const bool partial = !s.blocks.empty() && s.len % B != 0 && n_tokens > 0;
     bool cow;
@@ -191,6 +193,8 @@ int pa_pool_append_batch(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_se
         if (it == pool->seqs.end())
             return PA_POOL_ENOSEQ;
         const Seq &s = it->second;
+        if (n_tokens > pool->num_blocks * B - s.len)
+            return PA_POOL_ENOSPACE;
         const int64_t needed = cdiv(s.len + n_tokens, B) - static_cast<int64_t>(s.blocks.size());
         const bool partial = !s.blocks.empty() && s.len % B != 0 && n_tokens > 0;
         bool cow;

@@ -256,6 +256,25 @@ def test_errors_and_state_unchanged():
     pool.check()
 
 
+@pytest.mark.parametrize("n", [17, 2**40, 2**62, 2**63 - 1])
+def test_appends_beyond_the_pool_are_refused_without_overflow(n):
+    """No sequence can hold more than num_blocks * block_size tokens: such an
+    append (single or batched) is refused with the pool unchanged, however
+    large the count (the length arithmetic never overflows)."""
+    pool = BlockPool(4, 4)
+    pool.create(1)
+    pool.create(2)
+    assert pool.append(1, 3)
+    free = pool.num_free()
+    assert not pool.append(1, n)
+    assert not pool.append_batch([1, 2], n)
+    assert not pool.append(2, n)
+    assert pool.num_free() == free and pool.seq_len(1) == 3 and pool.seq_len(2) == 0
+    pool.check()
+    assert pool.append(1, 13)  # exactly the rest of the pool still fits
+    assert pool.num_free() == 0
+
+
 def test_step_slots_and_padding():
     pool = BlockPool(16, 4)
     for sid, n in [(1, 5), (2, 8)]:
