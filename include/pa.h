@@ -43,7 +43,9 @@ enum {
     PA_OK = 0,
     PA_EINVAL = -1,       /* null pointer, negative size, num_q_heads % num_kv_heads != 0 */
     PA_EUNSUPPORTED = -2, /* head_dim != 128, block_size not a power of two in [1, 64],
-                             group size not in {1, 2, 4, 8}, pointer not 16-byte aligned */
+                             group size not in {1, 2, 4, 8}, pointer not 16-byte aligned,
+                             num_kv_heads > 65535, or a count past the launch limits
+                             (more than INT32_MAX tokens or copy pairs) */
     PA_EWORKSPACE = -3,   /* workspace smaller than pa_decode_workspace_bytes() */
     PA_ECUDA = -4         /* a CUDA call or launch failed (see pa_last_cuda_error) */
 };

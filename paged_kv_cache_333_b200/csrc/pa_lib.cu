@@ -43,7 +43,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int check_cache(const pa_cache_t *c) {
     if (!c || !c->k_cache || !c->v_cache || c->num_blocks <= 0 || c->num_kv_heads <= 0)
         return PA_EINVAL;
-    if (c->head_dim != pa::kD)
+    if (c->head_dim != pa::kD || c->num_kv_heads > 65535)  // heads: a grid dimension, and int row sizes
         return PA_EUNSUPPORTED;
     const int32_t b = c->block_size;
     if (b < 1 || b > 64 || (b & (b - 1)) != 0)
@@ -443,6 +443,8 @@ int pa_write_kv(const void *k, const void *v, const int64_t *slot_mapping, int64
     if (!aligned16(k) || !aligned16(v))
         return PA_EUNSUPPORTED;
     const int row_vecs = cache->num_kv_heads * cache->head_dim * 2 / 16;
+    if (num_tokens > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
     const int64_t warps = num_tokens * 2;
     const int64_t blocks = (warps * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
     if (blocks > INT32_MAX)
@@ -464,6 +466,8 @@ int pa_compute_slot_mapping(const int64_t *positions, const int32_t *req_indices
         return PA_OK;
     if (!positions || !req_indices || !slot_mapping || (num_reqs > 0 && !block_tables))
         return PA_EINVAL;
+    if (num_tokens > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
     const int64_t blocks = (num_tokens + pa::kSlotThreads - 1) / pa::kSlotThreads;
     if (blocks > INT32_MAX)
         return PA_EUNSUPPORTED;
@@ -507,6 +511,8 @@ int pa_write_kv_positions(const void *k, const void *v, const int64_t *positions
     if (!aligned16(k) || !aligned16(v))
         return PA_EUNSUPPORTED;
     const int row_vecs = cache->num_kv_heads * cache->head_dim * 2 / 16;
+    if (num_tokens > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
     const int64_t blocks = (num_tokens * 2 * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
     if (blocks > INT32_MAX)
         return PA_EUNSUPPORTED;
@@ -530,6 +536,8 @@ int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs, int64_
         return PA_OK;
     if (!src_dst_pairs)
         return PA_EINVAL;
+    if (num_pairs > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
     const int64_t block_vecs =
         static_cast<int64_t>(cache->block_size) * cache->num_kv_heads * cache->head_dim * 2 / 16;
     const int chunks = static_cast<int>((block_vecs + pa::kCopyChunkVecs - 1) / pa::kCopyChunkVecs);
@@ -562,6 +570,8 @@ int pa_copy_blocks_layers(const pa_cache_t *caches, int32_t num_layers, const in
         return PA_OK;
     if (!src_dst_pairs)
         return PA_EINVAL;
+    if (num_pairs > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
     const pa_cache_t *c = &caches[0];
     const int64_t block_vecs = static_cast<int64_t>(c->block_size) * c->num_kv_heads * c->head_dim * 2 / 16;
     const int chunks = static_cast<int>((block_vecs + pa::kCopyChunkVecs - 1) / pa::kCopyChunkVecs);
@@ -589,6 +599,8 @@ int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_mapping, i
     if (!aligned16(k) || !aligned16(v))
         return PA_EUNSUPPORTED;
     const int row_vecs = cache->num_kv_heads * cache->head_dim * 2 / 16;
+    if (num_tokens > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
     const int64_t blocks = (num_tokens * 2 * 32 + pa::kWriteThreads - 1) / pa::kWriteThreads;
     if (blocks > INT32_MAX)
         return PA_EUNSUPPORTED;

@@ -273,3 +273,25 @@ def test_binding_refuses_tensors_of_another_device(monkeypatch):
     with pytest.raises(ValueError, match="stream is on cuda:1"):
         _abi._stream_ptr(Stream1())
     assert _abi._stream_ptr(5678) == 5678      # a raw handle: nothing to check
+
+
+def test_counts_past_the_launch_limits_are_refused_on_the_host():
+    """Token and pair counts above INT32_MAX, and more than 65535 KV heads,
+    are refused before any size arithmetic could overflow (fake pointers:
+    nothing is launched)."""
+    from paged_kv_cache_333_b200._abi import PA_EUNSUPPORTED, PaCache, PaCacheFp8, lib
+    c = ctypes.byref(PaCache(16, 16, 64, 16, 2, 128))
+    for n in (2**31, 2**40, 2**62, 2**63 - 1):
+        assert lib.pa_write_kv(16, 16, 16, n, c, None) == PA_EUNSUPPORTED
+        assert lib.pa_write_kv_positions(16, 16, 16, 16, n, 16, 8, 2, c, None) == PA_EUNSUPPORTED
+        assert lib.pa_compute_slot_mapping(16, 16, n, 16, 8, 2, 16, 64, 16, None) == PA_EUNSUPPORTED
+        assert lib.pa_write_kv_fp8(16, 16, 16, n, ctypes.byref(PaCacheFp8(16, 16, 64, 16, 2, 128, 1.0, 1.0)),
+                                   None) == PA_EUNSUPPORTED
+        assert lib.pa_copy_blocks(c, 16, n, None) == PA_EUNSUPPORTED
+        assert lib.pa_copy_blocks_layers((PaCache * 2)(PaCache(16, 16, 64, 16, 2, 128),
+                                                       PaCache(32, 32, 64, 16, 2, 128)), 2, 16, n,
+                                         None) == PA_EUNSUPPORTED
+    wide = ctypes.byref(PaCache(16, 16, 4, 16, 70000, 128))
+    assert lib.pa_write_kv(16, 16, 16, 1, wide, None) == PA_EUNSUPPORTED
+    assert lib.pa_copy_blocks(wide, 16, 1, None) == PA_EUNSUPPORTED
+    assert lib.pa_decode(16, wide, 16, 4, 16, 1, 64, 70000, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
