@@ -229,10 +229,11 @@ def algorithmic_bytes(st, rows_per_seq: int = 1) -> dict:
 
 def host_pool_step_us(w, steps: int = 200) -> dict:
     """Host time of the scheduler-side step (the block table and slot
-    mapping build) on the C++ pool: append one token to every sequence in one
-    call, take the queued copy pairs, and build the step's slot mapping and
-    lengths, with the block table kept across steps and updated append-only.  Timed on a fresh pool laid out as the workload
-    (the timed device step uses its own)."""
+    mapping build) on the C++ pool, as one pa_pool_step call: append one
+    token to every sequence, take the queued copy pairs, build the step's
+    slot mapping and lengths, and update the block table kept across steps
+    (append-only).  Output buffers are reused across steps.  Timed on a fresh
+    pool laid out as the workload (the timed device step uses its own)."""
     from paged_kv_cache_333_b200.pool import BlockPool
     sh = w.shape
     pool = BlockPool(sh.num_blocks, sh.block_size, w.free_order, "shared")
@@ -241,24 +242,22 @@ def host_pool_step_us(w, steps: int = 200) -> dict:
         w.suffix_ops(pool)
     pool.take_cow_pairs()
     ids = np.asarray(w.seq_ids, dtype=np.int64)
+    S = len(ids)
     width = max(pool.num_blocks_of(int(i)) for i in ids) + steps // sh.block_size + 2
-    table = np.full((len(ids), width), -1, dtype=np.int32)  # kept across steps, updated append-only
-    synced = np.zeros(len(ids), dtype=np.int32)
+    table = np.full((S, width), -1, dtype=np.int32)  # kept across steps, updated append-only
+    synced = np.zeros(S, dtype=np.int32)
     pool.block_table_update(ids, table, synced)
+    slots, lens, pairs = np.empty(S, np.int64), np.empty(S, np.int32), np.empty((S, 2), np.int64)
     done = 0
     t0 = time.perf_counter()
     for _ in range(steps):
-        if not pool.append_batch(ids, 1):
+        if pool.step(ids, 1, table, synced, slots, lens, pairs) is None:
             break
-        pool.take_cow_pairs()
-        pool.step_slots(ids, 1)
-        pool.block_table_update(ids, table, synced)
-        pool.seq_lens(ids)
         done += 1
     dt = time.perf_counter() - t0
-    return {"us": round(dt / max(done, 1) * 1e6, 2), "steps": done, "sequences": int(len(ids)),
-            "what": "append_batch (1 token per sequence) + copy pairs + slot mapping + block table (updated "
-                    "append-only) + lengths, C++ pool through ctypes, one host thread"}
+    return {"us": round(dt / max(done, 1) * 1e6, 2), "steps": done, "sequences": int(S),
+            "what": "pa_pool_step: append 1 token per sequence + copy pairs + slot mapping + block table "
+                    "(updated append-only) + lengths, one ctypes call, one host thread"}
 
 
 # --------------------------------------------------------------------------- ours

@@ -82,6 +82,22 @@ int pa_pool_append(pa_pool_t *pool, int64_t seq_id, int64_t n_tokens);
  * PA_POOL_ENOSPACE and nothing changed.  PA_POOL_EINVAL for a sequence listed
  * twice; PA_POOL_ENOSEQ for an unknown one (nothing changed). */
 int pa_pool_append_batch(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens);
+/* The whole host side of a decode step in one call: pa_pool_append_batch,
+ * then pa_pool_take_copies, pa_pool_step_slots, pa_pool_block_table_update
+ * and pa_pool_seq_lens over the same sequences, with the same results.
+ *   pairs_out   [pairs_capacity][2] int64: every queued copy pair (earlier
+ *               ones first); *num_pairs receives their count.
+ *   slots_out   [num_seqs * n_tokens] int64: the slots of each sequence's
+ *               last n_tokens positions, in call order.
+ *   table, synced, width, as pa_pool_block_table_update (pad already in place).
+ *   lens_out    [num_seqs] int32 lengths after the step.
+ * All or nothing: every check is made before anything changes.
+ * PA_POOL_ENOSPACE (too few free blocks), PA_POOL_ENOSEQ, PA_POOL_EINVAL
+ * (a sequence listed twice, or synced[r] past the sequence's blocks),
+ * PA_POOL_ERANGE (pairs_capacity, width or an int32 length too small). */
+int pa_pool_step(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens, int64_t *pairs_out,
+                 int64_t pairs_capacity, int64_t *num_pairs, int64_t *slots_out, int32_t width, int32_t *table,
+                 int32_t *synced, int32_t *lens_out);
 /* dst becomes a new sequence sharing every block of src (refcount + 1). */
 int pa_pool_fork(pa_pool_t *pool, int64_t src, int64_t dst);
 /* Drop the sequence; its blocks are freed in reverse order. */

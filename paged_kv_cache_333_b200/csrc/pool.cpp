@@ -22,6 +22,7 @@ struct Seq {
     std::vector<int32_t> blocks;
     int64_t len = 0;
     bool tail_owned = true;  // false while the tail block is inherited from a fork
+    uint64_t batch = 0;      // stamp of the last batch call that listed the sequence
 };
 
 // Ring buffer holding at most `cap` block ids; head() is the next to allocate.
@@ -66,10 +67,17 @@ struct pa_pool {
     FreeRing free_q;
     std::unordered_map<int64_t, Seq> seqs;
     std::vector<std::pair<int32_t, int32_t>> pending;
+    // Scratch of the batch calls, kept to avoid allocating per call: the
+    // listed sequences in order, and per block the owner references earlier
+    // appends of the batch move off it (reset before each call returns).
+    uint64_t batch_epoch = 0;
+    std::vector<Seq *> batch;
+    std::vector<int32_t> moved;
+    std::vector<int32_t> moved_touched;
 
     pa_pool(int64_t nb, int32_t bs, int32_t r)
         : num_blocks(nb), block_size(bs), rule(r), ref(static_cast<size_t>(nb), 0),
-          pin(static_cast<size_t>(nb), 0), free_q(nb) {}
+          pin(static_cast<size_t>(nb), 0), free_q(nb), moved(static_cast<size_t>(nb), 0) {}
 
     // Pop n blocks from the head of the free queue; each gets refcount 1.
     void take(int64_t n, std::vector<int32_t> &out) {
@@ -95,6 +103,137 @@ struct pa_pool {
             free_q.push_front(run[i]);
     }
 };
+
+namespace {
+
+// What appending n tokens to s takes: new blocks, and whether the partial
+// tail is copied first.  Shared rule: the tail is copied while another table
+// still names it; `moved_off_tail` counts owner references that earlier
+// appends of the same batch will have moved off it.  Inherited rule: while
+// the sequence has not written its forked tail.
+struct AppendPlan {
+    int64_t needed;
+    bool cow;
+};
+
+AppendPlan plan_append(const pa_pool &pool, const Seq &s, int64_t n_tokens, int32_t moved_off_tail) {
+    const int64_t B = pool.block_size;
+    AppendPlan a;
+    a.needed = cdiv(s.len + n_tokens, B) - static_cast<int64_t>(s.blocks.size());
+    const bool partial = !s.blocks.empty() && s.len % B != 0 && n_tokens > 0;
+    if (pool.rule == PA_COW_SHARED)
+        a.cow = partial && pool.ref[static_cast<size_t>(s.blocks.back())] - moved_off_tail > 1;
+    else
+        a.cow = partial && !s.tail_owned;
+    return a;
+}
+
+bool too_long(const pa_pool &pool, const Seq &s, int64_t n_tokens) {
+    // more than the whole pool holds (this also keeps len + n_tokens in range)
+    return n_tokens > pool.num_blocks * pool.block_size - s.len;
+}
+
+// Carry out an append whose blocks the caller has checked are free.
+void apply_append(pa_pool &pool, Seq &s, int64_t n_tokens, const AppendPlan &a) {
+    if (a.cow) {
+        const int32_t src = s.blocks.back();
+        const int32_t dst = pool.free_q.pop_front();
+        pool.ref[static_cast<size_t>(dst)] = 1;
+        // The sequence stops owning src; both ends stay pinned until the
+        // copy is handed to the device.
+        pool.ref[static_cast<size_t>(src)] -= 1;
+        pool.pin[static_cast<size_t>(src)] += 1;
+        pool.pin[static_cast<size_t>(dst)] += 1;
+        s.blocks.back() = dst;
+        pool.pending.emplace_back(src, dst);
+        s.tail_owned = true;
+    }
+    if (a.needed > 0) {
+        pool.take(a.needed, s.blocks);
+        s.tail_owned = true;
+    }
+    s.len += n_tokens;
+}
+
+// Dry run of appending n_tokens to each listed sequence in call order, with
+// the copy-on-write decisions of the earlier ones applied (a copy takes a
+// sequence off its shared tail, which a later sharer may then own alone).
+// Leaves the sequences in pool.batch; adds up the free blocks and the copies
+// the appends need.  Changes no visible state.
+int plan_batch(pa_pool &pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens, int64_t &blocks,
+               int64_t &copies) {
+    const uint64_t stamp = ++pool.batch_epoch;
+    pool.batch.clear();
+    pool.moved_touched.clear();
+    blocks = copies = 0;
+    int rc = PA_POOL_OK;
+    for (int32_t i = 0; i < num_seqs; ++i) {
+        auto it = pool.seqs.find(seq_ids[i]);
+        if (it == pool.seqs.end()) {
+            rc = PA_POOL_ENOSEQ;
+            break;
+        }
+        Seq &s = it->second;
+        if (s.batch == stamp) {
+            rc = PA_POOL_EINVAL;  // a sequence listed twice
+            break;
+        }
+        s.batch = stamp;
+        if (too_long(pool, s, n_tokens)) {
+            rc = PA_POOL_ENOSPACE;
+            break;
+        }
+        const int32_t tail = s.blocks.empty() ? -1 : s.blocks.back();
+        const AppendPlan a = plan_append(pool, s, n_tokens, tail >= 0 ? pool.moved[static_cast<size_t>(tail)] : 0);
+        if (a.cow && pool.rule == PA_COW_SHARED) {
+            if (pool.moved[static_cast<size_t>(tail)]++ == 0)
+                pool.moved_touched.push_back(tail);
+        }
+        blocks += a.needed + (a.cow ? 1 : 0);
+        copies += a.cow ? 1 : 0;
+        pool.batch.push_back(&s);
+    }
+    for (int32_t b : pool.moved_touched)
+        pool.moved[static_cast<size_t>(b)] = 0;
+    return rc;
+}
+
+// Append to every sequence of pool.batch (after a successful plan_batch
+// whose blocks are free): each decision is taken again on the live state,
+// which by then matches the dry run's.
+void apply_batch(pa_pool &pool, int64_t n_tokens) {
+    for (Seq *s : pool.batch)
+        apply_append(pool, *s, n_tokens, plan_append(pool, *s, n_tokens, 0));
+}
+
+// Move the queued pairs to pairs_out (capacity checked by the caller) and
+// drop the pins their endpoints held.
+int64_t take_copies(pa_pool &pool, int64_t *pairs_out) {
+    const int64_t n = static_cast<int64_t>(pool.pending.size());
+    std::vector<std::pair<int32_t, int32_t>> taken;
+    taken.swap(pool.pending);
+    for (int64_t i = 0; i < n; ++i) {
+        pairs_out[2 * i] = taken[static_cast<size_t>(i)].first;
+        pairs_out[2 * i + 1] = taken[static_cast<size_t>(i)].second;
+        const int32_t ends[2] = {taken[static_cast<size_t>(i)].first, taken[static_cast<size_t>(i)].second};
+        pool.release_refs(ends, 2, pool.pin);
+    }
+    taken.clear();
+    taken.swap(pool.pending);  // keep the capacity for the next step
+    return n;
+}
+
+// Rewrite the entries of a table row that can have changed since `synced`
+// of them were written: the old tail (a copy-on-write may have redirected
+// it) and every entry after it.
+void update_row(const Seq &s, int32_t *row, int32_t &synced) {
+    const int32_t n = static_cast<int32_t>(s.blocks.size());
+    const int32_t from = synced > 0 ? synced - 1 : 0;
+    std::copy(s.blocks.begin() + from, s.blocks.end(), row + from);
+    synced = n;
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -142,78 +281,63 @@ int pa_pool_append(pa_pool_t *pool, int64_t seq_id, int64_t n_tokens) {
     if (it == pool->seqs.end())
         return PA_POOL_ENOSEQ;
     Seq &s = it->second;
-    const int64_t B = pool->block_size;
-    if (n_tokens > pool->num_blocks * B - s.len)
-        return PA_POOL_ENOSPACE;  // more than the whole pool holds (and len + n_tokens cannot overflow)
-    const int64_t needed = cdiv(s.len + n_tokens, B) - static_cast<int64_t>(s.blocks.size());
-    const bool partial = !s.blocks.empty() && s.len % B != 0 && n_tokens > 0;
-    bool cow;
-    if (pool->rule == PA_COW_SHARED)
-        cow = partial && pool->ref[static_cast<size_t>(s.blocks.back())] > 1;
-    else
-        cow = partial && !s.tail_owned;
-    if (needed + (cow ? 1 : 0) > pool->free_q.size())
+    if (too_long(*pool, s, n_tokens))
         return PA_POOL_ENOSPACE;
-    if (cow) {
-        const int32_t src = s.blocks.back();
-        std::vector<int32_t> got;
-        pool->take(1, got);
-        const int32_t dst = got[0];
-        // The sequence stops owning src; both ends stay pinned until the
-        // copy is handed to the device.
-        pool->ref[static_cast<size_t>(src)] -= 1;
-        pool->pin[static_cast<size_t>(src)] += 1;
-        pool->pin[static_cast<size_t>(dst)] += 1;
-        s.blocks.back() = dst;
-        pool->pending.emplace_back(src, dst);
-        s.tail_owned = true;
-    }
-    if (needed > 0) {
-        pool->take(needed, s.blocks);
-        s.tail_owned = true;
-    }
-    s.len += n_tokens;
+    const AppendPlan a = plan_append(*pool, s, n_tokens, 0);
+    if (a.needed + (a.cow ? 1 : 0) > pool->free_q.size())
+        return PA_POOL_ENOSPACE;
+    apply_append(*pool, s, n_tokens, a);
     return PA_POOL_OK;
 }
 
 int pa_pool_append_batch(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens) {
     if (!pool || n_tokens < 0 || num_seqs < 0 || (num_seqs > 0 && !seq_ids))
         return PA_POOL_EINVAL;
-    // Dry run in call order: the blocks each append needs, with the copy-on-
-    // write decisions of the earlier ones applied (a copy takes the sequence
-    // off its shared tail, which a later sharer may then own alone).
-    const int64_t B = pool->block_size;
-    std::unordered_map<int32_t, int32_t> dropped;  // owner refs earlier copies removed
-    std::unordered_map<int64_t, bool> seen;
-    int64_t total = 0;
-    for (int32_t i = 0; i < num_seqs; ++i) {
-        if (!seen.emplace(seq_ids[i], true).second)
-            return PA_POOL_EINVAL;  // a sequence listed twice
-        auto it = pool->seqs.find(seq_ids[i]);
-        if (it == pool->seqs.end())
-            return PA_POOL_ENOSEQ;
-        const Seq &s = it->second;
-        if (n_tokens > pool->num_blocks * B - s.len)
-            return PA_POOL_ENOSPACE;
-        const int64_t needed = cdiv(s.len + n_tokens, B) - static_cast<int64_t>(s.blocks.size());
-        const bool partial = !s.blocks.empty() && s.len % B != 0 && n_tokens > 0;
-        bool cow;
-        if (pool->rule == PA_COW_SHARED) {
-            const int32_t tail = partial ? s.blocks.back() : -1;
-            cow = partial && pool->ref[static_cast<size_t>(tail)] - dropped[tail] > 1;
-            if (cow)
-                dropped[tail] += 1;
-        } else {
-            cow = partial && !s.tail_owned;
-        }
-        total += needed + (cow ? 1 : 0);
-    }
-    if (total > pool->free_q.size())
+    int64_t blocks = 0, copies = 0;
+    const int rc = plan_batch(*pool, seq_ids, num_seqs, n_tokens, blocks, copies);
+    if (rc != PA_POOL_OK)
+        return rc;
+    if (blocks > pool->free_q.size())
         return PA_POOL_ENOSPACE;
-    for (int32_t i = 0; i < num_seqs; ++i) {
-        const int rc = pa_pool_append(pool, seq_ids[i], n_tokens);
-        if (rc != PA_POOL_OK)
-            return rc;  // not reached: the dry run counted every block
+    apply_batch(*pool, n_tokens);
+    return PA_POOL_OK;
+}
+
+int pa_pool_step(pa_pool_t *pool, const int64_t *seq_ids, int32_t num_seqs, int64_t n_tokens, int64_t *pairs_out,
+                 int64_t pairs_capacity, int64_t *num_pairs, int64_t *slots_out, int32_t width, int32_t *table,
+                 int32_t *synced, int32_t *lens_out) {
+    if (!pool || n_tokens < 0 || num_seqs < 0 || width < 0 || pairs_capacity < 0 || !num_pairs ||
+        (num_seqs > 0 && (!seq_ids || !table || !synced || !lens_out || (n_tokens > 0 && !slots_out))))
+        return PA_POOL_EINVAL;
+    int64_t blocks = 0, copies = 0;
+    int rc = plan_batch(*pool, seq_ids, num_seqs, n_tokens, blocks, copies);
+    if (rc != PA_POOL_OK)
+        return rc;
+    if (blocks > pool->free_q.size())
+        return PA_POOL_ENOSPACE;
+    const int64_t npairs = static_cast<int64_t>(pool->pending.size()) + copies;
+    if (npairs > pairs_capacity || (npairs > 0 && !pairs_out))
+        return PA_POOL_ERANGE;
+    const int64_t B = pool->block_size;
+    for (int32_t r = 0; r < num_seqs; ++r) {
+        const Seq &s = *pool->batch[static_cast<size_t>(r)];
+        if (cdiv(s.len + n_tokens, B) > width || synced[r] < 0 || synced[r] > width || s.len + n_tokens > INT32_MAX)
+            return PA_POOL_ERANGE;
+        if (synced[r] > static_cast<int64_t>(s.blocks.size()))
+            return PA_POOL_EINVAL;  // the row was not reset for this sequence
+    }
+    // Every check is done: nothing below can fail.
+    apply_batch(*pool, n_tokens);
+    *num_pairs = take_copies(*pool, pairs_out);
+    for (int32_t r = 0; r < num_seqs; ++r) {
+        const Seq &s = *pool->batch[static_cast<size_t>(r)];
+        int64_t *out = slots_out + static_cast<int64_t>(r) * n_tokens;
+        for (int64_t i = 0; i < n_tokens; ++i) {
+            const int64_t pos = s.len - n_tokens + i;
+            out[i] = static_cast<int64_t>(s.blocks[static_cast<size_t>(pos / B)]) * B + pos % B;
+        }
+        update_row(s, table + static_cast<int64_t>(r) * width, synced[r]);
+        lens_out[r] = static_cast<int32_t>(s.len);
     }
     return PA_POOL_OK;
 }
@@ -258,16 +382,7 @@ int64_t pa_pool_take_copies(pa_pool_t *pool, int64_t *pairs_out, int64_t capacit
     const int64_t n = static_cast<int64_t>(pool->pending.size());
     if (n > capacity || (n > 0 && !pairs_out))
         return PA_POOL_ERANGE;
-    std::vector<std::pair<int32_t, int32_t>> taken;
-    taken.swap(pool->pending);
-    for (int64_t i = 0; i < n; ++i) {
-        pairs_out[2 * i] = taken[static_cast<size_t>(i)].first;
-        pairs_out[2 * i + 1] = taken[static_cast<size_t>(i)].second;
-        const int32_t ends[2] = {taken[static_cast<size_t>(i)].first,
-                                 taken[static_cast<size_t>(i)].second};
-        pool->release_refs(ends, 2, pool->pin);
-    }
-    return n;
+    return take_copies(*pool, pairs_out);
 }
 
 int64_t pa_pool_num_blocks(const pa_pool_t *pool) {
@@ -353,16 +468,8 @@ int pa_pool_block_table_update(const pa_pool_t *pool, const int64_t *seq_ids, in
         if (synced[r] > n)  // a sequence never loses blocks: the row names another one now
             return PA_POOL_EINVAL;
     }
-    for (int32_t r = 0; r < num_seqs; ++r) {
-        const std::vector<int32_t> &bl = pool->seqs.find(seq_ids[r])->second.blocks;
-        const int32_t n = static_cast<int32_t>(bl.size());
-        int32_t *row = out + static_cast<int64_t>(r) * width;
-        // Entries before the old tail never change; the old tail may have been
-        // redirected by a copy-on-write, and the entries after it are new.
-        const int32_t from = synced[r] > 0 ? synced[r] - 1 : 0;
-        std::copy(bl.begin() + from, bl.end(), row + from);
-        synced[r] = n;
-    }
+    for (int32_t r = 0; r < num_seqs; ++r)
+        update_row(pool->seqs.find(seq_ids[r])->second, out + static_cast<int64_t>(r) * width, synced[r]);
     return PA_POOL_OK;
 }
 

@@ -17,7 +17,7 @@ PA_POOL_OK, PA_POOL_EINVAL, PA_POOL_ENOSPACE, PA_POOL_ENOSEQ, PA_POOL_EEXIST, PA
 PA_COW_SHARED, PA_COW_INHERITED = 0, 1
 
 EXPORTED = ("pa_pool_create", "pa_pool_destroy", "pa_pool_seq_create", "pa_pool_append", "pa_pool_append_batch",
-            "pa_pool_fork",
+            "pa_pool_step", "pa_pool_fork",
             "pa_pool_release", "pa_pool_num_pending_copies", "pa_pool_take_copies", "pa_pool_num_blocks",
             "pa_pool_block_size", "pa_pool_num_free", "pa_pool_seq_len", "pa_pool_seq_num_blocks",
             "pa_pool_refcount", "pa_pool_pins", "pa_pool_free_list", "pa_pool_block_table",
@@ -33,6 +33,7 @@ for _name, _args, _res in [
     ("pa_pool_seq_create", [_P, _i64], ctypes.c_int),
     ("pa_pool_append", [_P, _i64, _i64], ctypes.c_int),
     ("pa_pool_append_batch", [_P, _P, _i32, _i64], ctypes.c_int),
+    ("pa_pool_step", [_P, _P, _i32, _i64, _P, _i64, _P, _P, _i32, _P, _P, _P], ctypes.c_int),
     ("pa_pool_fork", [_P, _i64, _i64], ctypes.c_int),
     ("pa_pool_release", [_P, _i64], ctypes.c_int),
     ("pa_pool_num_pending_copies", [_P], _i64),
@@ -119,6 +120,43 @@ class BlockPool:
             return False
         _ok(rc, "append_batch")
         return True
+
+    def step(self, seq_ids, n: int, table: np.ndarray, synced: np.ndarray, slots: np.ndarray | None = None,
+             lens: np.ndarray | None = None, pairs: np.ndarray | None = None):
+        """The host side of one decode step in one call (pa_pool_step): append
+        n tokens to every listed sequence, all or nothing, then hand out the
+        queued copy pairs, the step's slot mapping and the lengths, and bring
+        `table` (with `synced`, as block_table_update) up to date in place.
+        Returns (pairs [k, 2] int64, slots [num_seqs * n] int64, lens int32),
+        or None when the pool cannot hold the appends (nothing changed).
+        `slots`, `lens` and `pairs` may be passed in to be reused."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        S = len(ids)
+        if table.dtype != np.int32 or not table.flags.c_contiguous or table.ndim != 2 or table.shape[0] != S:
+            raise ValueError("table must be a C-contiguous int32 [num_seqs, width] array")
+        if synced.dtype != np.int32 or synced.shape != (S,) or not synced.flags.c_contiguous:
+            raise ValueError("synced must be int32 [num_seqs]")
+        if slots is None:
+            slots = np.empty(S * n, dtype=np.int64)
+        elif slots.dtype != np.int64 or slots.shape != (S * n,) or not slots.flags.c_contiguous:
+            raise ValueError("slots must be int64 [num_seqs * n]")
+        if lens is None:
+            lens = np.empty(S, dtype=np.int32)
+        elif lens.dtype != np.int32 or lens.shape != (S,) or not lens.flags.c_contiguous:
+            raise ValueError("lens must be int32 [num_seqs]")
+        if pairs is None:
+            pairs = np.empty((S + _ok(lib.pa_pool_num_pending_copies(self._h), "num_pending_copies"), 2),
+                             dtype=np.int64)
+        elif pairs.dtype != np.int64 or pairs.ndim != 2 or pairs.shape[1] != 2 or not pairs.flags.c_contiguous:
+            raise ValueError("pairs must be a C-contiguous int64 [capacity, 2] array")
+        k = ctypes.c_int64(0)
+        rc = lib.pa_pool_step(self._h, ids.ctypes.data, S, n, pairs.ctypes.data, pairs.shape[0], ctypes.byref(k),
+                              slots.ctypes.data, table.shape[1], table.ctypes.data, synced.ctypes.data,
+                              lens.ctypes.data)
+        if rc == PA_POOL_ENOSPACE:
+            return None
+        _ok(rc, "step")
+        return pairs[:k.value], slots, lens
 
     def fork(self, src: int, dst: int) -> None:
         _ok(lib.pa_pool_fork(self._h, src, dst), "fork")

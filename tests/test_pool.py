@@ -424,3 +424,121 @@ def test_incremental_block_table_refuses_a_row_that_was_not_reset():
     synced[:] = 0
     p.block_table_update([1], table, synced)
     assert np.array_equal(table, p.block_table([1], 6)) and synced.tolist() == [1]
+
+
+def _step_by_parts(p, ids, n, table, synced):
+    """The reference composition of pa_pool_step: the five separate calls."""
+    if not p.append_batch(ids, n):
+        return None
+    pairs = p.take_cow_pairs()
+    slots = p.step_slots(ids, n)
+    p.block_table_update(ids, table, synced)
+    return np.asarray(pairs, np.int64).reshape(-1, 2), slots, p.seq_lens(ids)
+
+
+def _full_state(p, NB):
+    return (list(p.free_list()), [p.refcount(b) for b in range(NB)], [p.pins(b) for b in range(NB)])
+
+
+@pytest.mark.parametrize("rule", ["shared", "inherited"])
+@pytest.mark.parametrize("seed", range(6))
+def test_fused_step_equals_the_separate_calls(rule, seed):
+    """pa_pool_step gives the pairs, slots, table, lengths and pool state of
+    append_batch + take_copies + step_slots + block_table_update + seq_lens,
+    step after step, on forks that share partial tails (copy-on-write under
+    either rule) until the pool runs out."""
+    gen = np.random.default_rng(seed)
+    NB, B = 48, 4
+    order = gen.permutation(NB).astype(np.int32)
+    a, b = BlockPool(NB, B, order, rule), BlockPool(NB, B, order, rule)
+    for p in (a, b):
+        p.create(0)
+        assert p.append(0, 6)
+        for k in (1, 2, 3):
+            p.fork(0, k)
+        p.create(4)
+        assert p.append(4, 3)
+    ids = np.array([3, 0, 4, 2, 1], np.int64)
+    width = NB
+    ta, tb = np.full((5, width), -1, np.int32), np.full((5, width), -1, np.int32)
+    sa, sb = np.zeros(5, np.int32), np.zeros(5, np.int32)
+    full = False
+    for step in range(40):
+        n = int(gen.integers(0, 4))
+        got = a.step(ids, n, ta, sa)
+        want = _step_by_parts(b, ids, n, tb, sb)
+        if want is None:
+            assert got is None
+            full = True
+            assert _full_state(a, NB) == _full_state(b, NB)
+            break
+        pairs, slots, lens = got
+        assert np.array_equal(pairs, want[0]) and np.array_equal(slots, want[1]) and np.array_equal(lens, want[2])
+        assert np.array_equal(ta, tb) and np.array_equal(sa, sb)
+        assert _full_state(a, NB) == _full_state(b, NB)
+        a.check()
+    assert full  # the run reached the end of the pool
+
+
+def test_fused_step_matches_the_oracle_pool_on_chat():
+    """Three decode steps of the chat workload (64 sequences, the 26,785-block
+    pool) through pa_pool_step against the oracle pool's appends, slots,
+    tables and lengths."""
+    w = synth.chat()
+    sh = w.shape
+    c, r = BlockPool(sh.num_blocks, sh.block_size, w.free_order), RefPool(sh.num_blocks, sh.block_size, w.free_order)
+    for p in (c, r):
+        w.ops(p)
+        p.take_cow_pairs()
+    ids = np.asarray(w.seq_ids, np.int64)
+    width = max(c.num_blocks_of(int(i)) for i in ids) + 2
+    table, synced = np.full((len(ids), width), -1, np.int32), np.zeros(len(ids), np.int32)
+    for _ in range(3):
+        pairs, slots, lens = c.step(ids, 1, table, synced)
+        assert r.append_batch(ids.tolist(), 1)
+        assert len(pairs) == len(r.take_cow_pairs()) == 0
+        assert slots.tolist() == [int(r.slots(int(i), r.seq_len(int(i)) - 1, 1)[0]) for i in ids]
+        assert lens.tolist() == [r.seq_len(int(i)) for i in ids]
+        assert np.array_equal(table, np.asarray(r.block_table(ids.tolist(), width)))
+
+
+def test_fused_step_refusals_change_nothing():
+    """Every refusal of pa_pool_step leaves the pool, the table and synced as
+    they were: too few free blocks, too little room for the copy pairs or
+    the table row, a row not reset, a sequence listed twice, an unknown one."""
+    from paged_kv_cache_333_b200.pool import PoolError
+    NB, B = 12, 4
+    p = BlockPool(NB, B, np.arange(NB, dtype=np.int32))
+    p.create(0)
+    assert p.append(0, 6)  # 2 blocks, partial tail
+    p.fork(0, 1)           # shares both
+    ids = np.array([0, 1], np.int64)
+    table, synced = np.full((2, 8), -1, np.int32), np.zeros(2, np.int32)
+    p.block_table_update(ids, table, synced)
+
+    def snap():
+        return (_full_state(p, NB), table.tolist(), synced.tolist(), [p.seq_len(0), p.seq_len(1)])
+
+    def refused(call, error=True):
+        before = snap()
+        if error:
+            with pytest.raises(PoolError):
+                call()
+        else:
+            assert call() is None
+        assert snap() == before
+
+    refused(lambda: p.step(ids, 40, table, synced), error=False)  # not enough free blocks
+    # 1 token: sequence 0 copies its shared tail, but there is room for 0 pairs
+    refused(lambda: p.step(ids, 1, table, synced, pairs=np.empty((0, 2), np.int64)))
+    narrow, nsync = np.full((2, 2), -1, np.int32), np.zeros(2, np.int32)
+    refused(lambda: p.step(ids, 3, narrow, nsync))  # a third block each: width 2 is too small
+    assert narrow.tolist() == [[-1, -1], [-1, -1]] and nsync.tolist() == [0, 0]
+    bad = synced.copy()
+    bad[1] = 3  # more entries than the sequence has blocks: the row was not reset
+    refused(lambda: p.step(ids, 1, table, bad))
+    refused(lambda: p.step(np.array([0, 0], np.int64), 1, table, synced))  # listed twice
+    refused(lambda: p.step(np.array([0, 7], np.int64), 1, table, synced))  # unknown sequence
+    pairs, slots, lens = p.step(ids, 1, table, synced)  # and the step itself still goes through
+    assert len(pairs) == 1 and lens.tolist() == [7, 7]
+    p.check()
