@@ -542,3 +542,62 @@ def test_fused_step_refusals_change_nothing():
     pairs, slots, lens = p.step(ids, 1, table, synced)  # and the step itself still goes through
     assert len(pairs) == 1 and lens.tolist() == [7, 7]
     p.check()
+
+
+@pytest.mark.parametrize("rule", ["shared", "inherited"])
+@pytest.mark.parametrize("seed", range(4))
+def test_fused_step_random_histories_match_the_oracle_pool(rule, seed):
+    """Random histories of creates, forks, releases and steps over random
+    subsets of the live sequences: after every step, pa_pool_step's copy
+    pairs, slots, lengths and incrementally kept table rows equal the oracle
+    pool's (each sequence keeps its own row and count between its steps, as
+    a scheduler would), and both pools hold the same blocks."""
+    gen = np.random.default_rng(100 + seed)
+    NB, B, W = 64, 4, 64
+    order = gen.permutation(NB).astype(np.int32)
+    c, r = BlockPool(NB, B, order, rule), RefPool(NB, B, order, rule)
+    rows: dict[int, tuple[np.ndarray, int]] = {}
+    live: list[int] = []
+    nxt = 0
+    for _ in range(300):
+        op = gen.random()
+        if op < 0.15 or not live:
+            for p in (c, r):
+                p.create(nxt)
+            rows[nxt] = (np.full(W, -1, np.int32), 0)
+            live.append(nxt)
+            nxt += 1
+        elif op < 0.25:
+            src = live[int(gen.integers(len(live)))]
+            for p in (c, r):
+                p.fork(src, nxt)
+            rows[nxt] = (np.full(W, -1, np.int32), 0)
+            live.append(nxt)
+            nxt += 1
+        elif op < 0.35:
+            victim = live.pop(int(gen.integers(len(live))))
+            for p in (c, r):
+                p.release(victim)
+            del rows[victim]
+        else:
+            k = int(gen.integers(1, len(live) + 1))
+            ids = [live[i] for i in gen.choice(len(live), size=k, replace=False)]
+            n = int(gen.integers(0, 4))
+            table = np.stack([rows[i][0] for i in ids])
+            synced = np.array([rows[i][1] for i in ids], np.int32)
+            got = c.step(np.array(ids, np.int64), n, table, synced)
+            ok = r.append_batch(ids, n)
+            if not ok:
+                assert got is None
+                continue
+            pairs, slots, lens = got
+            assert [tuple(x) for x in pairs.tolist()] == [tuple(x) for x in r.take_cow_pairs()]
+            want_slots = [int(s) for i in ids for s in r.slots(i, r.seq_len(i) - n, n)]
+            assert slots.tolist() == want_slots
+            assert lens.tolist() == [r.seq_len(i) for i in ids]
+            assert table.tolist() == np.asarray(r.block_table(ids, W)).tolist()
+            for j, i in enumerate(ids):
+                rows[i] = (table[j].copy(), int(synced[j]))
+        assert c.free_list() == r.free_list()
+    c.check()
+    r.check()
