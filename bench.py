@@ -232,9 +232,10 @@ def host_pool_step_us(w, steps: int = 200) -> dict:
     mapping build) on the C++ pool, as one pa_pool_step call: append one
     token to every sequence, take the queued copy pairs, build the step's
     slot mapping and lengths, and update the block table kept across steps
-    (append-only).  Output buffers are reused across steps.  Timed on a fresh
-    pool laid out as the workload (the timed device step uses its own)."""
-    from paged_kv_cache_333_b200.pool import BlockPool
+    (append-only).  The step's arrays are allocated once for the batch
+    (StepBuffers) and reused.  Timed on a fresh pool laid out as the workload
+    (the timed device step uses its own)."""
+    from paged_kv_cache_333_b200.pool import BlockPool, StepBuffers
     sh = w.shape
     pool = BlockPool(sh.num_blocks, sh.block_size, w.free_order, "shared")
     w.ops(pool)
@@ -242,22 +243,19 @@ def host_pool_step_us(w, steps: int = 200) -> dict:
         w.suffix_ops(pool)
     pool.take_cow_pairs()
     ids = np.asarray(w.seq_ids, dtype=np.int64)
-    S = len(ids)
     width = max(pool.num_blocks_of(int(i)) for i in ids) + steps // sh.block_size + 2
-    table = np.full((S, width), -1, dtype=np.int32)  # kept across steps, updated append-only
-    synced = np.zeros(S, dtype=np.int32)
-    pool.block_table_update(ids, table, synced)
-    slots, lens, pairs = np.empty(S, np.int64), np.empty(S, np.int32), np.empty((S, 2), np.int64)
+    buf = StepBuffers(ids, 1, width)
+    pool.step_into(buf)  # the first step writes whole table rows; the timed ones are incremental
     done = 0
     t0 = time.perf_counter()
     for _ in range(steps):
-        if pool.step(ids, 1, table, synced, slots, lens, pairs) is None:
+        if pool.step_into(buf) is None:
             break
         done += 1
     dt = time.perf_counter() - t0
-    return {"us": round(dt / max(done, 1) * 1e6, 2), "steps": done, "sequences": int(S),
+    return {"us": round(dt / max(done, 1) * 1e6, 2), "steps": done, "sequences": int(len(ids)),
             "what": "pa_pool_step: append 1 token per sequence + copy pairs + slot mapping + block table "
-                    "(updated append-only) + lengths, one ctypes call, one host thread"}
+                    "(updated append-only) + lengths, one ctypes call on arrays allocated once, one host thread"}
 
 
 # --------------------------------------------------------------------------- ours

@@ -91,13 +91,14 @@ class BlockPool:
         self._h = lib.pa_pool_create(int(num_blocks), int(block_size), fp, rule_id)
         if not self._h:
             raise PoolError(PA_POOL_EINVAL, "pa_pool_create")
+        self._destroy = lib.pa_pool_destroy  # kept: module globals may be gone when __del__ runs at exit
         self.num_blocks = int(num_blocks)
         self.block_size = int(block_size)
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h:
-            lib.pa_pool_destroy(h)
+            self._destroy(h)
             self._h = None
 
     # -- operations -------------------------------------------------------
@@ -157,6 +158,17 @@ class BlockPool:
             return None
         _ok(rc, "step")
         return pairs[:k.value], slots, lens
+
+    def step_into(self, buf: "StepBuffers") -> int | None:
+        """pa_pool_step on a StepBuffers (its sequences, its n_tokens): the
+        results land in buf.pairs[:k], buf.slots, buf.table (with buf.synced)
+        and buf.lens.  Returns k, the number of copy pairs, or None when the
+        pool cannot hold the appends (nothing changed)."""
+        rc = lib.pa_pool_step(self._h, *buf._args)
+        if rc == PA_POOL_ENOSPACE:
+            return None
+        _ok(rc, "step")
+        return buf._k.value
 
     def fork(self, src: int, dst: int) -> None:
         _ok(lib.pa_pool_fork(self._h, src, dst), "fork")
@@ -233,3 +245,30 @@ class BlockPool:
 
     def check(self) -> None:
         _ok(lib.pa_pool_check(self._h), "check")
+
+
+class StepBuffers:
+    """The arrays of pa_pool_step for one fixed batch of sequences, allocated
+    once and reused every step (their addresses are taken once, which is most
+    of the host cost of a step through ctypes).  The table starts empty
+    (synced 0), so the first step writes whole rows.
+      ids     int64 [S]            the batch, in order
+      table   int32 [S, width]     block table, kept up to date in place (pad -1)
+      synced  int32 [S]            entries of each row already written
+      slots   int64 [S * n_tokens] the step's slot mapping
+      lens    int32 [S]            lengths after the step
+      pairs   int64 [capacity, 2]  queued copy pairs handed out by the step"""
+
+    def __init__(self, seq_ids, n_tokens: int, width: int, pairs_capacity: int | None = None):
+        self.ids = np.array(seq_ids, dtype=np.int64)
+        S = len(self.ids)
+        self.n_tokens = int(n_tokens)
+        self.table = np.full((S, int(width)), -1, dtype=np.int32)
+        self.synced = np.zeros(S, dtype=np.int32)
+        self.slots = np.empty(S * self.n_tokens, dtype=np.int64)
+        self.lens = np.empty(S, dtype=np.int32)
+        self.pairs = np.empty((S if pairs_capacity is None else int(pairs_capacity), 2), dtype=np.int64)
+        self._k = ctypes.c_int64(0)
+        self._args = (self.ids.ctypes.data, S, self.n_tokens, self.pairs.ctypes.data, self.pairs.shape[0],
+                      ctypes.byref(self._k), self.slots.ctypes.data, int(width), self.table.ctypes.data,
+                      self.synced.ctypes.data, self.lens.ctypes.data)

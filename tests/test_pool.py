@@ -601,3 +601,35 @@ def test_fused_step_random_histories_match_the_oracle_pool(rule, seed):
         assert c.free_list() == r.free_list()
     c.check()
     r.check()
+
+
+@pytest.mark.parametrize("rule", ["shared", "inherited"])
+def test_step_buffers_give_the_same_steps(rule):
+    """step_into on reused StepBuffers (addresses taken once, table starting
+    empty) matches step() on fresh arrays, step after step, copy-on-write
+    included, until the pool is full."""
+    from paged_kv_cache_333_b200.pool import StepBuffers
+    NB, B = 48, 4
+    order = np.random.default_rng(5).permutation(NB).astype(np.int32)
+    a, b = BlockPool(NB, B, order, rule), BlockPool(NB, B, order, rule)
+    for p in (a, b):
+        p.create(0)
+        assert p.append(0, 6)
+        for k in (1, 2):
+            p.fork(0, k)
+    ids = [2, 0, 1]
+    buf = StepBuffers(ids, 2, NB)
+    table, synced = np.full((3, NB), -1, np.int32), np.zeros(3, np.int32)
+    for _ in range(30):
+        k = a.step_into(buf)
+        got = b.step(np.array(ids, np.int64), 2, table, synced)
+        if got is None:
+            assert k is None
+            break
+        pairs, slots, lens = got
+        assert buf.pairs[:k].tolist() == pairs.tolist()
+        assert buf.slots.tolist() == slots.tolist() and buf.lens.tolist() == lens.tolist()
+        assert buf.table.tolist() == table.tolist() and buf.synced.tolist() == synced.tolist()
+    else:
+        pytest.fail("the pool never filled")
+    a.check()
