@@ -71,8 +71,10 @@ def _ok(rc: int, what: str) -> int:
     return rc
 
 
-def _ptr(a: np.ndarray):
-    return a.ctypes.data_as(ctypes.c_void_p)
+def _ptr(a: np.ndarray) -> int:
+    """Address of a contiguous array's data, for a void* argument.  The caller
+    keeps `a` referenced until the call returns (an address holds no reference)."""
+    return a.ctypes.data
 
 
 class BlockPool:
