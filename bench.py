@@ -78,7 +78,10 @@ def parse_args():
                          "request are its rows (speculative decode / prefill chunk; pa_attention)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="KV cache element type (fp8 = OCP E4M3 codes with per-tensor scales)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.queries > 1 and args.kv_dtype == "fp8":
+        ap.error("--queries > 1 runs pa_attention, which reads a bf16 cache: use --kv-dtype bf16")
+    return args
 
 
 def dist_env():
