@@ -31,14 +31,22 @@ import numpy as np
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32 values to bfloat16 (nearest, ties to even); return uint16 bits."""
-    a = np.asarray(x, dtype=np.float32)
-    u = np.ascontiguousarray(a).reshape(-1).view(np.uint32)
-    nan = (u & 0x7FFFFFFF) > 0x7F800000
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
-    r = np.where(nan, np.uint16(0x7FC0), r)
-    return r.astype(np.uint16).reshape(a.shape)
+    """Round float32 values to bfloat16 (nearest, ties to even); return uint16
+    bits, 0x7FC0 for every NaN.  (Add 0x7FFF plus the kept half's lowest bit,
+    then drop the low 16 bits; done in place on one uint32 temporary.)"""
+    shape = np.shape(x)
+    a = np.ascontiguousarray(x, dtype=np.float32)
+    u = a.reshape(-1).view(np.uint32)
+    r = u >> 16
+    r &= 1
+    r += 0x7FFF
+    r += u  # wraps only for NaN patterns, which are replaced below
+    r >>= 16
+    out = r.astype(np.uint16)
+    nan = np.isnan(a.reshape(-1))
+    if nan.any():
+        out[nan] = 0x7FC0
+    return out.reshape(shape)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
