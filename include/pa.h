@@ -71,7 +71,7 @@ enum {
  * [num_blocks*block_size][num_kv_heads*head_dim] is token slot `slot`
  * ("PagedAttention: fragmentation, blocks, block tables", section 3 "The
  * slot mapping": block-major backing storage; the r7 walkthrough stores the
- * token "at flat row 30,608"). */
+ * token at row 30,608 of the cache so viewed). */
 typedef struct pa_cache {
     void *k_cache;
     void *v_cache;
@@ -84,9 +84,9 @@ typedef struct pa_cache {
 /*
  * pa_write_kv -- the KV-cache write of one step.
  * Defined by: "PagedAttention: fragmentation, blocks, block tables",
- * section 3 "The slot mapping" (the kernel writes new K/V at
- * slot_mapping[i]; every layer writes the same slot, only the tensor
- * differs; padded positions carry a PAD value).
+ * section 3 "The slot mapping" (each new token's K and V are stored at the
+ * slot that slot_mapping[i] names, the same slot in every layer's own
+ * tensor; padding entries hold a sentinel that is not a slot).
  *   k, v          [num_tokens][num_kv_heads][head_dim] bf16, contiguous.
  *   slot_mapping  [num_tokens] int64; row i goes to cache row slot_mapping[i];
  *                 a negative slot is padding and is skipped.  Slots must be
@@ -133,8 +133,8 @@ PA_API int pa_write_kv_positions(const void *k, const void *v, const int64_t *po
  * Defined by: "PagedAttention: fragmentation, blocks, block tables",
  * section 2 "The block table" (append_row maps the ids through
  * map_to_kernel_blocks when the kernel's block is smaller) and the passage
- * on decoupling the allocation block from the kernel's page (a 32-token
- * allocation block can feed a kernel that wants 16-token pages).  The cache
+ * on decoupling the allocation block from the kernel's page (allocation in
+ * 32-token units, say, while the attention kernel reads 16-token pages).  The cache
  * is block-major, so allocation block a (pages of block_size tokens) owns the
  * bytes of kernel blocks a*m .. a*m + m - 1 (pages of block_size / m tokens),
  * m = blocks_per_alloc: the same memory is a pa_cache_t with num_blocks * m
@@ -154,8 +154,8 @@ PA_API int pa_map_to_kernel_blocks(const int32_t *block_tables, int32_t num_rows
 /*
  * pa_copy_blocks -- copy-on-write block copies.
  * Defined by: "PagedAttention: fragmentation, blocks, block tables",
- * copy-on-write passage (a list of (src_block_id, dst_block_id) pairs runs
- * before the forward pass reads the cache; one assignment
+ * copy-on-write passage (the queued (src_block_id, dst_block_id) pairs are
+ * executed ahead of the step's attention reads; one assignment
  * blocks[dst] = blocks[src] over the block-major storage).
  *   src_dst_pairs [num_pairs][2] int64 (src, dst).  Every dst must be
  *                 distinct and no dst may also be a src (the pool's pairs
@@ -167,7 +167,8 @@ PA_API int pa_copy_blocks(const pa_cache_t *cache, const int64_t *src_dst_pairs,
 
 /*
  * pa_copy_blocks_layers -- pa_copy_blocks for every layer of a model in one
- * launch.  Same passage as pa_copy_blocks ("not a per-layer loop": there the
+ * launch.  Same passage as pa_copy_blocks (one batched copy for all layers
+ * rather than a loop over them: there the
  * layers alias one storage; here each layer has its own K and V tensors and
  * one grid covers them all).
  *   caches      HOST array of num_layers descriptors (<= 128), all with the
@@ -189,11 +190,11 @@ PA_API size_t pa_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, i
  * pa_decode -- decode attention over the paged cache, one query token per
  * sequence.
  * Defined by: "PagedAttention: fragmentation, blocks, block tables",
- * attention-metadata passage (block_table is [num_reqs, max_num_blocks_per_req]
- * int32; the kernel gathers past K/V by walking row r for
- * ceil(seq_lens[r] / block_size) entries; max_seq_len may be an upper bound)
- * and section 2 "The block table" (position p lives in entry p / B at
- * offset p % B); "The pantry of pigeonholes", "The mechanism: blocks, block
+ * attention-metadata passage (an int32 table with one row per request; for
+ * request r the gather reads the first ceil(seq_lens[r] / block_size)
+ * entries of its row; max_seq_len need only bound the lengths from above)
+ * and section 2 "The block table" (token p is found through entry p / B, at
+ * offset p % B inside that block); "The pantry of pigeonholes", "The mechanism: blocks, block
  * table and the kernel gather".
  * For sequence s and query head j, with h = j / (num_q_heads / num_kv_heads):
  *   out[s][j] = sum_t softmax_t(scale * q[s][j] . K[s,h,t]) V[s,h,t],
@@ -312,8 +313,8 @@ PA_API int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int
 
 /* ------------------------------------------------------------------------
  * FP8 KV cache ("The pantry of pigeonholes", "The 10 knobs", knob 4
- * kv_cache_dtype, and "How it connects to the rest of the stack": moving the
- * KV to FP8 halves the bytes per token).  Codes are OCP FP8 E4M3 (one byte,
+ * kv_cache_dtype, and "How it connects to the rest of the stack": one-byte
+ * codes take half the bytes of bf16 for every cached token).  Codes are OCP FP8 E4M3 (one byte,
  * bias 7, no infinities, largest finite 448); a code c of the K (V) tensor
  * stands for value(c) * k_scale (v_scale), one scale per tensor.
  * ------------------------------------------------------------------------ */

@@ -9,10 +9,10 @@
  *     section 1 "The block pool"    -- allocation pops the head of the free
  *        queue; a request that needs more blocks than are free is refused;
  *        freed blocks whose count reaches zero are put back at the FRONT of
- *        the queue, as one run in the order they were freed; a sequence's
- *        blocks are freed in reverse order;
+ *        the queue, as one run keeping their release order; a released
+ *        sequence gives its blocks back last block first;
  *     section 2 "The block table"   -- a sequence's table only grows at its
- *        tail; position p lives in entry p / B at offset p % B;
+ *        tail; token p is found through entry p / B, at offset p % B;
  *     section 3 "The slot mapping"  -- slot = table[p / B] * B + p % B;
  *     the copy-on-write passage     -- a redirected tail block and its source
  *        both stay retained until the copy has been handed to the device;

@@ -142,8 +142,8 @@ def map_to_kernel_blocks(block_table, blocks_per_alloc: int) -> np.ndarray:
     blocks_per_alloc kernel blocks per allocation block ("PagedAttention:
     fragmentation, blocks, block tables": section 2 "The block table", where
     append_row maps the ids through map_to_kernel_blocks when the kernel's
-    block is smaller, and the decoupling passage: a 32-token allocation block
-    can feed a kernel that wants 16-token pages).  Storage is block-major, so
+    block is smaller, and the decoupling passage: allocation in larger units,
+    say 32 tokens, while the attention kernel reads 16-token pages).  Storage is block-major, so
     allocation block a owns the bytes of kernel blocks a*m .. a*m + m - 1:
     entry i of a row becomes entries i*m .. i*m + m - 1.  Negative entries
     (padding) become m entries of -1."""

@@ -15,7 +15,7 @@
  *     tables", section 3 "The slot mapping"), and a flat row index
  *     block*block_size + offset is a "slot": row `slot` of the cache viewed as
  *     [num_blocks*block_size][num_kv_heads*head_dim] (same page, walkthrough
- *     step 9: the new token is stored "at flat row 30,608").
+ *     step 9: the new token lands at row 30,608 of the cache so viewed).
  *   - Query head j reads KV head j / (num_q_heads/num_kv_heads) (contiguous
  *     grouped-query heads; the pages are silent, this is the standard reading).
  */
@@ -37,8 +37,8 @@ static double bf16_to_double(uint16_t bits)
  * Write: token i's K row (num_kv_heads*head_dim values) is stored at flat
  * row slot_mapping[i] of k_cache, and its V row at the same row of v_cache.
  * A negative slot is padding and is skipped.  ("PagedAttention: fragmentation,
- * blocks, block tables", section 3 "The slot mapping": the kernel writes new
- * K/V at slot_mapping[i]; padded positions carry PAD_ID.)
+ * blocks, block tables", section 3 "The slot mapping": each new token's K/V
+ * go to the slot slot_mapping[i] names; padding entries hold a sentinel.)
  * Returns 0, or -1 if a slot is >= num_slots (nothing is written then).
  */
 int oracle_write_kv(const uint16_t *k, const uint16_t *v, const int64_t *slot_mapping,
@@ -111,8 +111,8 @@ int oracle_copy_blocks(const int64_t *pairs, int64_t num_pairs, int64_t block_el
  *   1. rebuild the contiguous K and V of (s, h): token t lives in physical
  *      block block_tables[s][t / B] at offset t % B ("PagedAttention:
  *      fragmentation, blocks, block tables", section 2 "The block table":
- *      position p lives in block table[p // block_size] at offset
- *      p % block_size; the kernel walks ceil(seq_len / block_size) entries);
+ *      token p is reached through table entry p / block_size, at offset
+ *      p % block_size, and n tokens use ceil(n / block_size) entries);
  *   2. z_t = scale * sum_d q[s][j][d] * K_t[d]            (all in double);
  *   3. p_t = exp(z_t - max z) / sum_u exp(z_u - max z);
  *   4. out[s][j][d] = sum_t p_t * V_t[d].

@@ -9,14 +9,15 @@ check the product's C++ pool operation by operation:
   refuses when too few blocks are free);
 - freeing decrements reference counts and puts blocks that reach zero back at
   the FRONT of the queue, as one run in the order given (same section:
-  unhashed blocks are prepended, "LIFO reuse"); a request's blocks are freed
-  in reverse order (same section, SingleTypeKVCacheManager.free);
+  blocks without a hash go back to the head, so the newest free block is
+  reused first); a released request gives its blocks back last block first
+  (same section, SingleTypeKVCacheManager.free);
 - a sequence owns a list of block ids; position p lives in block p // B at
   offset p % B (section 2 "The block table"), and its slot is
   table[p // B] * B + p % B (section 3 "The slot mapping");
-- fork shares every block by reference count, with no copy ("Full-block
-  sharing needs no copy at all", copy-on-write passage of the same page;
-  the CPU reference allocator's fork);
+- fork shares every block by reference count; sharing whole blocks takes
+  no copy (copy-on-write passage of the same page; the CPU reference
+  allocator's fork);
 - append allocates ceil((len + n) / B) - len(table) new blocks and, when the
   tail is partial and shared, first redirects the tail to a fresh block and
   queues a (src, dst) copy ("Memory management", Code: copy iff len % B != 0
@@ -25,8 +26,8 @@ check the product's C++ pool operation by operation:
   the partial tail was not allocated by this sequence, i.e. on every partial
   hit) is selectable with rule="inherited";
 - both endpoints of a queued copy stay retained until the copy is taken for
-  execution (copy-on-write passage of page 1: "Both copy endpoints stay
-  retained until the copy has run").  Such a retention is kept apart from
+  execution (copy-on-write passage of page 1: the source and destination
+  are held until the copy has been carried out).  Such a retention is kept apart from
   the owner references, as page 1's "Two kinds of references" keeps transfer
   pins apart from owners: the copy-on-write trigger counts owners (tables
   naming the block) only, and a block is free only when it has neither
@@ -72,8 +73,8 @@ class RefPool:
 
     def _release_refs(self, ordered: list[int], counts: list[int]) -> None:
         """Drop one reference of each block (from `counts`, which is self.ref
-        or self.pin); blocks left with no owner and no pin go to the front of
-        the free queue as one run, in the given order."""
+        or self.pin); blocks left with no owner and no pin are pushed back at
+        the head of the free queue together, keeping the given order."""
         run = []
         for b in ordered:
             counts[b] -= 1

@@ -1,8 +1,8 @@
 // Paged decode attention over an FP8 (OCP E4M3) KV cache.
 //
-// An FP8 cache halves the bytes per token ("The pantry of pigeonholes", "The
-// 10 knobs", knob 4 kv_cache_dtype; "How it connects to the rest of the
-// stack": moving the KV to FP8 halves the bytes per token).  A stored code c
+// An FP8 cache stores one byte per value where bf16 takes two ("The pantry
+// of pigeonholes", "The 10 knobs", knob 4 kv_cache_dtype, and "How it
+// connects to the rest of the stack", on quantising the cache).  A stored code c
 // of the K (V) tensor stands for value(c) * k_scale (v_scale).
 //
 // Same CTA decomposition, producer and split-K as decode_mma.cuh.  With half

@@ -89,8 +89,8 @@ struct pa_pool {
     }
 
     // Drop one reference (owner or pin, per `counts`) of each block in the
-    // given order; blocks left with neither owners nor pins go back to the
-    // front of the free queue as one run, keeping that order.
+    // given order; blocks left with neither owners nor pins are pushed back at
+    // the head of the free queue together, keeping that order.
     void release_refs(const int32_t *ordered, size_t n, std::vector<int32_t> &counts) {
         std::vector<int32_t> run;
         for (size_t i = 0; i < n; ++i) {

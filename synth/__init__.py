@@ -12,8 +12,8 @@ drawn N(0, 1) in float32 and rounded to bfloat16 (round to nearest even); they
 travel as ``uint16`` bit patterns.
 
 Workload shapes follow the pages' setting (Llama-3-8B: 32 query heads, 8 KV
-heads, head dim 128, 16-token blocks, a 26,785-block pool; a chat turn is a
-512-token prompt plus up to 100 generated tokens; 32K-token contexts).  See
+heads, head dim 128, 16-token blocks, a 26,785-block pool; chat turns of 512
+prompt tokens and at most 100 generated ones; 32K-token contexts).  See
 "PagedAttention: fragmentation, blocks, block tables", introduction, for the
 pool and the chat turn, and "The pantry of pigeonholes", "The maths that
 matter", for the per-token KV size.
@@ -259,8 +259,9 @@ def sweep(block_size: int, seed: int = 337, batch: int = 128, mean_len: int = 10
           cap: int = 8192, events: int = 10_000, occupancy: float = 0.9,
           slots: int = LLAMA3_8B_POOL_SLOTS) -> Workload:
     """Block-size sweep under fragmentation.  The pool keeps the same token
-    capacity for every block size (num_blocks = floor(428,560 / block_size), the
-    "block count halved" rule of page 1's experiment list).  Churn: ``events``
+    capacity for every block size (num_blocks = floor(428,560 / block_size), as
+    page 1's list of experiments halves the block count when the block size
+    doubles).  Churn: ``events``
     seeded events on background sequences, each either a create with a
     Geometric(1/mean_len) length capped at ``cap`` tokens or the release of a
     random live background sequence; then the batch of ``batch`` sequences
