@@ -314,6 +314,12 @@ def run_ours(args, world, rank, local):
         else:
             pa.pa_write_kv(k, v, slots, kc, vc)
 
+    def copy_op(kc, vc, pairs):
+        if fp8:
+            pa.pa_copy_blocks_fp8(kc, vc, pairs)
+        else:
+            pa.pa_copy_blocks(kc, vc, pairs)
+
     def decode_op(q, kc, vc, bt, lens, qsl=None, out=None, ws=None):
         out = inp["out"] if out is None else out
         ws = inp["ws"] if ws is None else ws
@@ -330,7 +336,7 @@ def run_ours(args, world, rank, local):
         kc, vc = st.caches[l]
         if with_write:
             if has_pairs:
-                pa.pa_copy_blocks(kc, vc, st.cow_pairs)
+                copy_op(kc, vc, st.cow_pairs)
             write_op(inp["k"], inp["v"], inp["slots"], kc, vc)
         if with_decode:
             decode_op(inp["q"], kc, vc, inp["bt"], inp["lens"], inp.get("qsl"))
@@ -474,7 +480,7 @@ def run_ours(args, world, rank, local):
                 kc, vc = st.caches[l]
                 main.wait_event(ready[l])
                 if has_pairs:
-                    pa.pa_copy_blocks(kc, vc, pairs_d)
+                    copy_op(kc, vc, pairs_d)
                 write_op(k_d[l], v_d[l], sm_d, kc, vc)
                 decode_op(q_d[l], kc, vc, bt_d, sl_d, qsl_d, out=out_d[l], ws=ws_d[l])
                 done = torch.cuda.Event()

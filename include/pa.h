@@ -343,6 +343,12 @@ PA_API int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_map
  * significant bits for the weights, as bf16 weights have in pa_decode), so
  * the result is within pa_decode's tolerance of the exact one.  A scale that
  * is not positive and finite gives PA_EINVAL. */
+/* pa_copy_blocks_fp8 -- pa_copy_blocks on an FP8 cache: the same whole-block
+ * copy-on-write copies, bit for bit, of block_size * num_kv_heads * head_dim
+ * one-byte codes per block and tensor (the scales are not used, but the
+ * descriptor must be valid).  Pairs and error behaviour as pa_copy_blocks. */
+PA_API int pa_copy_blocks_fp8(const pa_cache_fp8_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
+                              void *stream);
 PA_API size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
                                             const pa_cache_fp8_t *cache);
 PA_API int pa_decode_fp8(const void *q, const pa_cache_fp8_t *cache, const int32_t *block_tables,

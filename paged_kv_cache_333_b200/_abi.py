@@ -26,7 +26,7 @@ PA_DEVERR_QUERY_LOC = 32
 
 EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
             "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_map_to_kernel_blocks", "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
+            "pa_map_to_kernel_blocks", "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_copy_blocks_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
             "pa_decode_set_kernel", "pa_attention_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
@@ -76,6 +76,8 @@ lib.pa_attention.restype = ctypes.c_int
 PA_DECODE_STATIC_WS_BYTES = 8 * 1024 * 1024
 lib.pa_write_kv_fp8.argtypes = [_P, _P, _P, _i64, ctypes.POINTER(PaCacheFp8), _P]
 lib.pa_write_kv_fp8.restype = ctypes.c_int
+lib.pa_copy_blocks_fp8.argtypes = [ctypes.POINTER(PaCacheFp8), _P, _i64, _P]
+lib.pa_copy_blocks_fp8.restype = ctypes.c_int
 lib.pa_decode_fp8_workspace_bytes.argtypes = [_i32, _i32, _i32, ctypes.POINTER(PaCacheFp8)]
 lib.pa_decode_fp8_workspace_bytes.restype = ctypes.c_size_t
 lib.pa_decode_fp8.argtypes = [_P, ctypes.POINTER(PaCacheFp8), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
@@ -164,6 +166,17 @@ def pa_write_kv_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale: float, v_scal
     _check(lib.pa_write_kv_fp8(_dev(k, "k", torch.bfloat16), _dev(v, "v", torch.bfloat16),
                                _dev(slot_mapping, "slot_mapping", torch.int64), n, ctypes.byref(cache),
                                _stream_ptr(stream)), "pa_write_kv_fp8")
+
+
+def pa_copy_blocks_fp8(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
+    """cache[dst] = cache[src] for each (src, dst) row of an int64 [P, 2]
+    tensor, on FP8 caches (whole blocks of one-byte codes)."""
+    cache = make_cache_fp8(k_cache, v_cache, 1.0, 1.0)
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs, 2]")
+    p = src_dst_pairs.shape[0]
+    ptr = _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if p else None
+    _check(lib.pa_copy_blocks_fp8(ctypes.byref(cache), ptr, p, _stream_ptr(stream)), "pa_copy_blocks_fp8")
 
 
 def pa_decode_fp8_workspace_bytes(num_seqs: int, num_q_heads: int, max_seq_len: int, k_cache, v_cache,

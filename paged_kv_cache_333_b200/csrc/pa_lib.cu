@@ -612,6 +612,32 @@ int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_mapping, i
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "write_kv_fp8_kernel launch");
 }
 
+int pa_copy_blocks_fp8(const pa_cache_fp8_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
+                       void *stream) {
+    int rc = check_cache_fp8(cache);
+    if (rc)
+        return rc;
+    if (num_pairs < 0)
+        return PA_EINVAL;
+    if (num_pairs == 0)
+        return PA_OK;
+    if (!src_dst_pairs)
+        return PA_EINVAL;
+    if (num_pairs > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
+    // one byte per value: the same byte-level kernel with half the bf16 block size
+    const int64_t block_vecs = static_cast<int64_t>(cache->block_size) * cache->num_kv_heads * cache->head_dim / 16;
+    const int chunks = static_cast<int>((block_vecs + pa::kCopyChunkVecs - 1) / pa::kCopyChunkVecs);
+    const int64_t grid = num_pairs * 2 * chunks;
+    if (grid > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::copy_blocks_kernel, dim3(static_cast<unsigned>(grid)), dim3(pa::kCopyThreads),
+                               0, static_cast<cudaStream_t>(stream), static_cast<uint4 *>(cache->k_cache),
+                               static_cast<uint4 *>(cache->v_cache), src_dst_pairs, cache->num_blocks,
+                               block_vecs, chunks);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_kernel launch (fp8)");
+}
+
 size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
                                      const pa_cache_fp8_t *cache) {
     if (check_cache_fp8(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)

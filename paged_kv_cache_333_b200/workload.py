@@ -18,7 +18,7 @@ import dataclasses
 import numpy as np
 import torch
 
-from ._abi import (pa_copy_blocks, pa_decode, pa_decode_fp8, pa_decode_fp8_workspace_bytes,
+from ._abi import (pa_copy_blocks, pa_copy_blocks_fp8, pa_decode, pa_decode_fp8, pa_decode_fp8_workspace_bytes,
                    pa_decode_workspace_bytes, pa_write_kv, pa_write_kv_fp8)
 from .pool import BlockPool
 
@@ -121,7 +121,7 @@ def stage(w, device="cuda", layers: int = 1, rule: str = "shared", poison: bool 
         w.suffix_ops(pool)
     hist_pairs = pool.take_cow_pairs()
     if len(hist_pairs):
-        pa_copy_blocks(kc, vc, torch.from_numpy(hist_pairs).to(device))
+        (pa_copy_blocks_fp8 if fp8 else pa_copy_blocks)(kc, vc, torch.from_numpy(hist_pairs).to(device))
     _write_rows(w, pool, kc, vc,
                 [(sid, w.shared_len, pool.seq_len(sid)) for sid in w.seq_ids], device, fp8_scales=scales)
 
@@ -165,7 +165,7 @@ def run_step(st: DeviceStep, layer: int = 0, stream=None, out: torch.Tensor | No
     out = st.out if out is None else out
     if st.kv_dtype == "fp8":
         if st.cow_pairs.shape[0]:
-            raise NotImplementedError("copy-on-write pairs with an FP8 cache")
+            pa_copy_blocks_fp8(kc, vc, st.cow_pairs, stream=stream)
         pa_write_kv_fp8(st.k_new, st.v_new, st.slot_mapping, kc, vc, st.k_scale, st.v_scale, stream=stream)
         return pa_decode_fp8(st.q, kc, vc, st.k_scale, st.v_scale, st.block_tables, st.seq_lens, st.scale,
                              out=out, max_seq_len=st.max_seq_len, workspace=st.workspace, stream=stream)

@@ -86,6 +86,14 @@ def test_host_side_validation_of_the_widened_entry_points():
     for k_scale in (0.0, -1.0, float("inf"), float("nan")):
         bad = PaCacheFp8(16, 16, 64, 16, 2, 128, k_scale, 1.0)
         assert lib.pa_write_kv_fp8(16, 16, 16, 1, ctypes.byref(bad), None) == PA_EINVAL
+    assert lib.pa_copy_blocks_fp8(ctypes.byref(f8), None, 0, None) == 0
+    assert lib.pa_copy_blocks_fp8(ctypes.byref(f8), None, 3, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_fp8(ctypes.byref(f8), 16, -1, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_fp8(ctypes.byref(f8), 16, 2**31, None) == PA_EUNSUPPORTED
+    assert lib.pa_copy_blocks_fp8(ctypes.byref(PaCacheFp8(16, 16, 64, 12, 2, 128, 1.0, 1.0)), 16, 1,
+                                  None) == PA_EUNSUPPORTED  # block size not a power of two
+    assert lib.pa_copy_blocks_fp8(ctypes.byref(PaCacheFp8(16, 16, 64, 16, 2, 128, 0.0, 1.0)), 16, 1,
+                                  None) == PA_EINVAL        # the descriptor's scales must be valid
     bad_d = PaCacheFp8(16, 16, 64, 16, 2, 96, 1.0, 1.0)
     assert lib.pa_decode_fp8(16, ctypes.byref(bad_d), 16, 4, 16, 1, 64, 4, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
     assert lib.pa_decode_fp8(16, ctypes.byref(f8), 16, 4, 16, 1, 64, 6, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED

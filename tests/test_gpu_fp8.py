@@ -198,3 +198,83 @@ def test_fp8_workload_parity(pa, name):
     del st
     gc.collect()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,Hkv", [(16, 8), (1, 2), (64, 1)])
+def test_fp8_copy_blocks_bit_exact(pa, B, Hkv):
+    """pa_copy_blocks_fp8 copies whole blocks of codes bit for bit: every byte
+    of both caches equals the oracle's copy (applied to the same bytes, read
+    as 16-bit words); an out-of-range pair is skipped and flagged."""
+    gen = synth.make_rng(7100 + B + Hkv)
+    NB, D = 40, 128
+    k8 = gen.integers(0, 256, size=(NB, B, Hkv, D), dtype=np.uint8)
+    v8 = gen.integers(0, 256, size=(NB, B, Hkv, D), dtype=np.uint8)
+    pairs = np.array([[3, 10], [3, 11], [7, 12], [0, 39], [21, 2]], np.int64)  # distinct dsts, none a src
+    dk, dv = torch.from_numpy(k8).cuda(), torch.from_numpy(v8).cuda()
+    pa.pa_get_device_error(clear=True)
+    pa.pa_copy_blocks_fp8(dk, dv, torch.from_numpy(pairs).cuda())
+    torch.cuda.synchronize()
+    ek, ev = k8.copy(), v8.copy()
+    oracle.copy_blocks(pairs, ek.view(np.uint16), ev.view(np.uint16))
+    assert np.array_equal(dk.cpu().numpy(), ek) and np.array_equal(dv.cpu().numpy(), ev)
+    assert pa.pa_get_device_error(clear=True) == 0
+    # a pair naming a block past the pool is skipped; the valid one still runs
+    bad = torch.tensor([[5, NB], [6, 30]], dtype=torch.int64, device="cuda")
+    pa.pa_copy_blocks_fp8(dk, dv, bad)
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error(clear=True) == pa.PA_DEVERR_COPY_PAIR
+    oracle.copy_blocks(np.array([[6, 30]], np.int64), ek.view(np.uint16), ev.view(np.uint16))
+    assert np.array_equal(dk.cpu().numpy(), ek) and np.array_equal(dv.cpu().numpy(), ev)
+
+
+def test_fp8_prefix_copy_on_write_workload(pa):
+    """The prefix workload (256 sequences forked from a 2040-token prefix,
+    copy-on-write on first write) staged into FP8 caches: the copies run
+    through pa_copy_blocks_fp8, every code byte of both caches equals the
+    oracle's (which applies the same copies to the same bytes), and decode is
+    within tolerance of the fp8 oracle."""
+    from paged_kv_cache_333_b200.workload import run_step, stage
+    from oracle.pool import RefPool
+    w = synth.by_name("prefix")
+    st = stage(w, "cuda", kv_dtype="fp8", k_scale=KS, v_scale=VS)
+    assert st.history_pairs_np.shape[0] > 0  # the copies really ran
+    out = run_step(st)
+    torch.cuda.synchronize()
+    sh = w.shape
+    pool = RefPool(sh.num_blocks, sh.block_size, w.free_order)
+    w.ops(pool)
+    kc = np.full((sh.num_blocks, sh.block_size, sh.num_kv_heads, sh.head_dim), 0x7F, np.uint8)
+    vc = kc.copy()
+
+    def write(items):
+        for sid, a, b in items:
+            if b > a:
+                oracle.write_kv_fp8(np.ascontiguousarray(w.rows("k", sid, a, b)),
+                                    np.ascontiguousarray(w.rows("v", sid, a, b)), pool.slots(sid, a, b - a),
+                                    kc, vc, KS, VS)
+
+    def copy(pairs):
+        if len(pairs):
+            oracle.copy_blocks(np.array(pairs, np.int64), kc.view(np.uint16), vc.view(np.uint16))
+
+    write([(w.seq_ids[0], 0, w.shared_len)])
+    w.suffix_ops(pool)
+    copy(pool.take_cow_pairs())
+    write([(sid, w.shared_len, pool.seq_len(sid)) for sid in w.seq_ids])
+    for sid in w.seq_ids:
+        assert pool.append(sid, w.step_tokens)
+    copy(pool.take_cow_pairs())
+    lens = np.array([pool.seq_len(s) for s in w.seq_ids], np.int32)
+    write([(s, int(n) - w.step_tokens, int(n)) for s, n in zip(w.seq_ids, lens)])
+    bt = pool.block_table(w.seq_ids, st.block_tables_np.shape[1])
+    assert np.array_equal(bt, st.block_tables_np) and np.array_equal(lens, st.seq_lens_np)
+    assert np.array_equal(st.caches[0][0].cpu().numpy(), kc) and np.array_equal(st.caches[0][1].cpu().numpy(), vc)
+    # decode checked on every 11th sequence (24 of 256; the oracle reads the same caches)
+    pick = np.arange(0, len(w.seq_ids), 11)
+    ref = oracle.decode_fp8(np.ascontiguousarray(w.q[pick]), kc, vc, np.ascontiguousarray(bt[pick]),
+                            np.ascontiguousarray(lens[pick]), w.scale, KS, VS)
+    _close(out[torch.from_numpy(pick).cuda()], ref, "prefix")
+    assert pa.pa_get_device_error(clear=True) == 0
+    del st
+    gc.collect()
+    torch.cuda.empty_cache()
