@@ -1,6 +1,7 @@
 """The multi-GPU path is replicas only: every rank runs the whole step on its
 own GPU, the device times are combined as a max over ranks, and only rank 0
 prints.  These tests run that host-side plumbing as two gloo ranks on CPU."""
+import datetime
 import io
 import json
 import os
@@ -24,7 +25,9 @@ def _free_port():
 def _worker(rank, world, port, q):
     sys.path.insert(0, ROOT)
     import bench
-    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    # a short timeout: a rank whose peer is gone fails instead of waiting
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=30))
     try:
         # per-rank device times differ; the job time is the slowest rank's
         ms = bench.reduce_max(10.0 + 5.0 * rank, "cpu")
@@ -48,12 +51,18 @@ def test_two_gloo_ranks_take_the_max_time_and_rank0_prints():
     for p in procs:
         p.start()
     out = {}
-    for _ in range(2):
-        rank, ms, rate, text = q.get(timeout=120)
-        out[rank] = (ms, rate, text)
-    for p in procs:
-        p.join(timeout=60)
-        assert p.exitcode == 0
+    try:
+        for _ in range(2):
+            rank, ms, rate, text = q.get(timeout=120)
+            out[rank] = (ms, rate, text)
+        for p in procs:
+            p.join(timeout=60)
+            assert p.exitcode == 0
+    finally:
+        for p in procs:  # the workers this test started, if any is still running
+            if p.is_alive():
+                p.terminate()
+                p.join(timeout=10)
     assert out[0][0] == out[1][0] == 15.0
     assert out[0][1] == pytest.approx(2 * 2e9 / 15e-3 / 1e9)
     line = json.loads(out[0][2])
