@@ -349,6 +349,11 @@ PA_API int pa_write_kv_fp8(const void *k, const void *v, const int64_t *slot_map
  * descriptor must be valid).  Pairs and error behaviour as pa_copy_blocks. */
 PA_API int pa_copy_blocks_fp8(const pa_cache_fp8_t *cache, const int64_t *src_dst_pairs, int64_t num_pairs,
                               void *stream);
+/* pa_copy_blocks_layers_fp8 -- pa_copy_blocks_fp8 for every layer in one
+ * launch, as pa_copy_blocks_layers (caches: HOST array of num_layers <= 128
+ * FP8 descriptors with one block geometry). */
+PA_API int pa_copy_blocks_layers_fp8(const pa_cache_fp8_t *caches, int32_t num_layers,
+                                     const int64_t *src_dst_pairs, int64_t num_pairs, void *stream);
 PA_API size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
                                             const pa_cache_fp8_t *cache);
 PA_API int pa_decode_fp8(const void *q, const pa_cache_fp8_t *cache, const int32_t *block_tables,

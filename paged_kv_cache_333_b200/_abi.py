@@ -26,7 +26,7 @@ PA_DEVERR_QUERY_LOC = 32
 
 EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "pa_copy_blocks",
             "pa_copy_blocks_layers", "pa_decode_workspace_bytes", "pa_decode",
-            "pa_map_to_kernel_blocks", "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_copy_blocks_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
+            "pa_map_to_kernel_blocks", "pa_decode_static_ws", "pa_attention_workspace_bytes", "pa_attention", "pa_write_kv_fp8", "pa_copy_blocks_fp8", "pa_copy_blocks_layers_fp8", "pa_decode_fp8", "pa_decode_fp8_workspace_bytes",
             "pa_decode_set_kernel", "pa_attention_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
@@ -78,6 +78,8 @@ lib.pa_write_kv_fp8.argtypes = [_P, _P, _P, _i64, ctypes.POINTER(PaCacheFp8), _P
 lib.pa_write_kv_fp8.restype = ctypes.c_int
 lib.pa_copy_blocks_fp8.argtypes = [ctypes.POINTER(PaCacheFp8), _P, _i64, _P]
 lib.pa_copy_blocks_fp8.restype = ctypes.c_int
+lib.pa_copy_blocks_layers_fp8.argtypes = [ctypes.POINTER(PaCacheFp8), _i32, _P, _i64, _P]
+lib.pa_copy_blocks_layers_fp8.restype = ctypes.c_int
 lib.pa_decode_fp8_workspace_bytes.argtypes = [_i32, _i32, _i32, ctypes.POINTER(PaCacheFp8)]
 lib.pa_decode_fp8_workspace_bytes.restype = ctypes.c_size_t
 lib.pa_decode_fp8.argtypes = [_P, ctypes.POINTER(PaCacheFp8), _P, _i32, _P, _i32, _i32, _i32, ctypes.c_float,
@@ -177,6 +179,16 @@ def pa_copy_blocks_fp8(k_cache, v_cache, src_dst_pairs, stream=None) -> None:
     p = src_dst_pairs.shape[0]
     ptr = _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if p else None
     _check(lib.pa_copy_blocks_fp8(ctypes.byref(cache), ptr, p, _stream_ptr(stream)), "pa_copy_blocks_fp8")
+
+
+def pa_copy_blocks_layers_fp8(caches, src_dst_pairs, stream=None) -> None:
+    """pa_copy_blocks_fp8 over a list of (k_cache, v_cache) FP8 layers, one launch."""
+    arr = (PaCacheFp8 * max(1, len(caches)))(*[make_cache_fp8(k, v, 1.0, 1.0) for k, v in caches])
+    if src_dst_pairs.dim() != 2 or src_dst_pairs.shape[1] != 2:
+        raise ValueError("src_dst_pairs must be [num_pairs, 2]")
+    p = src_dst_pairs.shape[0]
+    ptr = _dev(src_dst_pairs, "src_dst_pairs", torch.int64) if p else None
+    _check(lib.pa_copy_blocks_layers_fp8(arr, len(caches), ptr, p, _stream_ptr(stream)), "pa_copy_blocks_layers_fp8")
 
 
 def pa_decode_fp8_workspace_bytes(num_seqs: int, num_q_heads: int, max_seq_len: int, k_cache, v_cache,

@@ -638,6 +638,40 @@ int pa_copy_blocks_fp8(const pa_cache_fp8_t *cache, const int64_t *src_dst_pairs
     return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_kernel launch (fp8)");
 }
 
+int pa_copy_blocks_layers_fp8(const pa_cache_fp8_t *caches, int32_t num_layers, const int64_t *src_dst_pairs,
+                              int64_t num_pairs, void *stream) {
+    if (!caches || num_layers < 0 || num_layers > pa::kMaxLayers || num_pairs < 0)
+        return num_layers > pa::kMaxLayers ? PA_EUNSUPPORTED : PA_EINVAL;
+    pa::LayerPtrs lp{};
+    for (int32_t l = 0; l < num_layers; ++l) {
+        const int rc = check_cache_fp8(&caches[l]);
+        if (rc)
+            return rc;
+        if (caches[l].num_blocks != caches[0].num_blocks || caches[l].block_size != caches[0].block_size ||
+            caches[l].num_kv_heads != caches[0].num_kv_heads)
+            return PA_EINVAL;  // one pair list needs one block geometry
+        lp.k[l] = static_cast<uint4 *>(caches[l].k_cache);
+        lp.v[l] = static_cast<uint4 *>(caches[l].v_cache);
+    }
+    if (num_layers == 0 || num_pairs == 0)
+        return PA_OK;
+    if (!src_dst_pairs)
+        return PA_EINVAL;
+    if (num_pairs > INT32_MAX)
+        return PA_EUNSUPPORTED;  // beyond any grid (and keeps the size arithmetic below in range)
+    const pa_cache_fp8_t *c = &caches[0];
+    // one byte per value: the byte-level kernel with the FP8 block size
+    const int64_t block_vecs = static_cast<int64_t>(c->block_size) * c->num_kv_heads * c->head_dim / 16;
+    const int chunks = static_cast<int>((block_vecs + pa::kCopyChunkVecs - 1) / pa::kCopyChunkVecs);
+    const int64_t grid = num_pairs * 2 * chunks;
+    if (grid > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    cudaError_t e = launch_pdl(pa::copy_blocks_layers_kernel, dim3(static_cast<unsigned>(grid), num_layers),
+                               dim3(pa::kCopyThreads), 0, static_cast<cudaStream_t>(stream), lp, src_dst_pairs,
+                               c->num_blocks, block_vecs, chunks);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks_layers_kernel launch (fp8)");
+}
+
 size_t pa_decode_fp8_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t max_seq_len,
                                      const pa_cache_fp8_t *cache) {
     if (check_cache_fp8(cache) != PA_OK || num_seqs <= 0 || num_q_heads <= 0 || max_seq_len < 0)

@@ -94,6 +94,14 @@ def test_host_side_validation_of_the_widened_entry_points():
                                   None) == PA_EUNSUPPORTED  # block size not a power of two
     assert lib.pa_copy_blocks_fp8(ctypes.byref(PaCacheFp8(16, 16, 64, 16, 2, 128, 0.0, 1.0)), 16, 1,
                                   None) == PA_EINVAL        # the descriptor's scales must be valid
+    layers8 = (PaCacheFp8 * 2)(f8, f8)
+    assert lib.pa_copy_blocks_layers_fp8(layers8, 2, None, 0, None) == 0
+    assert lib.pa_copy_blocks_layers_fp8(layers8, 2, None, 4, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_layers_fp8(None, 2, 16, 4, None) == PA_EINVAL
+    assert lib.pa_copy_blocks_layers_fp8(layers8, 129, 16, 4, None) == PA_EUNSUPPORTED
+    assert lib.pa_copy_blocks_layers_fp8(layers8, 2, 16, 2**31, None) == PA_EUNSUPPORTED
+    mixed8 = (PaCacheFp8 * 2)(f8, PaCacheFp8(32, 32, 64, 16, 4, 128, 1.0, 1.0))  # two geometries
+    assert lib.pa_copy_blocks_layers_fp8(mixed8, 2, 16, 4, None) == PA_EINVAL
     bad_d = PaCacheFp8(16, 16, 64, 16, 2, 96, 1.0, 1.0)
     assert lib.pa_decode_fp8(16, ctypes.byref(bad_d), 16, 4, 16, 1, 64, 4, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED
     assert lib.pa_decode_fp8(16, ctypes.byref(f8), 16, 4, 16, 1, 64, 6, 0.1, 16, None, 0, None) == PA_EUNSUPPORTED

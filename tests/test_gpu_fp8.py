@@ -278,3 +278,23 @@ def test_fp8_prefix_copy_on_write_workload(pa):
     del st
     gc.collect()
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,Hkv", [(16, 8), (2, 2)])
+def test_fp8_copy_blocks_layers_bit_exact(pa, B, Hkv):
+    """pa_copy_blocks_layers_fp8: one launch copies the pairs in every layer's
+    FP8 caches, each layer bit-exact against the oracle's copy of its bytes."""
+    gen = synth.make_rng(7200 + B + Hkv)
+    NB, D, L = 24, 128, 3
+    pairs = np.array([[1, 20], [4, 21], [4, 22], [9, 0]], np.int64)
+    host = [(gen.integers(0, 256, size=(NB, B, Hkv, D), dtype=np.uint8),
+             gen.integers(0, 256, size=(NB, B, Hkv, D), dtype=np.uint8)) for _ in range(L)]
+    dev = [(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda()) for k, v in host]
+    pa.pa_get_device_error(clear=True)
+    pa.pa_copy_blocks_layers_fp8(dev, torch.from_numpy(pairs).cuda())
+    torch.cuda.synchronize()
+    for (k, v), (dk, dv) in zip(host, dev):
+        ek, ev = k.copy(), v.copy()
+        oracle.copy_blocks(pairs, ek.view(np.uint16), ev.view(np.uint16))
+        assert np.array_equal(dk.cpu().numpy(), ek) and np.array_equal(dv.cpu().numpy(), ev)
+    assert pa.pa_get_device_error(clear=True) == 0
