@@ -81,3 +81,23 @@ def test_reference_arm_prints_one_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_clock_samples_give_median_max_and_active_reasons():
+    """The bench line's `clocks` field from nvidia-smi samples: median SM clock
+    under load, the max clock, the throttle reasons seen Active, and only
+    this GPU's rows when the sampler knows its UUID (other GPUs ignored)."""
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.uuid = "GPU-aaa"
+    s.proc = types.SimpleNamespace(terminate=lambda: None, wait=lambda timeout=None: 0, kill=lambda: None)
+    row = "{u}, {sm}, 1965, 700.5, 0x0, Not Active, Not Active, {swt}, {cap}"
+    s.lines = [row.format(u="GPU-aaa", sm=1965, swt="Not Active", cap="Not Active"),
+               row.format(u="GPU-aaa", sm=1900, swt="Not Active", cap="Active"),
+               row.format(u="GPU-aaa", sm=1800, swt="Not Active", cap="Not Active"),
+               row.format(u="GPU-bbb", sm=300, swt="Active", cap="Active"),   # another GPU on the host
+               "garbage line"]
+    c = bench.ClockSampler.stop(s)
+    assert c["sm_mhz"] == 1900 and c["sm_max_mhz"] == 1965 and c["samples"] == 3
+    assert c["reasons"] == ["sw_power_cap"]
+    s.proc = None
+    assert bench.ClockSampler.stop(s)["reasons"] == ["nvidia-smi unavailable"]
