@@ -101,3 +101,13 @@ def test_clock_samples_give_median_max_and_active_reasons():
     assert c["reasons"] == ["sw_power_cap"]
     s.proc = None
     assert bench.ClockSampler.stop(s)["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_roofline_peak_reads_the_measured_file_else_falls_back(tmp_path, monkeypatch):
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peak, how = bench.measured_peak()
+    assert peak == bench.FALLBACK_HBM_GBS and how.startswith("fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6558.4, "bf16_tflops": 1590}))
+    peak, how = bench.measured_peak()
+    assert peak == 6558.4 and how.startswith("measured")
