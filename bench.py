@@ -14,10 +14,12 @@ attention.  Inputs are resident in HBM when the timed region starts.
   roofline = the decode kernel alone: unique KV bytes per launch / its mean
            duration (CUDA events on its stream) vs. measured HBM peak.
 
---impl reference times the CPU oracle (one thread) on a bounded sample of
-the same workload.  With torchrun (N > 1) every rank runs its own replica
-(the path does not shard; no collective is needed) and the time is the max
-over ranks.
+--impl reference times the CPU oracle (its (sequence, head) pairs split over
+the host's cores) on a bounded sample of the same workload.  The default run
+also reports the oracle in cpu_baseline, with a one-thread timing beside it,
+and times the 32K long-context decode under per_config.  With torchrun
+(N > 1) every rank runs its own replica (the path does not shard; no
+collective is needed) and the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -76,8 +78,14 @@ def parse_args():
     ap.add_argument("--queries", type=int, default=1,
                     help="query rows per request: 1 = decode (pa_decode); Q > 1 = the last Q tokens of every "
                          "request are its rows (speculative decode / prefill chunk; pa_attention)")
+    ap.add_argument("--attention-kernel", choices=["default", "mma", "tcgen05"], default="default",
+                    help="pa_attention kernel for --queries > 1 (default = the library's own choice)")
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8"], default="bf16",
                     help="KV cache element type (fp8 = OCP E4M3 codes with per-tensor scales)")
+    ap.add_argument("--extra-configs", default="auto",
+                    help="comma-separated workloads whose bf16 decode is also timed in this run and reported "
+                         "under per_config (auto = the 32K long-context one when the main run is the chat "
+                         "decode; none = no extra)")
     args = ap.parse_args()
     if args.queries > 1 and args.kv_dtype == "fp8":
         ap.error("--queries > 1 runs pa_attention, which reads a bf16 cache: use --kv-dtype bf16")
@@ -159,7 +167,12 @@ class ClockSampler:
         rows = [r.split(", ") for r in self.lines if r.count(",") >= 8]
         if self.uuid:
             mine = [r for r in rows if r[0].strip() == self.uuid]
-            rows = mine or rows
+            if rows and not mine:
+                # Samples came back, none of them for this GPU: report no
+                # clock rather than other jobs' clocks and throttle reasons.
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["uuid not matched"],
+                        "samples": 0, "uuid": self.uuid}
+            rows = mine
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -261,6 +274,37 @@ def host_pool_step_us(w, steps: int = 200) -> dict:
                     "(updated append-only) + lengths, one ctypes call on arrays allocated once, one host thread"}
 
 
+# --------------------------------------------------------------------------- timing
+def capture_graph(fn, dev):
+    """One CUDA graph of `fn`'s launches (no host work in the timed loop)."""
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            fn()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    return g
+
+
+def timed_replays(g, reps, dev, world):
+    """Device milliseconds of `reps` replays of graph g, with CUDA events on
+    the replay stream, a barrier and a synchronize on both sides; the max over
+    ranks."""
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0.record()
+    for _ in range(reps):
+        g.replay()
+    t1.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    return reduce_max(t0.elapsed_time(t1), dev)
+
+
 # --------------------------------------------------------------------------- ours
 def run_ours(args, world, rank, local):
     import synth
@@ -271,6 +315,8 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     if args.part_tokens:
         pa.pa_decode_set_partition_tokens(args.part_tokens)
+    if args.attention_kernel != "default":
+        pa.pa_attention_set_kernel(args.attention_kernel)
     w = synth.by_name(args.config)
     fp8 = args.kv_dtype == "fp8"
     st = stage(w, dev, layers=args.layers, kv_dtype=args.kv_dtype)
@@ -341,32 +387,8 @@ def run_ours(args, world, rank, local):
         if with_decode:
             decode_op(inp["q"], kc, vc, inp["bt"], inp["lens"], inp.get("qsl"))
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
-    def capture(fn):
-        """One CUDA graph of `fn`'s launches (no host work in the timed loop)."""
-        g = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(g, stream=side):
-                fn()
-        torch.cuda.current_stream(dev).wait_stream(side)
-        return g
-
-    def timed(g, reps):
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        torch.cuda.synchronize()
-        t0.record()
-        for _ in range(reps):
-            g.replay()
-        t1.record()
-        torch.cuda.synchronize()
-        barrier()
-        return reduce_max(t0.elapsed_time(t1), dev)
+    capture = lambda fn: capture_graph(fn, dev)
+    timed = lambda g, reps: timed_replays(g, reps, dev, world)
 
     # eager warm-up (kernel attributes, tensor maps), then graphs
     for l in range(L):
@@ -525,6 +547,7 @@ def run_ours(args, world, rank, local):
                         + (f"; {Q} query rows per sequence (its last {Q} tokens, causal), pa_attention" if Q > 1
                            else ""),
             "query_rows_per_seq": Q,
+            "attention_kernel": args.attention_kernel if Q > 1 else None,
             "layers_per_step": L,
             "batch": S,
             "block_size": st.block_size,
@@ -560,10 +583,99 @@ def run_ours(args, world, rank, local):
         "gpu_launches": K * L * launches_per_layer,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and Q == 1:
-        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
-    if rank == 0:
-        print(json.dumps(result), flush=True)
+    return result, w
+
+
+def extra_configs(args) -> list:
+    """Workloads timed after the main one: by default the long-context
+    decode, the second configuration the bandwidth target names, when the
+    main run is the bf16 chat decode."""
+    if args.extra_configs == "auto":
+        default = args.config == "chat" and args.queries == 1 and args.kv_dtype == "bf16" and not args.part_tokens
+        return ["long"] if default else []
+    if args.extra_configs in ("", "none"):
+        return []
+    names = [n.strip() for n in args.extra_configs.split(",") if n.strip()]
+    return [n for n in names if n != args.config]
+
+
+def time_decode_config(name, args, world, local) -> dict:
+    """The bf16 decode step of workload `name`, staged and timed like the main
+    one: --layers distinct layer caches, a CUDA graph of the whole step
+    (queued copies, the KV write, pa_decode per layer) and one of the decode
+    calls alone, each replayed --steps times after --warmup replays, clocks
+    sampled during the step replays.  Returns the per-config record."""
+    import synth
+    import paged_kv_cache_333_b200 as pa
+    from paged_kv_cache_333_b200.workload import stage
+
+    dev = torch.device("cuda", local)
+    w = synth.by_name(name)
+    st = stage(w, dev, layers=args.layers)
+    L, K = args.layers, args.steps
+    nbytes = algorithmic_bytes(st)
+    step_bytes = L * (nbytes["decode_kv"] + nbytes["write"] + nbytes["copy"])
+    has_pairs = st.cow_pairs.shape[0] > 0
+    split = st.workspace is not None
+
+    def layer_ops(l, with_write=True):
+        kc, vc = st.caches[l]
+        if with_write:
+            if has_pairs:
+                pa.pa_copy_blocks(kc, vc, st.cow_pairs)
+            pa.pa_write_kv(st.k_new, st.v_new, st.slot_mapping, kc, vc)
+        pa.pa_decode(st.q, kc, vc, st.block_tables, st.seq_lens, st.scale, out=st.out,
+                     max_seq_len=st.max_seq_len, workspace=st.workspace)
+
+    for l in range(L):
+        layer_ops(l)
+    torch.cuda.synchronize()
+    g_step = capture_graph(lambda: [layer_ops(l) for l in range(L)], dev)
+    g_dec = capture_graph(lambda: [layer_ops(l, with_write=False) for l in range(L)], dev)
+    for _ in range(args.warmup):
+        g_step.replay()
+    torch.cuda.synchronize()
+    assert pa.pa_get_device_error(clear=True) == 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms_total = timed_replays(g_step, K, dev, world)
+    clk = clocks.stop()
+    for _ in range(args.warmup):
+        g_dec.replay()
+    dec_ms_total = timed_replays(g_dec, K, dev, world)
+    assert pa.pa_get_device_error(clear=True) == 0
+    ms_step = ms_total / K
+    dec_mean_ms = dec_ms_total / (K * L)
+    peak, peak_src = measured_peak()
+    achieved = nbytes["decode_kv"] / (dec_mean_ms * 1e-3) / 1e9
+    value = whole_job_rate(world, step_bytes, ms_step * 1e-3)
+    S = len(st.ids)
+    rec = {
+        "workload": WORKLOAD_TEXT.get(name, name),
+        "batch": S, "block_size": st.block_size, "num_blocks": st.num_blocks, "max_seq_len": st.max_seq_len,
+        "layers_per_step": L, "steps": K, "warmup": args.warmup,
+        "value": round(value, 2), "unit": "GB/s", "ms_per_step": round(ms_step, 4),
+        "decode_us_per_layer": round(dec_mean_ms * 1e3, 3),
+        "decode_tokens_per_s_per_layer": round(world * S / (dec_mean_ms * 1e-3), 1),
+        "pct_of_peak": {"measured": round(100 * achieved / peak, 2),
+                        "nominal_8tbs": round(100 * achieved / NOMINAL_HBM_GBS, 2)},
+        "per_op_bytes_per_layer": nbytes,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic(name, "bf16"),
+                     "kernel": "pa_decode (partition kernel" + (" + LSE merge)" if split else ")"),
+                     "mean_launch_us": round(dec_mean_ms * 1e3, 3), "bytes_per_launch": nbytes["decode_kv"],
+                     "how": f"CUDA graph of {L} back-to-back pa_decode calls (one per layer cache), {K} replays "
+                            "timed with CUDA events on the replay stream; mean per call",
+                     "peak_source": peak_src},
+        "l2": f"inputs larger than L2: {L} distinct layer caches, {L * nbytes['decode_kv'] / 1e9:.2f} GB of KV "
+              "touched per step",
+        "gpu_launches": K * L * (2 + (1 if split else 0) + (1 if has_pairs else 0)),
+        "clocks": clk,
+    }
+    del g_step, g_dec, st
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
 # --------------------------------------------------------------------------- oracle
@@ -585,48 +697,90 @@ def _oracle_layer(w, ref, sample_seqs):
     oracle.decode(w.q, ref["k_cache"], ref["v_cache"], ref["block_tables"], ref["seq_lens"], w.scale, which)
 
 
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
+def _oracle_layer_threads(w, ref, pool, threads: int):
+    """One layer of the oracle's decode, its (sequence, head) pairs split into
+    `threads` disjoint contiguous shares, one oracle call per share on a
+    worker thread.  The oracle is unchanged: a C call through ctypes, which
+    releases the interpreter lock and keeps no global state, so the calls
+    run in parallel on the host's cores."""
+    import oracle
+    pairs = np.array([(s, j) for s in range(len(w.seq_ids)) for j in range(w.shape.num_q_heads)], np.int32)
+    shares = [a for a in np.array_split(pairs, threads) if len(a)]
+    futs = [pool.submit(oracle.decode, w.q, ref["k_cache"], ref["v_cache"], ref["block_tables"], ref["seq_lens"],
+                        w.scale, a) for a in shares]
+    for f in futs:
+        f.result()
+
+
 def cpu_baseline(w, seconds: float) -> dict:
-    """The oracle (plain C, fp64, one thread) on a bounded sample: whole
-    layers of the same workload, repeated until `seconds` have passed."""
+    """The oracle (plain C, fp64) on bounded samples of the same workload:
+    whole layers, repeated until `seconds` have passed, fanned out over all
+    the host's cores (the reported value), and on one thread."""
+    from concurrent.futures import ThreadPoolExecutor
     ref, kv_bytes = _oracle_setup(w)
     S = len(w.seq_ids)
-    t0 = time.perf_counter()
-    layers = 0
-    while True:
-        _oracle_layer(w, ref, range(S))
-        layers += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": round(layers * kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{layers} full layer(s) of the same workload ({S} seqs x {w.shape.num_q_heads} heads), "
-                      f"{dt:.1f} s, decode only"}
+    cores = host_cores()
+
+    def run(fn, budget):
+        t0 = time.perf_counter()
+        layers = 0
+        while True:
+            fn()
+            layers += 1
+            if time.perf_counter() - t0 >= budget:
+                break
+        return layers, time.perf_counter() - t0
+
+    with ThreadPoolExecutor(max_workers=cores) as pool:
+        ln, dt = run(lambda: _oracle_layer_threads(w, ref, pool, cores), seconds / 2)
+    l1, dt1 = run(lambda: _oracle_layer(w, ref, range(S)), seconds / 2)
+    what = f"({S} seqs x {w.shape.num_q_heads} heads), decode only"
+    return {"value": round(ln * kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cores_available": cores,
+            "sample": f"{ln} full layer(s) of the same workload {what}, {dt:.1f} s; its (sequence, head) pairs "
+                      f"split over {cores} threads, one oracle call each",
+            "single_thread": {"value": round(l1 * kv_bytes / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "sample": f"{l1} full layer(s) {what}, {dt1:.1f} s, one thread"}}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return
+    from concurrent.futures import ThreadPoolExecutor
     import synth
     w = synth.by_name(args.config)
     ref, kv_bytes = _oracle_setup(w)
     S = len(w.seq_ids)
-    # one step = one full layer of the workload's decode, on one host thread
-    for _ in range(args.warmup):
-        _oracle_layer(w, ref, range(min(S, 8)))
+    cores = host_cores()
+    # one step = one full layer of the workload's decode, its (sequence,
+    # head) pairs split over the host's cores
     times = []
-    for _ in range(args.steps):
-        t = time.perf_counter()
-        _oracle_layer(w, ref, range(S))
-        times.append(time.perf_counter() - t)
+    with ThreadPoolExecutor(max_workers=cores) as pool:
+        for _ in range(args.warmup):
+            _oracle_layer(w, ref, range(min(S, 8)))
+        for _ in range(args.steps):
+            t = time.perf_counter()
+            _oracle_layer_threads(w, ref, pool, cores)
+            times.append(time.perf_counter() - t)
     ms_step = 1e3 * statistics.mean(times)
     value = kv_bytes / (ms_step * 1e-3) / 1e9
-    sample = f"{args.steps} steps of one full layer ({S} seqs x {w.shape.num_q_heads} heads), decode only"
+    sample = (f"{args.steps} steps of one full layer ({S} seqs x {w.shape.num_q_heads} heads, split over {cores} "
+              "threads), decode only")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT.get(args.config, args.config), "layers_per_step": 1},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "decode_tokens_per_s_per_layer": round(S / (ms_step * 1e-3), 2),
     }), flush=True)
@@ -642,7 +796,16 @@ def main():
         if args.impl == "reference":
             run_reference(args, world, rank)
         else:
-            run_ours(args, world, rank, local)
+            result, w = run_ours(args, world, rank, local)
+            # the other configurations the bandwidth target names, each timed
+            # the same way in this process after the main one's caches are freed
+            for name in extra_configs(args):
+                torch.cuda.empty_cache()
+                result.setdefault("per_config", {})[name] = time_decode_config(name, args, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline and args.queries == 1:
+                result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+            if rank == 0:
+                print(json.dumps(result), flush=True)
     finally:
         if world > 1 and torch.distributed.is_initialized():
             torch.distributed.destroy_process_group()

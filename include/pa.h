@@ -252,6 +252,15 @@ PA_API int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_
                         int32_t num_q_heads, float scale, void *out, void *workspace, size_t workspace_bytes,
                         void *stream);
 
+/* ------------------------------------------------------------------------
+ * Tuning knobs.  The three setters below change one process-wide setting
+ * each, which every later call from every host thread reads, including
+ * calls made by any other user of this library in the same process.  They
+ * exist for measurement and tests; a library user should leave them at their
+ * defaults, or set them once at start-up and restore the previous value
+ * (each setter returns it) when done.  Each call reads each setting once.
+ * ------------------------------------------------------------------------ */
+
 /* Which partition kernel pa_decode runs (process wide; returns the previous
  * value; other values are ignored).  Both compute the same result within
  * the stated tolerance.
@@ -295,11 +304,18 @@ PA_API int32_t pa_decode_set_partition_tokens(int32_t tokens);
  *   larger returns PA_EWORKSPACE (message in pa_last_cuda_error) and enqueues
  *   nothing.  The call allocates nothing.
  *   Set-up: the first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current and caches it; make that
- *   first call before any stream capture.  A call with num_seqs = 0 does only
- *   this set-up and enqueues nothing.
- *   Errors: the argument checks of pa_decode, then the scratch size check,
- *   run on the host before any CUDA call.
+ *   (cudaGetSymbolAddress) with that device current and caches it with the
+ *   id of the device's current context; make that first call before any
+ *   stream capture.  A device reset (cudaDeviceReset) gives the device a new
+ *   context, in which the library's module is loaded afresh; the next call
+ *   sees the new context id and looks the address up again, so make the
+ *   first call after a reset outside stream capture too.  A call with
+ *   num_seqs = 0 does only this set-up and enqueues nothing.
+ *   Errors: the argument checks of pa_decode run first, on the host alone.
+ *   The scratch size check follows; it asks the CUDA runtime for the
+ *   device's SM count (the split-K partition size depends on it), which
+ *   can replace a runtime error the caller left pending on this thread.
+ *   Neither check enqueues anything.
  *   Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents (nothing in it needs to start at zero).  Calls that may
  *   overlap on the GPU (other streams, other host threads) race on it:

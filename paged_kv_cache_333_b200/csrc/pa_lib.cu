@@ -56,14 +56,54 @@ int check_cache(const pa_cache_t *c) {
     return PA_OK;
 }
 
+// SM count of the current device, read once per device through the CUDA
+// runtime.  If no device can be queried (a host without a GPU), 148 (B200)
+// is assumed and the runtime error the failed query recorded is cleared, so
+// that the caller's next error check does not see it.  A host-side call that
+// reaches this function (the workspace sizes, the launch shapes) may thereby
+// clear a runtime error the caller left pending on this thread.
 int sm_count() {
+    static std::atomic<int> cached[64] = {};
     int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
-        cudaGetLastError();  // clear a sticky "no device" error from the query
-        return 148;          // B200
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
     }
+    if (dev >= 0 && dev < 64 && (n = cached[dev].load(std::memory_order_relaxed)) > 0)
+        return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    if (dev >= 0 && dev < 64)
+        cached[dev].store(n, std::memory_order_relaxed);
     return n;
+}
+
+// Unique id of the calling thread's current CUDA context, 0 when there is
+// none or it cannot be read.  Ids are never reused within a process, so
+// per-device set-up cached under the id is redone after the device's
+// primary context is destroyed and created anew (cudaDeviceReset), which
+// reloads this library's module and resets kernel attributes.
+unsigned long long current_ctx_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
 }
 
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -195,13 +235,17 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Per-device record of the context a one-time set-up was done in.
+using CtxDone = std::atomic<unsigned long long>[64];
+
 // Opt a kernel into its dynamic shared memory and the all-shared carveout
-// (so that its CTAs-per-SM target fits), once per device.
+// (so that its CTAs-per-SM target fits), once per device and context.
 template <typename K>
-int prepare_kernel(K kernel, size_t smem, std::atomic<bool> (&done)[64]) {
+int prepare_kernel(K kernel, size_t smem, CtxDone &done) {
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire))
+    const unsigned long long ctx = current_ctx_id();
+    if (ctx != 0 && dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire) == ctx)
         return PA_OK;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -211,8 +255,8 @@ int prepare_kernel(K kernel, size_t smem, std::atomic<bool> (&done)[64]) {
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
-    if (dev >= 0 && dev < 64)
-        done[dev].store(true, std::memory_order_release);  // setting the attributes twice is harmless
+    if (dev >= 0 && dev < 64)  // the context the attributes were set in (setting them twice is harmless)
+        done[dev].store(current_ctx_id(), std::memory_order_release);
     return PA_OK;
 }
 
@@ -231,7 +275,7 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
         const int64_t ctas = static_cast<int64_t>(grid.x) * grid.y * grid.z;
         const bool one_wave = ctas <= static_cast<int64_t>(sm_count()) * pa::kMmaCtasPerSm;
         const bool two = one_wave || p.num_parts > 16;
-        static std::atomic<bool> done2[64] = {}, done3[64] = {};
+        static CtxDone done2 = {}, done3 = {};
         int rc = two ? prepare_kernel(pa::decode_partition_mma_kernel<G, 2>, pa::kDecodeSmemBytesM, done2)
                      : prepare_kernel(pa::decode_partition_mma_kernel<G, 3>, pa::kDecodeSmemBytesM, done3);
         if (rc)
@@ -243,7 +287,7 @@ int launch_decode_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Deco
         if (e != cudaSuccess)
             return cuda_fail(e, "decode_partition_mma_kernel launch");
     } else {
-        static std::atomic<bool> done[64] = {};
+        static CtxDone done = {};
         int rc = prepare_kernel(pa::decode_partition_kernel<G>, pa::kDecodeSmemBytes, done);
         if (rc)
             return rc;
@@ -313,7 +357,7 @@ int launch_row_merge(const pa::AttendParams &ap, cudaStream_t stream) {
 template <int G, int W>
 int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap, int32_t num_kv_heads,
                     cudaStream_t stream) {
-    static std::atomic<bool> done[64] = {};
+    static CtxDone done = {};
     constexpr size_t smem = pa::attend_smem_bytes<W>();
     int rc = prepare_kernel(pa::attend_partition_kernel<G, W>, smem, done);
     if (rc)
@@ -330,7 +374,7 @@ int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Atte
 template <int G>
 int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap,
                        int32_t num_kv_heads, cudaStream_t stream) {
-    static std::atomic<bool> done[64] = {};
+    static CtxDone done = {};
     int rc = prepare_kernel(pa::attend_tc_kernel<G>, pa::kAttendTcSmemBytes, done);
     if (rc)
         return rc;
@@ -368,7 +412,7 @@ int check_cache_fp8(const pa_cache_fp8_t *c) {
 template <int G, int CW>
 int launch_decode_fp8_cw(const CUtensorMap &tk, const CUtensorMap &tv, const pa::DecodeParams &p,
                          int32_t num_kv_heads, cudaStream_t stream) {
-    static std::atomic<bool> done[64] = {};
+    static CtxDone done = {};
     int rc = prepare_kernel(pa::decode_partition_fp8_kernel<G, CW>, pa::kDecodeSmemBytesF, done);
     if (rc)
         return rc;
@@ -945,14 +989,20 @@ int pa_get_device_error(int32_t *host_code, int clear) {
 // memory (see include/pa.h).  The array is a file-scope __device__ object: one
 // copy per device that loads the library, kept until the process exits.  In
 // host code its name only stands in for the object; the device address comes
-// from cudaGetSymbolAddress, looked up once per device (on the first call made
-// with that device current) and cached.
+// from cudaGetSymbolAddress, looked up on the first call made with a device
+// current and cached with the id of that device's context (looked up again
+// after a device reset).
 // ---------------------------------------------------------------------------
 static __device__ __align__(256) unsigned char g_decode_static_scratch[PA_DECODE_STATIC_WS_BYTES];
 
 namespace {
+// Per device: the array's device address and the context it was looked up in.
+struct StaticScratch {
+    void *ptr;
+    unsigned long long ctx;
+};
 std::mutex g_static_scratch_mu;
-void *g_static_scratch_ptr[64] = {};
+StaticScratch g_static_scratch[64] = {};
 }  // namespace
 
 int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int32_t *block_tables,
@@ -983,15 +1033,25 @@ int pa_decode_static_ws(const void *q, const pa_cache_t *cache, const int32_t *b
         return PA_EUNSUPPORTED;
     void *scratch = nullptr;
     {
+        // The address is looked up again whenever the current context is not
+        // the one it was found in: a device reset gives the device a new
+        // primary context, which loads this module afresh, possibly at other
+        // addresses.
         std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-        if (!g_static_scratch_ptr[dev]) {
-            e = cudaGetSymbolAddress(&g_static_scratch_ptr[dev], g_decode_static_scratch);
+        StaticScratch &c = g_static_scratch[dev];
+        const unsigned long long ctx = current_ctx_id();
+        if (!c.ptr || ctx == 0 || c.ctx != ctx) {
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_decode_static_scratch);
             if (e != cudaSuccess) {
-                g_static_scratch_ptr[dev] = nullptr;
+                c.ptr = nullptr;
+                c.ctx = 0;
                 return cuda_fail(e, "cudaGetSymbolAddress(static decode scratch)");
             }
+            c.ptr = p;
+            c.ctx = current_ctx_id();  // the lookup above made the device's context current
         }
-        scratch = g_static_scratch_ptr[dev];
+        scratch = c.ptr;
     }
     return pa_decode(q, cache, block_tables, max_blocks_per_seq, seq_lens, num_seqs, max_seq_len,
                      num_q_heads, scale, out, scratch, PA_DECODE_STATIC_WS_BYTES, stream);

@@ -61,8 +61,8 @@ def test_host_pool_step_timing_runs_the_step():
 
 def test_reference_arm_prints_one_contract_line():
     """`bench.py --impl reference` (the CPU oracle on a bounded sample of the
-    chat workload, one host thread) prints exactly one JSON line with the
-    contract's keys, its metric and unit matching the GPU arm's."""
+    chat workload, split over the host's cores) prints exactly one JSON line
+    with the contract's keys, its metric and unit matching the GPU arm's."""
     import json
     import subprocess
     import sys
@@ -79,7 +79,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["steps"] == 3 and d["warmup"] == 3 and d["n_gpus"] == 1 and d["higher_is_better"] is True
     assert d["value"] > 0 and d["vs_baseline"] is None and "workload" in d["config"]
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] == bench.host_cores() and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
@@ -99,6 +99,12 @@ def test_clock_samples_give_median_max_and_active_reasons():
     c = bench.ClockSampler.stop(s)
     assert c["sm_mhz"] == 1900 and c["sm_max_mhz"] == 1965 and c["samples"] == 3
     assert c["reasons"] == ["sw_power_cap"]
+    # rows only for other GPUs (a UUID format this sampler does not match):
+    # no clock is reported, and nothing of the other GPUs leaks in
+    s.uuid = "MIG-ccc"
+    c = bench.ClockSampler.stop(s)
+    assert c["sm_mhz"] is None and c["sm_max_mhz"] is None and c["samples"] == 0
+    assert c["reasons"] == ["uuid not matched"]
     s.proc = None
     assert bench.ClockSampler.stop(s)["reasons"] == ["nvidia-smi unavailable"]
 
@@ -111,3 +117,38 @@ def test_roofline_peak_reads_the_measured_file_else_falls_back(tmp_path, monkeyp
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6558.4, "bf16_tflops": 1590}))
     peak, how = bench.measured_peak()
     assert peak == 6558.4 and how.startswith("measured")
+
+
+def test_cpu_baseline_states_cores_and_keeps_the_one_thread_timing():
+    """The oracle fanned out over every host core (the reported value, its
+    thread count stated) and on one thread, on the same workload."""
+    cb = bench.cpu_baseline(synth.tiny(), 0.4)
+    assert cb["kind"] == "oracle" and cb["cores"] == cb["cores_available"] == bench.host_cores()
+    assert cb["value"] > 0 and cb["single_thread"]["cores"] == 1 and cb["single_thread"]["value"] > 0
+
+
+def test_split_oracle_layer_computes_every_pair_once(monkeypatch):
+    """The all-cores timing splits a layer's (sequence, head) pairs into
+    disjoint shares that together cover every pair exactly once."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    w = synth.tiny()
+    seen = []
+    monkeypatch.setattr(oracle, "decode", lambda *a: seen.append(np.asarray(a[-1]).copy()))
+    with ThreadPoolExecutor(max_workers=3) as pool:
+        bench._oracle_layer_threads(w, {"k_cache": None, "v_cache": None, "block_tables": None, "seq_lens": None},
+                                    pool, 3)
+    pairs = np.concatenate(seen)
+    assert len(seen) == 3
+    expect = {(s, j) for s in range(len(w.seq_ids)) for j in range(w.shape.num_q_heads)}
+    assert len(pairs) == len(expect) and {tuple(p) for p in pairs} == expect
+
+
+def test_extra_configs_default_to_the_long_context_decode():
+    args = bench.argparse.Namespace(extra_configs="auto", config="chat", queries=1, kv_dtype="bf16", part_tokens=0)
+    assert bench.extra_configs(args) == ["long"]
+    for change in ({"config": "long"}, {"queries": 4}, {"kv_dtype": "fp8"}, {"part_tokens": 640}):
+        assert bench.extra_configs(bench.argparse.Namespace(**{**vars(args), **change})) == []
+    assert bench.extra_configs(bench.argparse.Namespace(**{**vars(args), "extra_configs": "none"})) == []
+    assert bench.extra_configs(bench.argparse.Namespace(**{**vars(args), "extra_configs": "long,chat,sweep_b1"})) == [
+        "long", "sweep_b1"]

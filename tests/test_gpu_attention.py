@@ -2,7 +2,9 @@
 the oracle: within the decode tolerance on every output element, for
 speculative-decode-sized and prefill-chunk-sized queries, every group size
 and block size, split-K, requests without rows, and unused storage poisoned
-with NaN."""
+with NaN.  Every case runs on both attention kernels: the mma.sync kernel
+(8 (row, head) columns per warp) and the tcgen05 kernel (128 columns per CTA,
+S and O in tensor memory)."""
 import numpy as np
 import pytest
 
@@ -17,13 +19,15 @@ MAX_ABS, MEAN_ABS = 1.5e-2, 1e-3
 SCALE = float(np.float32(1 / np.sqrt(128)))
 
 
-@pytest.fixture(scope="module")
-def pa():
+@pytest.fixture(scope="module", params=["mma", "tcgen05"])
+def pa(request):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import paged_kv_cache_333_b200 as m
     m.pa_get_device_error(clear=True)
+    prev = m.pa_attention_set_kernel(request.param)
     yield m
+    m.pa_attention_set_kernel(prev)
     m.pa_decode_set_partition_tokens(0)
 
 
