@@ -275,14 +275,19 @@ PA_API int32_t pa_decode_set_kernel(int32_t kind);
 /* Which kernel pa_attention runs (process wide; returns the previous value;
  * other values are ignored).  pa_attention_workspace_bytes() follows the
  * setting, so query it after choosing.
- *   PA_ATTENTION_KERNEL_MMA     (default) warps of 8 (row, head) columns on
- *                               mma.m16n8k16, 16-token K/V tiles;
+ *   PA_ATTENTION_KERNEL_MMA     warps of 8 (row, head) columns on
+ *                               mma.m16n8k16, 16-token K/V tiles: for a few
+ *                               rows per request (speculative decoding);
  *   PA_ATTENTION_KERNEL_TCGEN05 128 columns per CTA on tcgen05.mma with the
  *                               S and O accumulators in tensor memory, 64-token
  *                               K/V tiles: for requests with many rows
- *                               (prefill chunks).  Not yet validated on a
- *                               GPU; the default stays the MMA kernel. */
-enum { PA_ATTENTION_KERNEL_MMA = 0, PA_ATTENTION_KERNEL_TCGEN05 = 1 };
+ *                               (prefill chunks);
+ *   PA_ATTENTION_KERNEL_AUTO    (default) per call: the tcgen05 kernel when
+ *                               max_query_len x (num_q_heads / num_kv_heads)
+ *                               is at least PA_ATTENTION_TCGEN05_MIN_COLUMNS,
+ *                               else the mma.sync kernel. */
+enum { PA_ATTENTION_KERNEL_MMA = 0, PA_ATTENTION_KERNEL_TCGEN05 = 1, PA_ATTENTION_KERNEL_AUTO = 2 };
+#define PA_ATTENTION_TCGEN05_MIN_COLUMNS 64
 PA_API int32_t pa_attention_set_kernel(int32_t kind);
 
 /* Tokens per split-K partition used by pa_decode: 0 = automatic (the

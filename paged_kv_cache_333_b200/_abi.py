@@ -30,7 +30,8 @@ EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "
             "pa_decode_set_kernel", "pa_attention_set_kernel", "pa_decode_set_partition_tokens", "pa_get_device_error",
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
-PA_ATTENTION_KERNEL_MMA, PA_ATTENTION_KERNEL_TCGEN05 = 0, 1
+PA_ATTENTION_KERNEL_MMA, PA_ATTENTION_KERNEL_TCGEN05, PA_ATTENTION_KERNEL_AUTO = 0, 1, 2
+PA_ATTENTION_TCGEN05_MIN_COLUMNS = 64  # include/pa.h
 
 
 class PaCache(ctypes.Structure):
@@ -410,11 +411,17 @@ def pa_decode_set_kernel(kind: str) -> str:
     return "mma" if prev == PA_DECODE_KERNEL_MMA else "simt"
 
 
+_ATTENTION_KERNELS = {"mma": PA_ATTENTION_KERNEL_MMA, "tcgen05": PA_ATTENTION_KERNEL_TCGEN05,
+                      "auto": PA_ATTENTION_KERNEL_AUTO}
+
+
 def pa_attention_set_kernel(kind: str) -> str:
-    """Select the pa_attention kernel: "mma" (default) or "tcgen05" (128
-    columns per CTA, accumulators in tensor memory); returns the previous one."""
-    prev = lib.pa_attention_set_kernel({"mma": PA_ATTENTION_KERNEL_MMA, "tcgen05": PA_ATTENTION_KERNEL_TCGEN05}[kind])
-    return "mma" if prev == PA_ATTENTION_KERNEL_MMA else "tcgen05"
+    """Select the pa_attention kernel: "auto" (default: "tcgen05" from
+    PA_ATTENTION_TCGEN05_MIN_COLUMNS (row, head) columns per request, else
+    "mma"), "mma" (8 columns per warp on mma.sync) or "tcgen05" (128 columns
+    per CTA, accumulators in tensor memory); returns the previous setting."""
+    prev = lib.pa_attention_set_kernel(_ATTENTION_KERNELS[kind])
+    return {v: k for k, v in _ATTENTION_KERNELS.items()}[prev]
 
 
 def pa_decode_set_partition_tokens(tokens: int) -> int:

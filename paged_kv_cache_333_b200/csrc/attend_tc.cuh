@@ -215,6 +215,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// max(a, b, c) in one instruction (the three-input form of max.f32, sm_100).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// Largest of 8 consecutive values.
+__device__ __forceinline__ float max8(const float *x) {
+    return fmax3f(fmax3f(x[0], x[1], x[2]), fmax3f(x[3], x[4], x[5]), fmaxf(x[6], x[7]));
+}
+
 // 16-byte cp.async that writes zeros when src_bytes is 0.
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
@@ -331,14 +342,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     if (warp < 4) {
         // Q rows of the chunk's columns into the swizzled K-major tile; zeros
         // for columns past the chunk (their scores are masked anyway).
+        // A negative scale is folded into q here (bf16 negation is exact), so
+        // that the softmax below multiplies the scores by |scale| > 0 and can
+        // take its maximum over the raw scores.
         const int c = col0 + threadIdx.x;
         const bool ok = c <= last_col;
+        const uint32_t sign = p.scale_log2 < 0.f ? 0x80008000u : 0u;
         const uint4 *qrow = p.q + ((static_cast<int64_t>(q0) + (ok ? c / G : 0)) * p.num_q_heads + h * G +
                                    (ok ? c % G : 0)) *
                                       (kD / 8);
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            const uint4 v = ok ? __ldg(qrow + k) : make_uint4(0u, 0u, 0u, 0u);
+            uint4 v = ok ? __ldg(qrow + k) : make_uint4(0u, 0u, 0u, 0u);
+            v.x ^= sign;
+            v.y ^= sign;
+            v.z ^= sign;
+            v.w ^= sign;
             *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(&sm.q[k >> 3][0]) + swz(threadIdx.x, k & 7)) = v;
         }
         fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
@@ -475,7 +494,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int lim = c <= last_col ? first_visible + c / G : -1;  // last position column c sees
         const bool warp_live = __any_sync(FULL, lim >= t_begin);
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const float sl2 = p.scale_log2;
+        const float sl2 = fabsf(p.scale_log2);  // q carries the scale's sign
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int t = 0; t < num_tiles; ++t) {
@@ -487,17 +506,32 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             const int t0 = t_begin + t * kTokTc;
             const int ntok = min(kTokTc, t_end - t0);
             const int jcount = max(0, min(ntok, lim - t0 + 1));  // tokens of this tile column c sees
+            // Raw scores of the tile, -inf for tokens column c does not see.
+            // Every tile but the causal diagonal and the range end is seen
+            // whole: no selects there.
             float x[kTokTc];
             if (warp_live) {
                 uint32_t s[32];
                 tmem_ld32(tmem + lane_base + (t & 1) * kTokTc, s);
+                if (jcount == kTokTc) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    x[j] = j < jcount ? __uint_as_float(s[j]) * sl2 : -INFINITY;
+                    for (int j = 0; j < 32; ++j)
+                        x[j] = __uint_as_float(s[j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        x[j] = j < jcount ? __uint_as_float(s[j]) : -INFINITY;
+                }
                 tmem_ld32(tmem + lane_base + (t & 1) * kTokTc + 32, s);
+                if (jcount == kTokTc) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    x[32 + j] = 32 + j < jcount ? __uint_as_float(s[j]) * sl2 : -INFINITY;
+                    for (int j = 0; j < 32; ++j)
+                        x[32 + j] = __uint_as_float(s[j]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        x[32 + j] = 32 + j < jcount ? __uint_as_float(s[j]) : -INFINITY;
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -511,10 +545,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     break;
             }
             if (warp_live) {
-                float mt = -INFINITY;
+                // the tile's max in the log2 domain: sl2 > 0, so it is sl2 x the raw max
+                float m8[8];
 #pragma unroll
-                for (int j = 0; j < kTokTc; ++j)
-                    mt = fmaxf(mt, x[j]);
+                for (int i = 0; i < 8; ++i)
+                    m8[i] = max8(&x[8 * i]);
+                const float mt = sl2 * fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                                              fmaxf(m8[6], m8[7]));
                 float alpha = 1.f;
                 bool rescale = false;
                 if (mt > m_ref + kLazyRescaleLog2) {  // false while the column has seen nothing
@@ -543,18 +580,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     }
                     tmem_st_wait();
                 }
-                // P row: 2^(x - m_ref), 0 where masked or while nothing is seen
-                const bool seen = m_ref != -INFINITY;
+                // P row: 2^(sl2 x - m_ref), one FMA and one exp2 per token; 0
+                // where masked (x = -inf).  While the column has seen nothing,
+                // every x is -inf and m_ref is too: the offset 0 keeps the
+                // FMA at -inf (not -inf + inf) and P at 0.
+                const float neg = m_ref != -INFINITY ? -m_ref : 0.f;
                 uint8_t *prow = reinterpret_cast<uint8_t *>(&sm.p[t & 1][0]);
                 float lsum = 0.f;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     float e[8];
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        e[u] = seen ? exp2_approx(x[8 * k + u] - m_ref) : 0.f;
-                        lsum += e[u];
-                    }
+                    for (int u = 0; u < 8; ++u)
+                        e[u] = exp2_approx(fmaf(x[8 * k + u], sl2, neg));
+                    lsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
                     uint4 w;
                     w.x = pack_bf16x2(e[0], e[1]);
                     w.y = pack_bf16x2(e[2], e[3]);

@@ -30,7 +30,7 @@ thread_local char g_last_cuda_error[256] = "";
 // thread and a call on another do not race.  A call reads each knob once.
 std::atomic<int32_t> g_part_tokens_override{0};
 std::atomic<int32_t> g_decode_kernel{PA_DECODE_KERNEL_MMA};
-std::atomic<int32_t> g_attention_kernel{PA_ATTENTION_KERNEL_MMA};
+std::atomic<int32_t> g_attention_kernel{PA_ATTENTION_KERNEL_AUTO};
 
 
 int cuda_fail(cudaError_t e, const char *what) {
@@ -147,8 +147,13 @@ struct WorkspaceLayout {
 };
 
 bool decode_kernel_is_mma() { return g_decode_kernel.load(std::memory_order_relaxed) == PA_DECODE_KERNEL_MMA; }
-bool attention_kernel_is_tcgen05() {
-    return g_attention_kernel.load(std::memory_order_relaxed) == PA_ATTENTION_KERNEL_TCGEN05;
+// The pa_attention kernel for a call with these columns per request
+// (max_query_len x group size): the knob, or under PA_ATTENTION_KERNEL_AUTO
+// the tcgen05 kernel from PA_ATTENTION_TCGEN05_MIN_COLUMNS columns on.
+bool attention_kernel_is_tcgen05(int64_t columns) {
+    const int32_t k = g_attention_kernel.load(std::memory_order_relaxed);
+    return k == PA_ATTENTION_KERNEL_TCGEN05 ||
+           (k == PA_ATTENTION_KERNEL_AUTO && columns >= PA_ATTENTION_TCGEN05_MIN_COLUMNS);
 }
 
 WorkspaceLayout workspace_layout(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
@@ -802,8 +807,9 @@ size_t pa_attention_workspace_bytes(int32_t num_reqs, int32_t num_tokens, int32_
     if (check_cache(cache) != PA_OK || num_reqs <= 0 || num_tokens <= 0 || max_query_len <= 0 ||
         num_q_heads <= 0 || max_seq_len < 0 || num_q_heads % cache->num_kv_heads != 0)
         return 0;
+    const int64_t columns = static_cast<int64_t>(max_query_len) * (num_q_heads / cache->num_kv_heads);
     return attend_layout(num_reqs, num_tokens, max_query_len, num_q_heads, cache->num_kv_heads, max_seq_len,
-                         cache->block_size, attention_kernel_is_tcgen05())
+                         cache->block_size, attention_kernel_is_tcgen05(columns))
         .total;
 }
 
@@ -831,7 +837,8 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     if (!std::isfinite(scale))
         return PA_EINVAL;
     const AttendLayout a = attend_layout(num_reqs, num_tokens, max_query_len, num_q_heads, cache->num_kv_heads,
-                                         max_seq_len, cache->block_size, attention_kernel_is_tcgen05());
+                                         max_seq_len, cache->block_size,
+                                         attention_kernel_is_tcgen05(static_cast<int64_t>(max_query_len) * G));
     if (static_cast<int64_t>(num_reqs) * a.chunks > 65535 || cache->num_kv_heads > 65535)
         return PA_EUNSUPPORTED;
     if (a.total > 0 && (workspace == nullptr || workspace_bytes < a.total))
@@ -900,7 +907,7 @@ int32_t pa_decode_set_kernel(int32_t kind) {
 }
 
 int32_t pa_attention_set_kernel(int32_t kind) {
-    if (kind == PA_ATTENTION_KERNEL_MMA || kind == PA_ATTENTION_KERNEL_TCGEN05)
+    if (kind == PA_ATTENTION_KERNEL_MMA || kind == PA_ATTENTION_KERNEL_TCGEN05 || kind == PA_ATTENTION_KERNEL_AUTO)
         return g_attention_kernel.exchange(kind);
     return g_attention_kernel.load();
 }

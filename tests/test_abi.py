@@ -74,7 +74,10 @@ def test_host_side_validation_of_the_widened_entry_points():
     assert attn(Hq=24) == PA_EUNSUPPORTED                 # group size 3
     assert attn(q=18) == PA_EUNSUPPORTED                  # q not 16-byte aligned
     assert attn(scale=float("nan")) == PA_EINVAL
-    assert attn(R=40000, T=40000, maxq=16) == PA_EUNSUPPORTED  # requests x column chunks > 65535
+    # requests x column chunks > 65535: 40000 x 2 chunks of 32 columns (48 per request) on the mma.sync kernel, and
+    # 70000 x 1 chunk of 128 on the tcgen05 one (which the automatic choice takes from 64 columns)
+    assert attn(R=40000, T=40000, maxq=12) == PA_EUNSUPPORTED
+    assert attn(R=70000, T=70000, maxq=16) == PA_EUNSUPPORTED
     assert attn(maxlen=32768) == PA_EWORKSPACE            # split-K needs scratch, none given
     assert lib.pa_attention_workspace_bytes(64, 256, 4, 32, 600, c) == 0
     assert lib.pa_attention_workspace_bytes(8, 32, 4, 32, 32768, c) > 0
@@ -223,8 +226,9 @@ def test_attention_kernel_knob_and_the_tensor_memory_chunking():
     per CTA instead of 32, which the workspace size shows through the split-K
     partition heuristic (fewer column chunks -> fewer units -> more, shorter
     partitions).  Only sizes are computed here: nothing is launched."""
-    from paged_kv_cache_333_b200._abi import (PA_ATTENTION_KERNEL_MMA, PA_ATTENTION_KERNEL_TCGEN05, PaCache,
-                                              lib)
+    from paged_kv_cache_333_b200._abi import (PA_ATTENTION_KERNEL_AUTO, PA_ATTENTION_KERNEL_MMA,
+                                              PA_ATTENTION_KERNEL_TCGEN05, PA_ATTENTION_TCGEN05_MIN_COLUMNS,
+                                              PaCache, lib)
     c = ctypes.byref(PaCache(16, 16, 26785, 16, 8, 128))
 
     def ws_bytes(rows, parts):
@@ -250,9 +254,16 @@ def test_attention_kernel_knob_and_the_tensor_memory_chunking():
         assert parts(R * 2) == 52 and parts(R * 8) == 19
         # chat lengths stay one partition either way: no scratch
         assert lib.pa_attention_workspace_bytes(64, 64 * 16, 16, 32, 612, c) == 0
+        # automatic choice: the tensor-memory kernel from the column threshold on
+        assert lib.pa_attention_set_kernel(PA_ATTENTION_KERNEL_AUTO) == PA_ATTENTION_KERNEL_TCGEN05
+        assert maxq * 4 >= PA_ATTENTION_TCGEN05_MIN_COLUMNS
+        assert lib.pa_attention_workspace_bytes(R, R * maxq, maxq, 32, L, c) == ws_bytes(R * maxq, parts(R * 2))
+        few = PA_ATTENTION_TCGEN05_MIN_COLUMNS // 4 - 1  # rows per request just below the threshold at G = 4
+        assert lib.pa_attention_workspace_bytes(R, R * few, few, 32, L, c) == ws_bytes(
+            R * few, parts(R * -(-(few * 4) // 32)))
     finally:
         lib.pa_attention_set_kernel(prev)
-    assert lib.pa_attention_set_kernel(prev) == prev == PA_ATTENTION_KERNEL_MMA
+    assert lib.pa_attention_set_kernel(prev) == prev == PA_ATTENTION_KERNEL_AUTO
 
 
 def test_binding_refuses_tensors_of_another_device(monkeypatch):

@@ -114,6 +114,22 @@ def test_attention_split_k(pa, part):
     assert pa.pa_get_device_error(clear=True) == 0
 
 
+@pytest.mark.parametrize("scale", [-SCALE, 2 * SCALE])
+def test_attention_negative_and_large_scale(pa, scale):
+    """Any finite scale is the caller's: a negative one flips which keys
+    dominate (the tcgen05 kernel folds its sign into q), a large one sharpens
+    the softmax; split into partitions so the merge sees the same domain."""
+    lens = [5, 70, 300, 1000]
+    q, kc, vc, bt, qsl, n = _case(83, lens, [5, 9, 40, 100], 16, 32, 8)
+    ref = oracle.attention(q, kc, vc, bt, qsl, n, scale)
+    prev = pa.pa_decode_set_partition_tokens(256)
+    try:
+        _check(_run(pa, q, kc, vc, bt, qsl, n, scale=scale), ref, f"scale={scale}")
+    finally:
+        pa.pa_decode_set_partition_tokens(prev)
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
 def test_attention_whole_prefill(pa):
     """q_len = n: the first rows see a handful of tokens, the last all."""
     lens = [1, 16, 31, 160]
