@@ -44,6 +44,8 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <type_traits>
+
 #include "decode_mma.cuh"
 
 namespace pa {
@@ -156,7 +158,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesF; ++i) {
             mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], 1);
+            mbar_init(&sm.empty[i], 32);  // every lane of the consuming warp releases the stage
         }
         mbar_init_fence();
     }
@@ -233,13 +235,24 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     // =================================================================== consumers
     const int g = lane >> 2;  // MMA group: S^T token row / B column (head)
     const int t4 = lane & 3;  // thread in group
+    // Packed columns (group sizes up to 4).  The MMAs' N = 8 columns hold 8
+    // heads; with G <= 4 half of them would be empty.  There column n < 4
+    // carries the hi part of head n and column n + 4 its lo part, for q
+    // (S^T) and for P (O^T alike): one MMA where two would run.  The lane of
+    // a hi column and the lane of its lo column (t4 and t4 ^ 2 in the C
+    // fragments) then hold the same two heads: their partial scores are
+    // summed by one shuffle, and the two halves of O are summed at the end.
+    constexpr bool kPack = G <= 4;
     // q as the B operand of S^T, split into e4m3 hi + lo after a per-head
-    // power-of-two scale.  Lane (g, t) holds head g, dims 32kk + 4t + i
-    // (register 0) and 32kk + 16 + 4t + i (register 1) of k-step kk.
+    // power-of-two scale.  Lane (g, t) holds head g (packed: head g % 4, hi
+    // part for g < 4, lo part above), dims 32kk + 4t + i (register 0) and
+    // 32kk + 16 + 4t + i (register 1) of k-step kk.
     uint32_t qh[4][2], ql[4][2];
-    float sl2A, sl2B;  // score scale (log2 domain) of heads 2t and 2t+1
+    float sl2A, sl2B;  // score scale (log2 domain) of the lane's two C-fragment heads
     {
-        const int qr = g < G ? g : G - 1;
+        const int qhead = kPack ? (g & 3) : g;
+        const bool qreal = qhead < G;
+        const int qr = qreal ? qhead : G - 1;
         const __nv_bfloat16 *qrow = reinterpret_cast<const __nv_bfloat16 *>(p.q) +
                                     (static_cast<int64_t>(s) * p.num_q_heads + h * G + qr) * kD;
         float qv[4][2][4];
@@ -249,10 +262,10 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const uint2 u = __ldg(reinterpret_cast<const uint2 *>(qrow + 32 * kk + 16 * r + 4 * t4));
-                qv[kk][r][0] = g < G ? bf16lo(u.x) : 0.f;
-                qv[kk][r][1] = g < G ? bf16hi(u.x) : 0.f;
-                qv[kk][r][2] = g < G ? bf16lo(u.y) : 0.f;
-                qv[kk][r][3] = g < G ? bf16hi(u.y) : 0.f;
+                qv[kk][r][0] = qreal ? bf16lo(u.x) : 0.f;
+                qv[kk][r][1] = qreal ? bf16hi(u.x) : 0.f;
+                qv[kk][r][2] = qreal ? bf16lo(u.y) : 0.f;
+                qv[kk][r][3] = qreal ? bf16hi(u.y) : 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
                     amax = fmaxf(amax, fabsf(qv[kk][r][i]));
@@ -277,11 +290,16 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                 for (int i = 0; i < 4; ++i)
                     x[i] = qv[kk][r][i] * up;
                 split_f32x4(x, qh[kk][r], ql[kk][r]);
+                if constexpr (kPack)
+                    qh[kk][r] = g < 4 ? qh[kk][r] : ql[kk][r];  // lo columns carry the lo part
             }
         }
         const float base = p.scale_log2 * p.k_scale;
-        const int shA = __shfl_sync(FULL, sh, 8 * t4);      // head 2t lives in group 2t
-        const int shB = __shfl_sync(FULL, sh, 8 * t4 + 4);  // head 2t+1 in group 2t+1
+        // the lane's C-fragment columns 2t, 2t+1 are heads 2hs, 2hs+1 (packed:
+        // column c is head c % 4), whose shifts live in groups 2hs and 2hs+1
+        const int hs = kPack ? (t4 & 1) : t4;
+        const int shA = __shfl_sync(FULL, sh, 8 * hs);
+        const int shB = __shfl_sync(FULL, sh, 8 * hs + 4);
         sl2A = base * __int_as_float((127 - shA) << 23);
         sl2B = base * __int_as_float((127 - shB) << 23);
     }
@@ -294,10 +312,14 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     const int mi = lane >> 3;  // which 8x8 matrix of an x4 load this lane addresses
     const int k_tok = (lane & 7) + ((mi & 1) << 3), k_chk = mi >> 1;
 
-    auto consume = [&](int slot, int ntok, auto &&loaded) {
+    // One tile.  kFull (compile time): all 32 tokens are in range, which is
+    // every tile but the last of a partition; the masked body is only
+    // instantiated for that last one.
+    auto consume = [&](auto full, int slot, int ntok, auto &&loaded) {
+        constexpr bool kFull = decltype(full)::value;
         const uint32_t kb = smem_addr(&sm.kv[slot][0][0]);
         const uint32_t vb = smem_addr(&sm.kv[slot][1][0]);
-        if (ntok < kTileF) {
+        if constexpr (!kFull) {
             uint4 *v = reinterpret_cast<uint4 *>(&sm.kv[slot][1][0]);
             for (int idx = ntok * 8 + lane; idx < kTileF * 8; idx += 32)
                 v[idx] = make_uint4(0, 0, 0, 0);
@@ -317,8 +339,17 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                 uint32_t kf[4];
                 ldmatrix_x4(kf, kb + swz(16 * mt + k_tok, 2 * kk + k_chk));
                 mma_16832_e4m3(shi[mt], kf, qh[kk][0], qh[kk][1]);
-                mma_16832_e4m3(slo[mt], kf, ql[kk][0], ql[kk][1]);
+                if constexpr (!kPack)
+                    mma_16832_e4m3(slo[mt], kf, ql[kk][0], ql[kk][1]);
             }
+        }
+        if constexpr (kPack) {
+            // the other part of the same heads' scores, from the lane two over
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    slo[mt][i] = __shfl_xor_sync(FULL, shi[mt][i], 2);
         }
         // V^T fragments, in two halves of four 16-dim tiles (fewer live
         // registers): matrix i of load c = tokens 8i..8i+7, dims 16c..16c+15.
@@ -336,7 +367,7 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
             x[mt][1] = (shi[mt][1] + slo[mt][1]) * sl2B;
             x[mt][2] = (shi[mt][2] + slo[mt][2]) * sl2A;
             x[mt][3] = (shi[mt][3] + slo[mt][3]) * sl2B;
-            if (ntok < kTileF) {
+            if constexpr (!kFull) {
                 if (16 * mt + g >= ntok) x[mt][0] = x[mt][1] = -INFINITY;
                 if (16 * mt + g + 8 >= ntok) x[mt][2] = x[mt][3] = -INFINITY;
             }
@@ -365,17 +396,35 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         lA = fmaf(lA, aA, (pr[0][0] + pr[0][2]) + (pr[1][0] + pr[1][2]));
         lB = fmaf(lB, aB, (pr[0][1] + pr[0][3]) + (pr[1][1] + pr[1][3]));
         // P^T as the B operand: movmatrix k gives head g, tokens 8k + 2t, 8k + 2t + 1
-        uint32_t ph[4], pl[4];
+        uint32_t ph[4];
+        [[maybe_unused]] uint32_t pl[4];  // unpacked path only
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                const uint32_t u = movmatrix_trans(pack_f16x2(pr[mt][2 * hf], pr[mt][2 * hf + 1]));
-                split_f16x2(u, ph[2 * mt + hf], pl[2 * mt + hf]);
+                if constexpr (kPack) {
+                    // lanes of lo columns (t >= 2) hand over the f16 residual
+                    // P - hi(P); after the transpose every lane encodes what it
+                    // holds: hi(P) in columns 0-3, lo(P) in columns 4-7, exactly
+                    // the split_f16x2 pair of the unpacked path
+                    const uint32_t v = pack_f16x2(pr[mt][2 * hf], pr[mt][2 * hf + 1]);
+                    const uint32_t back = e4m3x2_to_f16x2(f16x2_to_e4m3x2(v));
+                    const __half2 r = __hsub2(*reinterpret_cast<const __half2 *>(&v),
+                                              *reinterpret_cast<const __half2 *>(&back));
+                    const uint32_t w = t4 >= 2 ? *reinterpret_cast<const uint32_t *>(&r) : v;
+                    ph[2 * mt + hf] = f16x2_to_e4m3x2(movmatrix_trans(w));
+                } else {
+                    const uint32_t u = movmatrix_trans(pack_f16x2(pr[mt][2 * hf], pr[mt][2 * hf + 1]));
+                    split_f16x2(u, ph[2 * mt + hf], pl[2 * mt + hf]);
+                }
             }
         }
         const uint32_t pbh0 = __byte_perm(ph[0], ph[1], 0x5410), pbh1 = __byte_perm(ph[2], ph[3], 0x5410);
-        const uint32_t pbl0 = __byte_perm(pl[0], pl[1], 0x5410), pbl1 = __byte_perm(pl[2], pl[3], 0x5410);
+        [[maybe_unused]] uint32_t pbl0 = 0, pbl1 = 0;
+        if constexpr (!kPack) {
+            pbl0 = __byte_perm(pl[0], pl[1], 0x5410);
+            pbl1 = __byte_perm(pl[2], pl[3], 0x5410);
+        }
         // ---- O^T = alpha O^T + V^T P^T: d-tile c, A row g <-> dim 16c+2g, row
         // g+8 <-> 16c+2g+1.  The tile's product starts from zero and joins the
         // running sum in fp32 outside the MMA, so the sum over thousands of
@@ -397,7 +446,8 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                                        __byte_perm(vf[c4][2], vf[c4][3], 0x7531)};  // dim 2g+1, tokens +16
                 float o[4] = {0.f, 0.f, 0.f, 0.f};
                 mma_16832_e4m3(o, a, pbh0, pbh1);
-                mma_16832_e4m3(o, a, pbl0, pbl1);
+                if constexpr (!kPack)
+                    mma_16832_e4m3(o, a, pbl0, pbl1);
                 acc[c][0] = fmaf(acc[c][0], aA, o[0]);
                 acc[c][1] = fmaf(acc[c][1], aB, o[1]);
                 acc[c][2] = fmaf(acc[c][2], aA, o[2]);
@@ -408,21 +458,22 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
     auto tile_tokens = [&](int it) { return min(kTileF, t_end - (t_begin + it * kTileF)); };
 
     if (use_tma) {
+        // Every lane polls the stage's barrier (no divergent branch around a
+        // single waiter) and, once its own fragment loads are done, arrives
+        // on the stage's release barrier (count 32).
         for (int it = warp; it < num_tiles; it += kConsumerWarpsF) {
             const int slot = it % kStagesF;
-            bool ok = true;
-            if (lane == 0)
-                ok = mbar_wait(&sm.full[slot], (it / kStagesF) & 1);
-            if (!__shfl_sync(FULL, ok, 0))
+            if (!__all_sync(FULL, mbar_wait(&sm.full[slot], (it / kStagesF) & 1)))
                 break;
             const int ntok = tile_tokens(it);
-            consume(slot, ntok, [&] {
-                if (ntok < kTileF)
-                    fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0)
+            if (ntok == kTileF) {
+                consume(std::true_type{}, slot, ntok, [&] { mbar_arrive(&sm.empty[slot]); });
+            } else {
+                consume(std::false_type{}, slot, ntok, [&] {
+                    fence_proxy_async_smem();  // the V rows this warp zeroed, before the next async refill
                     mbar_arrive(&sm.empty[slot]);
-            });
+                });
+            }
         }
     } else {
         // Blocks of 1, 2 or 4 tokens: each consumer warp gathers its own tiles
@@ -456,7 +507,11 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
         for (int it = warp; it < num_tiles; it += kConsumerWarpsF) {
             asm volatile("cp.async.wait_group %0;" ::"n"(kAhead - 1) : "memory");
             __syncwarp();
-            consume(it % kStagesF, tile_tokens(it), [] {});
+            const int ntok = tile_tokens(it);
+            if (ntok == kTileF)
+                consume(std::true_type{}, it % kStagesF, ntok, [] {});
+            else
+                consume(std::false_type{}, it % kStagesF, ntok, [] {});
             __syncwarp();
             gather(it + kAhead * kConsumerWarpsF);
         }
@@ -516,8 +571,13 @@ decode_partition_fp8_kernel(const __grid_constant__ CUtensorMap tm_k,
                 L = fmaf(sm.wl[w][gq], sc, L);
 #pragma unroll
                 for (int u = 0; u < kPer; ++u)
-                    if (threadIdx.x + kStride * u < kD)
-                        o[u] = fmaf(wacc[(w * 8 + gq) * kD + threadIdx.x + kStride * u], sc, o[u]);
+                    if (threadIdx.x + kStride * u < kD) {
+                        const int d = threadIdx.x + kStride * u;
+                        float part = wacc[(w * 8 + gq) * kD + d];
+                        if constexpr (kPack)
+                            part += wacc[(w * 8 + gq + 4) * kD + d];  // the lo columns' share
+                        o[u] = fmaf(part, sc, o[u]);
+                    }
             }
         }
         const int jq = h * G + gq;
