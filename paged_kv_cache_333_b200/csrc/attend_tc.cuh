@@ -7,29 +7,41 @@
 // prefill, long speculative runs.
 //
 // Work decomposition.  A column is one (query row, query head of the KV group)
-// pair, c = i * G + g, as in attend.cuh.  One CTA handles one (split-K
-// partition, KV head, request, chunk of 128 columns) and streams the chunk's
-// token range in 64-token tiles:
+// pair, c = i * G + g, as in attend.cuh.  A work unit is one (split-K
+// partition, KV head, request, chunk of 128 columns); its token range is
+// streamed in 64-token tiles:
 //   S = Q K^T    M = 128 columns, N = 64 tokens, K = 128 dims: 8 MMAs of K = 16
 //   O += P V     M = 128 columns, N = 128 dims, K = 64 tokens: 4 MMAs of K = 16
 // (tcgen05.mma.cta_group::1.kind::f16, bf16 operands, fp32 accumulators in
-// tensor memory).  Q, K, P are K-major and V is MN-major, all in the 128-byte
-// swizzled layout the TMA loads write: rows of 128 bytes, 16-byte chunk j of
-// row r at position j ^ (r % 8), 8-row groups 1024 bytes apart.
+// tensor memory).  Q and K are K-major and V is MN-major in shared memory, in
+// the 128-byte swizzled layout the TMA loads write: rows of 128 bytes, 16-byte
+// chunk j of row r at position j ^ (r % 8), 8-row groups 1024 bytes apart.
+// P is the A operand of the P V product straight from tensor memory.
+//
+// Persistent grid.  One CTA per SM (shared memory) walks the units
+// blockIdx.x, blockIdx.x + gridDim.x, ...; every role derives the same unit
+// fields from global memory (loaded one unit ahead) and skips the same empty
+// units.  Tiles, S buffers and P buffers are counted across units, so the
+// producer streams the next unit's q tile and K/V tiles while the current
+// unit's softmax and epilogue finish; a CTA per unit left its SM without
+// loads in flight for about a third of its life (set-up, first load,
+// epilogue).
 //
 // Roles (192 threads):
-//   warps 0-3  softmax: thread t owns column t of the chunk, which is tensor-
+//   warps 0-3  softmax: thread t owns column t of the unit, which is tensor-
 //              memory lane t (a warp may only read lanes 32 * (warp % 4) ..
 //              + 31).  Per tile: read its S row (64 fp32), mask, online
 //              softmax with a lazily moved reference max, write its P row
-//              (bf16) to shared memory; at the end read its O row and write
-//              the output (or the split-K partials);
-//   warp 4     producer: 64-token K/V tiles into a 4-stage ring, by TMA for
-//              whole tiles of blocks >= 8 tokens, else by a cp.async gather
-//              that zero-fills the rows past the range;
+//              (bf16 pairs) to tensor memory; per unit: read its O row and
+//              write the output (or the split-K partials), then free O;
+//   warp 4     producer: per unit, the block-table slice into shared memory,
+//              the q tile by TMA (two buffers), and the 64-token K/V tiles
+//              into a 5-stage ring, by TMA for whole tiles of blocks >= 8
+//              tokens, else by a cp.async gather that zero-fills the rows past
+//              the range;
 //   warp 5     allocates tensor memory; one thread issues the MMAs.
-// Tensor memory: S double-buffered in columns [0, 64) and [64, 128), O in
-// [128, 256); 256 columns per CTA, one CTA per SM (shared memory).
+// Tensor memory (512 columns): S double-buffered in [0, 64) and [64, 128),
+// O in [128, 256), P double-buffered in [256, 288) and [288, 320).
 //
 // Lazy rescaling.  A column keeps a reference max m_ref (log2 domain) and
 // moves it only when a tile's max exceeds it by more than 8; the weights
@@ -39,13 +51,17 @@
 // completed.  (m_ref, l, O) is a consistent triple at any reference, which is
 // all the final division and the split-K merge need.
 //
-// Synchronisation (all mbarriers, every wait bounded):
-//   full[s]    producer -> MMA      stage s holds tile t (TMA bytes or cp.async)
-//   empty[s]   MMA commit -> producer  P V of tile t done: stage s reusable
-//   s_full[b]  MMA commit -> softmax   S of tile t in buffer b = t % 2
-//   s_free[b]  softmax (4 warps) -> MMA  S buffer b read
-//   p_full[b]  softmax (4 warps) -> MMA  P buffer b written, O rescaled
-//   pv_done[b] MMA commit -> softmax   P V of tile t done: P buffer b free, O current
+// Synchronisation (all mbarriers, every wait bounded; t counts tiles and k
+// units with work, both across the CTA's units):
+//   full[s]     producer -> MMA       stage s holds tile t (TMA bytes or cp.async)
+//   empty[s]    MMA commit -> producer  P V of tile t done: stage s reusable
+//   q_full[b]   producer (TMA) -> MMA  q tile of unit k in buffer b = k % 2
+//   q_empty[b]  MMA commit -> producer  unit k's last S read buffer b
+//   s_full[b]   MMA commit -> softmax  S of tile t in buffer b = t % 2
+//   s_free[b]   softmax (4 warps) -> MMA  S buffer b read
+//   p_full[b]   softmax (4 warps) -> MMA  P buffer b written, O rescaled
+//   pv_done[b]  MMA commit -> softmax  P V of tile t done: P buffer b free, O current
+//   o_free      softmax (4 warps) -> MMA  unit k's O read: the next unit may overwrite it
 // The MMA thread issues S(t + 1) before P V(t), so the tensor pipe computes
 // the next scores while the softmax warps work on the current tile.  No
 // waiter can fall two phases behind a barrier: each phase it waits for is
@@ -57,9 +73,10 @@
 namespace pa {
 
 constexpr int kTokTc = 64;      // tokens per tile
-constexpr int kStagesTc = 4;    // K/V ring depth
+constexpr int kStagesTc = 5;    // K/V ring depth
+constexpr int kMaxPartBlocksTc = 256;  // block-table entries one work unit may cover
 constexpr int kColsTc = 128;    // columns per CTA (= MMA M = tensor-memory lanes)
-constexpr int kTmemColsTc = 256;
+constexpr int kTmemColsTc = 512;  // S 2x64, O 128, P 2x32 (bf16 pairs)
 constexpr int kTcThreads = 192;
 constexpr int kTcSoftmaxThreads = 128;
 constexpr int kTcProducerWarp = 4;
@@ -181,6 +198,17 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D (tensor memory) = A B (+ D); A in tensor memory (K-major: lane = row m,
+// 32-bit column j = elements 2j, 2j+1 of the k-step), B in shared memory.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 // Arrive once on `bar` when every tcgen05.mma this thread issued so far is complete.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -240,73 +268,113 @@ __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
 
 struct AttendTcSmem {
     uint16_t kv[kStagesTc][4][kTokTc * 64];  // [stage][K lo, K hi, V lo, V hi][64 tokens x 64 dims], swizzled
-    uint16_t q[2][kColsTc * 64];             // [dims lo, dims hi][128 columns x 64 dims], swizzled
-    uint16_t p[2][kColsTc * kTokTc];         // [buffer][128 columns x 64 tokens], swizzled
+    uint16_t q[2][2][kColsTc * 64];          // [buffer][dims lo, dims hi][128 columns x 64 dims], swizzled
     uint64_t full[kStagesTc];
     uint64_t empty[kStagesTc];
     uint64_t s_full[2];
     uint64_t s_free[2];
     uint64_t p_full[2];
     uint64_t pv_done[2];
+    uint64_t q_full[2];
+    uint64_t q_empty[2];
+    uint64_t o_free;
     uint64_t mma_done;
     uint32_t tmem_base;
-    int32_t blocks[kMaxPartBlocksM];
+    int32_t blocks[kMaxPartBlocksTc];
 };
 constexpr size_t kAttendTcSmemBytes = sizeof(AttendTcSmem) + 1024;
 static_assert(kAttendTcSmemBytes <= 227 * 1024, "shared memory per CTA");
-static_assert(offsetof(AttendTcSmem, q) % 1024 == 0 && offsetof(AttendTcSmem, p) % 1024 == 0,
-              "swizzle atoms start on 1024-byte boundaries");
+static_assert(offsetof(AttendTcSmem, q) % 1024 == 0, "swizzle atoms start on 1024-byte boundaries");
 
+// One work unit: (split-K partition, KV head, request, 128-column chunk),
+// numbered as part + P * (head + Hkv * (request * chunks + chunk)).  Every
+// role derives the same fields from global memory, so all agree on which
+// units have work and on their tile counts.
+struct TcUnit {
+    int part, h, r, chunk;
+    int q0, n, col0, last_col, first_visible, t_begin, t_end, num_tiles;
+    bool bad;   // query_start_loc / seq_lens inconsistent for this request
+    bool work;  // at least one tile
+};
+
+// The unit's raw metadata, loaded one unit ahead so that its latency
+// overlaps the current unit's tiles; tc_unit() derives the rest.
+struct TcRaw {
+    int u, q0, q1, n;
+};
+__device__ __forceinline__ TcRaw tc_raw(const AttendParams &ap, int u) {
+    TcRaw raw{u, 0, 0, 0};
+    if (u < ap.num_units) {
+        const int r = (u / ap.d.num_parts / ap.num_kv_heads) / ap.chunks;
+        raw.q0 = ap.query_start_loc[r];
+        raw.q1 = ap.query_start_loc[r + 1];
+        raw.n = ap.d.seq_lens[r];
+    }
+    return raw;
+}
+
+template <int G>
+__device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &raw) {
+    const DecodeParams &p = ap.d;
+    TcUnit w{};
+    const int u = raw.u;
+    w.part = u % p.num_parts;
+    int rest = u / p.num_parts;
+    w.h = rest % ap.num_kv_heads;
+    rest /= ap.num_kv_heads;
+    w.r = rest / ap.chunks;
+    w.chunk = rest % ap.chunks;
+    int n = raw.n;  // clamped as clamp_seq_len does
+    {
+        const int64_t cap64 = static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size;
+        const int cap = static_cast<int>(cap64 < p.max_seq_len ? cap64 : p.max_seq_len);
+        if (n < 0 || n > cap) {
+            flag_error(PA_DEVERR_SEQ_LEN);
+            n = n < 0 ? 0 : cap;
+        }
+    }
+    const int q0 = raw.q0, q1 = raw.q1;
+    const int q_len = q1 - q0;
+    w.q0 = q0;
+    w.n = n;
+    w.bad = q_len < 0 || q_len > n || q_len > ap.max_query_len || q0 < 0 || q1 > ap.num_tokens ||
+            (w.r == 0 && q0 != 0) || (w.r == p.num_seqs - 1 && q1 != ap.num_tokens);
+    if (w.bad)
+        return w;
+    const int cols = q_len * G;
+    w.col0 = w.chunk * kColsTc;
+    if (w.col0 >= cols)
+        return w;
+    w.last_col = min(cols, w.col0 + kColsTc) - 1;
+    w.first_visible = n - q_len;  // row i sees positions <= first_visible + i
+    const int lim_max = w.first_visible + w.last_col / G;
+    w.t_begin = w.part * p.part_tokens;
+    if (w.t_begin > lim_max)
+        return w;
+    w.t_end = min(lim_max + 1, w.t_begin + p.part_tokens);
+    w.num_tiles = (w.t_end - w.t_begin + kTokTc - 1) / kTokTc;
+    w.work = true;
+    return w;
+}
+
+// Persistent: one CTA per SM walks the work units blockIdx.x, blockIdx.x +
+// gridDim.x, ...  Tiles, S buffers and P buffers are counted across units
+// (T), so the producer streams the next unit's q tile and K/V tiles while
+// the current unit's softmax and epilogue finish.
 template <int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const AttendParams ap) {
+                 const __grid_constant__ CUtensorMap tm_q, const AttendParams ap) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     constexpr unsigned FULL = 0xffffffffu;
     const DecodeParams &p = ap.d;
     extern __shared__ uint8_t smem_raw[];
     AttendTcSmem &sm = *reinterpret_cast<AttendTcSmem *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-
-    const int part = blockIdx.x;
-    const int h = blockIdx.y;
-    const int r = blockIdx.z / ap.chunks;
-    const int chunk = blockIdx.z % ap.chunks;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int B = p.block_size;
-    const int Hkv = gridDim.y;
-
-    if (warp == kTcProducerWarp && lane == 0 && B >= 8) {
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-    }
-    grid_dependency_wait();
-
-    // ---- the request's rows, this CTA's columns and token range -------------
-    // (every exit before the tensor-memory allocation below is CTA-uniform)
-    const int q0 = ap.query_start_loc[r];
-    const int q1 = ap.query_start_loc[r + 1];
-    const int n = clamp_seq_len(p, r);
-    const int q_len = q1 - q0;
-    if (q_len < 0 || q_len > n || q_len > ap.max_query_len || q0 < 0 || q1 > ap.num_tokens ||
-        (r == 0 && q0 != 0) || (r == p.num_seqs - 1 && q1 != ap.num_tokens)) {
-        if (part == 0 && h == 0 && chunk == 0 && threadIdx.x == 0)
-            flag_error(PA_DEVERR_QUERY_LOC);
-        return;
-    }
-    const int cols = q_len * G;
-    const int col0 = chunk * kColsTc;
-    if (col0 >= cols)
-        return;
-    const int last_col = min(cols, col0 + kColsTc) - 1;
-    const int first_visible = n - q_len;               // row i sees positions <= first_visible + i
-    const int lim_max = first_visible + last_col / G;  // >= 0
-    const int t_begin = part * p.part_tokens;
-    if (t_begin > lim_max)
-        return;
-    const int t_end = min(lim_max + 1, t_begin + p.part_tokens);
-    const int num_tiles = (t_end - t_begin + kTokTc - 1) / kTokTc;
+    const int Hkv = ap.num_kv_heads;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kStagesTc; ++i) {
@@ -318,49 +386,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_init(&sm.s_free[b], 4);
             mbar_init(&sm.p_full[b], 4);
             mbar_init(&sm.pv_done[b], 1);
+            mbar_init(&sm.q_full[b], 1);
+            mbar_init(&sm.q_empty[b], 1);
         }
+        mbar_init(&sm.o_free, 4);
         mbar_init(&sm.mma_done, 1);
         mbar_init_fence();
     }
-    if (p.num_parts > 1 && part == 0 && h == 0 && warp == 0) {
-        for (int i = col0 / G + lane; i <= last_col / G; i += 32)
-            ap.row_len[q0 + i] = first_visible + i + 1;
-    }
-    const int first_blk = t_begin / B;
-    if (warp == kTcProducerWarp) {
-        const int32_t *row = p.block_tables + static_cast<int64_t>(r) * p.max_blocks_per_seq + first_blk;
-        const int nblk = (t_end - 1) / B - first_blk + 1;
-        for (int i = lane; i < nblk; i += 32) {
-            int32_t b = __ldg(row + i);
-            if (b < 0 || b >= p.num_blocks) {
-                flag_error(PA_DEVERR_BLOCK_ID);
-                b = 0;
-            }
-            sm.blocks[i] = b;
+    if (warp == kTcProducerWarp && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        if (B >= 8) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
         }
-    }
-    if (warp < 4) {
-        // Q rows of the chunk's columns into the swizzled K-major tile; zeros
-        // for columns past the chunk (their scores are masked anyway).
-        // A negative scale is folded into q here (bf16 negation is exact), so
-        // that the softmax below multiplies the scores by |scale| > 0 and can
-        // take its maximum over the raw scores.
-        const int c = col0 + threadIdx.x;
-        const bool ok = c <= last_col;
-        const uint32_t sign = p.scale_log2 < 0.f ? 0x80008000u : 0u;
-        const uint4 *qrow = p.q + ((static_cast<int64_t>(q0) + (ok ? c / G : 0)) * p.num_q_heads + h * G +
-                                   (ok ? c % G : 0)) *
-                                      (kD / 8);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            uint4 v = ok ? __ldg(qrow + k) : make_uint4(0u, 0u, 0u, 0u);
-            v.x ^= sign;
-            v.y ^= sign;
-            v.z ^= sign;
-            v.w ^= sign;
-            *reinterpret_cast<uint4 *>(reinterpret_cast<uint8_t *>(&sm.q[k >> 3][0]) + swz(threadIdx.x, k & 7)) = v;
-        }
-        fence_proxy_async_smem();  // generic-proxy writes, read by the tensor cores
     }
     if (warp == kTcMmaWarp) {
         tmem_alloc(&sm.tmem_base, kTmemColsTc);
@@ -371,118 +409,188 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t tmem_o = tmem + 2 * kTokTc;
+    const uint32_t tmem_p = tmem + 2 * kTokTc + kD;  // two P buffers of 32 columns
+    grid_dependency_wait();
 
     if (warp == kTcProducerWarp) {
         // ============================================================ producer
         const uint64_t pol = l2_evict_first_policy();
-        int issued = 0;
+        int T = 0, k = 0;
         bool dead = false;
-        for (int it = 0; it < num_tiles && !dead; ++it) {
-            const int slot = it % kStagesTc;
-            if (it >= kStagesTc) {
+        TcRaw raw = tc_raw(ap, blockIdx.x);
+        for (int u = blockIdx.x; u < ap.num_units && !dead; u += gridDim.x) {
+            const TcUnit w = tc_unit<G>(ap, raw);
+            raw = tc_raw(ap, u + gridDim.x);
+            if (w.bad && w.part == 0 && w.h == 0 && w.chunk == 0 && lane == 0)
+                flag_error(PA_DEVERR_QUERY_LOC);
+            if (!w.work)
+                continue;
+            // the unit's slice of the block table (only this warp reads it)
+            const int first_blk = w.t_begin / B;
+            __syncwarp();
+            {
+                const int32_t *row = p.block_tables + static_cast<int64_t>(w.r) * p.max_blocks_per_seq + first_blk;
+                const int nblk = (w.t_end - 1) / B - first_blk + 1;
+                for (int i = lane; i < nblk; i += 32) {
+                    int32_t b = __ldg(row + i);
+                    if (b < 0 || b >= p.num_blocks) {
+                        flag_error(PA_DEVERR_BLOCK_ID);
+                        b = 0;
+                    }
+                    sm.blocks[i] = b;
+                }
+            }
+            __syncwarp();
+            // the unit's q tile: rows q0 + col0/G .., heads hG .. hG+G-1, both
+            // 64-dim halves; rows past the request hold other rows or zeros
+            // (their columns are masked)
+            const int qb = k & 1;
+            if (k >= 2) {
                 bool ok = true;
                 if (lane == 0)
-                    ok = mbar_wait(&sm.empty[slot], ((it / kStagesTc) + 1) & 1);
+                    ok = mbar_wait(&sm.q_empty[qb], ((k >> 1) - 1) & 1);
                 if (!__shfl_sync(FULL, ok, 0)) {
                     dead = true;
                     break;
                 }
             }
-            const int t0 = t_begin + it * kTokTc;
-            const int ntok = min(kTokTc, t_end - t0);
-            if (B >= 8 && ntok == kTokTc) {
-                // whole tile by TMA: boxes of min(B, 16) rows, 4 quarters each
-                const int rows = B < kTile ? B : kTile;
-                const int nbox = kTokTc / rows;  // 4 or 8
-                if (lane == 0)
-                    mbar_arrive_expect_tx(&sm.full[slot], static_cast<uint32_t>(kTokTc * 128 * 4));
-                __syncwarp();
-                const int j = lane >> 2, qd = lane & 3;  // box j of quarter qd (K lo, K hi, V lo, V hi)
-                if (j < nbox) {
-                    const int t = t0 + j * rows;
-                    const int32_t rr = sm.blocks[t / B - first_blk] * B + (t % B);
-                    tma_load_3d(&sm.kv[slot][qd][j * rows * 64], (qd < 2) ? &tm_k : &tm_v, (qd & 1) * 64, h, rr,
-                                &sm.full[slot], pol);
-                }
-            } else {
-                // gather: lane = (quarter, 16-byte chunk); rows past the range
-                // are zero-filled so that 0-weight V rows stay finite
-                const int qd = lane >> 3, ch = lane & 7;
-                const uint16_t *cache = static_cast<const uint16_t *>(qd < 2 ? p.k_cache : p.v_cache);
-                // cache rows of tokens lane and lane + 32, handed out by shuffle
-                int64_t row_lo = 0, row_hi = 0;
-                if (lane < ntok) {
-                    const int t = t0 + lane;
-                    row_lo = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + h;
-                }
-                if (lane + 32 < ntok) {
-                    const int t = t0 + lane + 32;
-                    row_hi = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + h;
-                }
-                const uint32_t base = smem_addr(&sm.kv[slot][qd][0]);
-                for (int i = 0; i < kTokTc; ++i) {
-                    const int64_t rr = __shfl_sync(FULL, i < 32 ? row_lo : row_hi, i & 31);
-                    const bool in = i < ntok;
-                    cp_async16_zfill(base + swz(i, ch), cache + (in ? rr * kD + (qd & 1) * 64 + ch * 8 : 0),
-                                     in ? 16u : 0u);
-                }
-                cp_async_mbar_arrive(&sm.full[slot]);
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&sm.full[slot]);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.q_full[qb], static_cast<uint32_t>(2 * kColsTc * 128));
+                tma_load_3d(&sm.q[qb][0][0], &tm_q, 0, w.h * G, w.q0 + w.col0 / G, &sm.q_full[qb], pol);
+                tma_load_3d(&sm.q[qb][1][0], &tm_q, 64, w.h * G, w.q0 + w.col0 / G, &sm.q_full[qb], pol);
             }
-            issued = it + 1;
+            for (int it = 0; it < w.num_tiles; ++it, ++T) {
+                const int slot = T % kStagesTc;
+                if (T >= kStagesTc) {
+                    bool ok = true;
+                    if (lane == 0)
+                        ok = mbar_wait(&sm.empty[slot], ((T / kStagesTc) + 1) & 1);
+                    if (!__shfl_sync(FULL, ok, 0)) {
+                        dead = true;
+                        break;
+                    }
+                }
+                const int t0 = w.t_begin + it * kTokTc;
+                const int ntok = min(kTokTc, w.t_end - t0);
+                if (B >= 8 && ntok == kTokTc) {
+                    // whole tile by TMA: boxes of min(B, 16) rows, 4 quarters each
+                    const int rows = B < kTile ? B : kTile;
+                    const int nbox = kTokTc / rows;  // 4 or 8
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(&sm.full[slot], static_cast<uint32_t>(kTokTc * 128 * 4));
+                    __syncwarp();
+                    const int j = lane >> 2, qd = lane & 3;  // box j of quarter qd (K lo, K hi, V lo, V hi)
+                    if (j < nbox) {
+                        const int t = t0 + j * rows;
+                        const int32_t rr = sm.blocks[t / B - first_blk] * B + (t % B);
+                        tma_load_3d(&sm.kv[slot][qd][j * rows * 64], (qd < 2) ? &tm_k : &tm_v, (qd & 1) * 64, w.h,
+                                    rr, &sm.full[slot], pol);
+                    }
+                } else {
+                    // gather: lane = (quarter, 16-byte chunk); rows past the range
+                    // are zero-filled so that 0-weight V rows stay finite
+                    const int qd = lane >> 3, ch = lane & 7;
+                    const uint16_t *cache = static_cast<const uint16_t *>(qd < 2 ? p.k_cache : p.v_cache);
+                    int64_t row_lo = 0, row_hi = 0;
+                    if (lane < ntok) {
+                        const int t = t0 + lane;
+                        row_lo = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + w.h;
+                    }
+                    if (lane + 32 < ntok) {
+                        const int t = t0 + lane + 32;
+                        row_hi = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + w.h;
+                    }
+                    const uint32_t base = smem_addr(&sm.kv[slot][qd][0]);
+                    for (int i = 0; i < kTokTc; ++i) {
+                        const int64_t rr = __shfl_sync(FULL, i < 32 ? row_lo : row_hi, i & 31);
+                        const bool in = i < ntok;
+                        cp_async16_zfill(base + swz(i, ch), cache + (in ? rr * kD + (qd & 1) * 64 + ch * 8 : 0),
+                                         in ? 16u : 0u);
+                    }
+                    cp_async_mbar_arrive(&sm.full[slot]);
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&sm.full[slot]);
+                }
+            }
+            ++k;
         }
         // nothing may still be copying into shared memory when the CTA ends
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0) {
-            for (int sl = 0; sl < kStagesTc && sl < issued; ++sl) {
-                const int last = sl + ((issued - 1 - sl) / kStagesTc) * kStagesTc;
+            for (int sl = 0; sl < kStagesTc && sl < T; ++sl) {
+                const int last = sl + ((T - 1 - sl) / kStagesTc) * kStagesTc;
                 mbar_wait(&sm.full[sl], (last / kStagesTc) & 1);
+            }
+            for (int b = 0; b < 2 && b < k; ++b) {
+                const int last = b + ((k - 1 - b) / 2) * 2;
+                mbar_wait(&sm.q_full[b], (last >> 1) & 1);
             }
         }
     } else if (warp == kTcMmaWarp) {
         // ============================================================ MMA issue
         if (lane == 0) {
-            const uint32_t q_base = smem_addr(&sm.q[0][0]);
-            auto pv = [&](int u) -> bool {
-                if (!mbar_wait(&sm.p_full[u & 1], (u >> 1) & 1))
+            // P V of tile pt (the first of its unit when first; unit index pk):
+            // O is overwritten by the first one, after the previous unit's
+            // epilogue has read it
+            auto pv = [&](int pt, bool first, int pk) -> bool {
+                if (!mbar_wait(&sm.p_full[pt & 1], (pt >> 1) & 1))
+                    return false;
+                if (first && pk >= 1 && !mbar_wait(&sm.o_free, (pk - 1) & 1))
                     return false;
                 tc_fence_after();
-                const uint32_t p_base = smem_addr(&sm.p[u & 1][0]);
-                const uint32_t v_base = smem_addr(&sm.kv[u % kStagesTc][2][0]);
+                const uint32_t v_base = smem_addr(&sm.kv[pt % kStagesTc][2][0]);
 #pragma unroll
                 for (int kk = 0; kk < kTokTc / 16; ++kk)
-                    umma_bf16_ss(tmem_o, umma_sdesc_sw128(p_base + p_step(kk), kLboK, kSbo),
+                    umma_bf16_ts(tmem_o, tmem_p + (pt & 1) * 32 + kk * 8,
                                  umma_sdesc_sw128(v_base + v_step(kk), kLboV, kSbo), kIdescPV,
-                                 (u > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&sm.pv_done[u & 1]);
-                umma_commit(&sm.empty[u % kStagesTc]);
+                                 (!first || kk > 0) ? 1u : 0u);
+                umma_commit(&sm.pv_done[pt & 1]);
+                umma_commit(&sm.empty[pt % kStagesTc]);
                 return true;
             };
             bool ok = true;
-            for (int t = 0; t < num_tiles && ok; ++t) {
-                const int slot = t % kStagesTc;
-                ok = mbar_wait(&sm.full[slot], (t / kStagesTc) & 1);
-                if (ok && t >= 2)
-                    ok = mbar_wait(&sm.s_free[t & 1], ((t >> 1) - 1) & 1);
-                if (!ok)
-                    break;
-                // a gathered stage was written by cp.async (generic proxy);
-                // the tensor cores read it through the async proxy
-                fence_proxy_async_smem();
-                tc_fence_after();
-                const uint32_t k_base = smem_addr(&sm.kv[slot][0][0]);
+            int T = 0, k = 0;
+            int prev_t = -1, prev_k = 0;
+            bool prev_first = false;
+            TcRaw raw = tc_raw(ap, blockIdx.x);
+            for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
+                const TcUnit w = tc_unit<G>(ap, raw);
+                raw = tc_raw(ap, u + gridDim.x);
+                if (!w.work)
+                    continue;
+                const int qb = k & 1;
+                ok = mbar_wait(&sm.q_full[qb], (k >> 1) & 1);
+                const uint32_t q_base = smem_addr(&sm.q[qb][0][0]);
+                for (int t = 0; t < w.num_tiles && ok; ++t, ++T) {
+                    const int slot = T % kStagesTc;
+                    ok = mbar_wait(&sm.full[slot], (T / kStagesTc) & 1);
+                    if (ok && T >= 2)
+                        ok = mbar_wait(&sm.s_free[T & 1], ((T >> 1) - 1) & 1);
+                    if (!ok)
+                        break;
+                    // a gathered stage was written by cp.async (generic proxy);
+                    // the tensor cores read it through the async proxy
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    const uint32_t k_base = smem_addr(&sm.kv[slot][0][0]);
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
-                    umma_bf16_ss(tmem + (t & 1) * kTokTc, umma_sdesc_sw128(q_base + q_step(kk), kLboK, kSbo),
-                                 umma_sdesc_sw128(k_base + k_step(kk), kLboK, kSbo), kIdescS, kk > 0 ? 1u : 0u);
-                umma_commit(&sm.s_full[t & 1]);
-                if (t >= 1)
-                    ok = pv(t - 1);
+                    for (int kk = 0; kk < kD / 16; ++kk)
+                        umma_bf16_ss(tmem + (T & 1) * kTokTc, umma_sdesc_sw128(q_base + q_step(kk), kLboK, kSbo),
+                                     umma_sdesc_sw128(k_base + k_step(kk), kLboK, kSbo), kIdescS, kk > 0 ? 1u : 0u);
+                    umma_commit(&sm.s_full[T & 1]);
+                    if (t == w.num_tiles - 1)
+                        umma_commit(&sm.q_empty[qb]);  // the unit's last S read of this q buffer
+                    if (prev_t >= 0)
+                        ok = pv(prev_t, prev_first, prev_k);
+                    prev_t = T;
+                    prev_first = t == 0;
+                    prev_k = k;
+                }
+                ++k;
             }
-            if (ok)
-                pv(num_tiles - 1);
+            if (ok && prev_t >= 0)
+                pv(prev_t, prev_first, prev_k);
             // everything issued above has completed before the allocation is freed
             umma_commit(&sm.mma_done);
             mbar_wait(&sm.mma_done, 0);
@@ -490,166 +598,201 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         __syncwarp();
     } else {
         // ============================================================ softmax
-        const int c = col0 + threadIdx.x;
-        const int lim = c <= last_col ? first_visible + c / G : -1;  // last position column c sees
-        const bool warp_live = __any_sync(FULL, lim >= t_begin);
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const float sl2 = fabsf(p.scale_log2);  // q carries the scale's sign
-        float m_ref = -INFINITY, l = 0.f;
+        // score multiplier (log2 domain) with the scale's sign; masked tokens
+        // are set to the value that the multiplier sends to -inf
+        const float sl2 = p.scale_log2;
+        const bool pos = sl2 >= 0.f;
+        const float masked = pos ? -INFINITY : INFINITY;
         bool ok = true;
-        for (int t = 0; t < num_tiles; ++t) {
-            if (lane == 0)
-                ok = mbar_wait(&sm.s_full[t & 1], (t >> 1) & 1);
-            if (!__shfl_sync(FULL, ok, 0))
-                break;
-            tc_fence_after();
-            const int t0 = t_begin + t * kTokTc;
-            const int ntok = min(kTokTc, t_end - t0);
-            const int jcount = max(0, min(ntok, lim - t0 + 1));  // tokens of this tile column c sees
-            // Raw scores of the tile, -inf for tokens column c does not see.
-            // Every tile but the causal diagonal and the range end is seen
-            // whole: no selects there.
-            float x[kTokTc];
-            if (warp_live) {
-                uint32_t s[32];
-                tmem_ld32(tmem + lane_base + (t & 1) * kTokTc, s);
-                if (jcount == kTokTc) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[j] = __uint_as_float(s[j]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[j] = j < jcount ? __uint_as_float(s[j]) : -INFINITY;
-                }
-                tmem_ld32(tmem + lane_base + (t & 1) * kTokTc + 32, s);
-                if (jcount == kTokTc) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[32 + j] = __uint_as_float(s[j]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        x[32 + j] = 32 + j < jcount ? __uint_as_float(s[j]) : -INFINITY;
-                }
+        int T = 0, k = 0;
+        TcRaw raw = tc_raw(ap, blockIdx.x);
+        for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
+            const TcUnit w = tc_unit<G>(ap, raw);
+            raw = tc_raw(ap, u + gridDim.x);
+            if (!w.work)
+                continue;
+            const int c = w.col0 + threadIdx.x;
+            const int lim = c <= w.last_col ? w.first_visible + c / G : -1;  // last position column c sees
+            const bool warp_live = __any_sync(FULL, lim >= w.t_begin);
+            if (p.num_parts > 1 && w.part == 0 && w.h == 0 && warp == 0) {
+                for (int i = w.col0 / G + lane; i <= w.last_col / G; i += 32)
+                    ap.row_len[w.q0 + i] = w.first_visible + i + 1;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.s_free[t & 1]);
-            // the P buffer of this tile was last read by P V of tile t - 2
-            if (t >= 2) {
+            float m_ref = -INFINITY, l = 0.f;
+            for (int t = 0; t < w.num_tiles; ++t, ++T) {
                 if (lane == 0)
-                    ok = mbar_wait(&sm.pv_done[t & 1], ((t >> 1) - 1) & 1);
+                    ok = mbar_wait(&sm.s_full[T & 1], (T >> 1) & 1);
                 if (!__shfl_sync(FULL, ok, 0))
                     break;
-            }
-            if (warp_live) {
-                // the tile's max in the log2 domain: sl2 > 0, so it is sl2 x the raw max
-                float m8[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    m8[i] = max8(&x[8 * i]);
-                const float mt = sl2 * fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
-                                              fmaxf(m8[6], m8[7]));
-                float alpha = 1.f;
-                bool rescale = false;
-                if (mt > m_ref + kLazyRescaleLog2) {  // false while the column has seen nothing
-                    if (m_ref != -INFINITY) {
-                        alpha = exp2_approx(m_ref - mt);
-                        rescale = true;
-                    }
-                    m_ref = mt;
-                }
-                l *= alpha;
-                if (__any_sync(FULL, rescale)) {
-                    // O must hold P V of tile t - 1 before it is scaled
-                    if (lane == 0)
-                        ok = mbar_wait(&sm.pv_done[(t - 1) & 1], ((t - 1) >> 1) & 1);
-                    if (!__shfl_sync(FULL, ok, 0))
-                        break;
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int cc = 0; cc < kD / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem_o + lane_base + cc * 32, o);
+                tc_fence_after();
+                const int t0 = w.t_begin + t * kTokTc;
+                const int ntok = min(kTokTc, w.t_end - t0);
+                const int jcount = max(0, min(ntok, lim - t0 + 1));  // tokens of this tile column c sees
+                // raw scores; tokens column c does not see get `masked`
+                float x[kTokTc];
+                if (warp_live) {
+                    uint32_t s[32];
+                    tmem_ld32(tmem + lane_base + (T & 1) * kTokTc, s);
+                    if (jcount == kTokTc) {
 #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                        tmem_st32(tmem_o + lane_base + cc * 32, o);
+                            x[j] = __uint_as_float(s[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            x[j] = j < jcount ? __uint_as_float(s[j]) : masked;
                     }
+                    tmem_ld32(tmem + lane_base + (T & 1) * kTokTc + 32, s);
+                    if (jcount == kTokTc) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            x[32 + j] = __uint_as_float(s[j]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            x[32 + j] = 32 + j < jcount ? __uint_as_float(s[j]) : masked;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.s_free[T & 1]);
+                // the P buffer of this tile was last read by P V of tile T - 2
+                if (T >= 2) {
+                    if (lane == 0)
+                        ok = mbar_wait(&sm.pv_done[T & 1], ((T >> 1) - 1) & 1);
+                    if (!__shfl_sync(FULL, ok, 0))
+                        break;
+                }
+                if (warp_live) {
+                    // the tile's max of sl2 * x in the log2 domain: the max of x
+                    // scaled, or with a negative scale the min of x
+                    float m8[8];
+                    float mt;
+                    if (pos) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            m8[i] = max8(&x[8 * i]);
+                        mt = sl2 * fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                                          fmaxf(m8[6], m8[7]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            float v = x[8 * i];
+#pragma unroll
+                            for (int j = 1; j < 8; ++j)
+                                v = fminf(v, x[8 * i + j]);
+                            m8[i] = v;
+                        }
+                        float v = m8[0];
+#pragma unroll
+                        for (int i = 1; i < 8; ++i)
+                            v = fminf(v, m8[i]);
+                        mt = sl2 * v;
+                    }
+                    float alpha = 1.f;
+                    bool rescale = false;
+                    if (mt > m_ref + kLazyRescaleLog2) {  // false while the column has seen nothing
+                        if (m_ref != -INFINITY) {
+                            alpha = exp2_approx(m_ref - mt);
+                            rescale = true;
+                        }
+                        m_ref = mt;
+                    }
+                    l *= alpha;
+                    if (__any_sync(FULL, rescale)) {
+                        // O must hold P V of tile T - 1 (of this unit: t >= 1) before it is scaled
+                        if (lane == 0)
+                            ok = mbar_wait(&sm.pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1);
+                        if (!__shfl_sync(FULL, ok, 0))
+                            break;
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int cc = 0; cc < kD / 32; ++cc) {
+                            uint32_t o[32];
+                            tmem_ld32(tmem_o + lane_base + cc * 32, o);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+                            tmem_st32(tmem_o + lane_base + cc * 32, o);
+                        }
+                        tmem_st_wait();
+                    }
+                    // P row: 2^(sl2 x - m_ref), one FMA and one exp2 per token;
+                    // 0 where masked.  While the column has seen nothing,
+                    // m_ref is -inf: the offset 0 keeps the FMA at -inf.
+                    const float neg = m_ref != -INFINITY ? -m_ref : 0.f;
+                    uint32_t pw[32];
+                    float lsum = 0.f;
+#pragma unroll
+                    for (int kq = 0; kq < 8; ++kq) {
+                        float e[8];
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            e[v] = exp2_approx(fmaf(x[8 * kq + v], sl2, neg));
+                        lsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+                        pw[4 * kq + 0] = pack_bf16x2(e[0], e[1]);
+                        pw[4 * kq + 1] = pack_bf16x2(e[2], e[3]);
+                        pw[4 * kq + 2] = pack_bf16x2(e[4], e[5]);
+                        pw[4 * kq + 3] = pack_bf16x2(e[6], e[7]);
+                    }
+                    tmem_st32(tmem_p + lane_base + (T & 1) * 32, pw);
                     tmem_st_wait();
+                    l += lsum;
                 }
-                // P row: 2^(sl2 x - m_ref), one FMA and one exp2 per token; 0
-                // where masked (x = -inf).  While the column has seen nothing,
-                // every x is -inf and m_ref is too: the offset 0 keeps the
-                // FMA at -inf (not -inf + inf) and P at 0.
-                const float neg = m_ref != -INFINITY ? -m_ref : 0.f;
-                uint8_t *prow = reinterpret_cast<uint8_t *>(&sm.p[t & 1][0]);
-                float lsum = 0.f;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sm.p_full[T & 1]);
+            }
+            // ---- epilogue: this column's O row, then O is free for the next unit
+            if (ok && lane == 0)
+                ok = mbar_wait(&sm.pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1);
+            ok = __shfl_sync(FULL, ok, 0);
+            if (ok && warp_live) {
+                tc_fence_after();
+                const bool valid = c <= w.last_col;
+                const int64_t qrow = valid ? w.q0 + c / G : 0;
+                const int j = w.h * G + c % G;
+#pragma unroll 1
+                for (int cc = 0; cc < kD / 32; ++cc) {
+                    uint32_t o[32];
+                    __syncwarp();  // the load is warp-collective
+                    tmem_ld32(tmem_o + lane_base + cc * 32, o);
+                    if (!valid) {
+                    } else if (p.num_parts == 1) {
+                        const float inv = l > 0.f ? 1.f / l : 0.f;
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qrow * p.num_q_heads + j) * kD + cc * 32);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    float e[8];
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                            v.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                            v.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                            v.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
+                            dst[q4] = v;
+                        }
+                    } else {
+                        const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + w.part;
+                        float4 *dst = reinterpret_cast<float4 *>(p.part_acc + idx * kD + cc * 32);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        e[u] = exp2_approx(fmaf(x[8 * k + u], sl2, neg));
-                    lsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-                    uint4 w;
-                    w.x = pack_bf16x2(e[0], e[1]);
-                    w.y = pack_bf16x2(e[2], e[3]);
-                    w.z = pack_bf16x2(e[4], e[5]);
-                    w.w = pack_bf16x2(e[6], e[7]);
-                    *reinterpret_cast<uint4 *>(prow + swz(threadIdx.x, k)) = w;
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
+                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+                        if (cc == 0)
+                            p.part_ml[idx] = make_float2(m_ref, l);
+                    }
                 }
-                l += lsum;
-                fence_proxy_async_smem();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&sm.p_full[t & 1]);
+                mbar_arrive(&sm.o_free);
+            ++k;
         }
         if (threadIdx.x == 0)
             grid_launch_dependents();
-        // ---- epilogue: this column's O row -----------------------------------
-        if (ok && lane == 0)
-            ok = mbar_wait(&sm.pv_done[(num_tiles - 1) & 1], ((num_tiles - 1) >> 1) & 1);
-        ok = __shfl_sync(FULL, ok, 0);
-        if (ok && warp_live) {
-            tc_fence_after();
-            const bool valid = c <= last_col;
-            const int64_t qrow = valid ? q0 + c / G : 0;
-            const int j = h * G + c % G;
-#pragma unroll 1
-            for (int cc = 0; cc < kD / 32; ++cc) {
-                uint32_t o[32];
-                __syncwarp();  // the load is warp-collective
-                tmem_ld32(tmem_o + lane_base + cc * 32, o);
-                if (!valid) {
-                } else if (p.num_parts == 1) {
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qrow * p.num_q_heads + j) * kD + cc * 32);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-                        dst[k] = w;
-                    }
-                } else {
-                    const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + part;
-                    float4 *dst = reinterpret_cast<float4 *>(p.part_acc + idx * kD + cc * 32);
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                                             __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
-                    if (cc == 0)
-                        p.part_ml[idx] = make_float2(m_ref, l);
-                }
-            }
-        }
     }
     // every role is done with tensor memory before it is freed
     tc_fence_before();

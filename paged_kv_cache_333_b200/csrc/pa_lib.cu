@@ -334,6 +334,8 @@ AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_que
     a.chunks = static_cast<int32_t>(std::max<int64_t>(1, (cols + per_cta - 1) / per_cta));
     const int64_t units = std::min<int64_t>(INT32_MAX, static_cast<int64_t>(num_reqs) * a.chunks);
     a.part_tokens = choose_part_tokens(static_cast<int32_t>(units), num_kv_heads, max_seq_len, block_size, true);
+    if (tcgen05)  // its table holds fewer entries
+        a.part_tokens = std::min<int32_t>(a.part_tokens, pa::kMaxPartBlocksTc * block_size / 64 * 64);
     a.num_parts = max_seq_len > 0 ? (max_seq_len + a.part_tokens - 1) / a.part_tokens : 1;
     if (a.num_parts <= 1) {
         a.num_parts = 1;
@@ -376,16 +378,52 @@ int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Atte
 }
 
 // The tensor-memory variant (attend_tc.cuh): 128 columns per CTA, one CTA per SM.
+// The q rows as a 3-D tensor (dim, head, row) for the tcgen05 kernel's TMA
+// loads of its q tiles: boxes of (64 dims, G heads, 128 / G rows), the
+// 128-byte swizzle, rows past num_tokens read as zeros.
+int encode_q_map(CUtensorMap *tm, const void *q, int32_t num_tokens, int32_t num_q_heads, int32_t G) {
+    auto fn = encode_fn();
+    if (!fn) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled unavailable");
+        return PA_ECUDA;
+    }
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(pa::kD), static_cast<cuuint64_t>(num_q_heads),
+                                static_cast<cuuint64_t>(num_tokens)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pa::kD) * 2,
+                                   static_cast<cuuint64_t>(num_q_heads) * pa::kD * 2};
+    const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(pa::kColsTc / G)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        std::snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "cuTensorMapEncodeTiled (q) failed (%d)",
+                      static_cast<int>(r));
+        return PA_ECUDA;
+    }
+    return PA_OK;
+}
+
+// The tensor-memory variant (attend_tc.cuh): 128 columns per work unit, a
+// persistent grid of one CTA per SM walking the units.
 template <int G>
-int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::AttendParams &ap,
+int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const void *q, pa::AttendParams ap,
                        int32_t num_kv_heads, cudaStream_t stream) {
     static CtxDone done = {};
     int rc = prepare_kernel(pa::attend_tc_kernel<G>, pa::kAttendTcSmemBytes, done);
     if (rc)
         return rc;
-    const dim3 grid(ap.d.num_parts, num_kv_heads, ap.d.num_seqs * ap.chunks);
+    CUtensorMap tq;
+    if ((rc = encode_q_map(&tq, q, ap.num_tokens, ap.d.num_q_heads, G)) != PA_OK)
+        return rc;
+    const int64_t units = static_cast<int64_t>(ap.d.num_parts) * num_kv_heads * ap.d.num_seqs * ap.chunks;
+    if (units > INT32_MAX)
+        return PA_EUNSUPPORTED;
+    ap.num_kv_heads = num_kv_heads;
+    ap.num_units = static_cast<int32_t>(units);
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, sm_count())));
     cudaError_t e = launch_pdl(pa::attend_tc_kernel<G>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
-                               stream, tk, tv, ap);
+                               stream, tk, tv, tq, ap);
     if (e != cudaSuccess)
         return cuda_fail(e, "attend_tc_kernel launch");
     return launch_row_merge(ap, stream);
@@ -881,10 +919,10 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (a.tcgen05) {
         switch (G) {
-        case 1: return launch_attend_tc_g<1>(tk, tv, ap, cache->num_kv_heads, st);
-        case 2: return launch_attend_tc_g<2>(tk, tv, ap, cache->num_kv_heads, st);
-        case 4: return launch_attend_tc_g<4>(tk, tv, ap, cache->num_kv_heads, st);
-        default: return launch_attend_tc_g<8>(tk, tv, ap, cache->num_kv_heads, st);
+        case 1: return launch_attend_tc_g<1>(tk, tv, q, ap, cache->num_kv_heads, st);
+        case 2: return launch_attend_tc_g<2>(tk, tv, q, ap, cache->num_kv_heads, st);
+        case 4: return launch_attend_tc_g<4>(tk, tv, q, ap, cache->num_kv_heads, st);
+        default: return launch_attend_tc_g<8>(tk, tv, q, ap, cache->num_kv_heads, st);
         }
     }
     const bool w2 = a.warps == 2;
