@@ -184,13 +184,14 @@ class ClockSampler:
 
 # --------------------------------------------------------------------------- ncu traffic
 PROFILE_FOR = {"bf16": "decode_mma_chat_full.md", "fp8": "decode_fp8_chat_full.md",
-               "rows4": "attention_q4_chat_full.md"}
+               "rows4": "attention_q4_chat_full.md", "rows16_tcgen05": "attention_tc_q16_chat_full.md"}
 
 
 def profiled_traffic(config: str, kind: str = "bf16"):
     """DRAM bytes (read + write) per launch of the timed kernel from the
     committed ncu capture of that kernel (kind: "bf16" decode, "fp8" decode,
-    "rows4" = pa_attention with 4 rows per sequence), if that capture was of
+    "rows4" = pa_attention with 4 rows per sequence on the mma.sync kernel,
+    "rows16_tcgen05" = 16 rows on the tcgen05 kernel), if that capture was of
     this workload and of the kernel sources as they are now; otherwise None."""
     import hashlib
     if kind not in PROFILE_FOR:
@@ -347,6 +348,10 @@ def run_ours(args, world, rank, local):
         inp["out"] = torch.empty_like(inp["q"])
         need = pa.pa_attention_workspace_bytes(S, S * Q, Q, st.num_q_heads, st.max_seq_len, *st.caches[0])
         inp["ws"] = torch.empty(need, dtype=torch.uint8, device=dev) if need else None
+    # which pa_attention kernel runs (the library's automatic choice unless forced)
+    group = st.num_q_heads // st.num_kv_heads
+    attention_tc = Q > 1 and (args.attention_kernel == "tcgen05" or (
+        args.attention_kernel == "default" and Q * group >= pa._abi.PA_ATTENTION_TCGEN05_MIN_COLUMNS))
     nbytes = algorithmic_bytes(st, rows_per_seq=Q)
     step_bytes = L * (nbytes["decode_kv"] + nbytes["write"] + nbytes["copy"])
     stream = torch.cuda.current_stream(dev)
@@ -547,7 +552,7 @@ def run_ours(args, world, rank, local):
                         + (f"; {Q} query rows per sequence (its last {Q} tokens, causal), pa_attention" if Q > 1
                            else ""),
             "query_rows_per_seq": Q,
-            "attention_kernel": args.attention_kernel if Q > 1 else None,
+            "attention_kernel": ("tcgen05" if attention_tc else "mma") if Q > 1 else None,
             "layers_per_step": L,
             "batch": S,
             "block_size": st.block_size,
@@ -570,7 +575,8 @@ def run_ours(args, world, rank, local):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": None if args.part_tokens else profiled_traffic(
-                         args.config, "fp8" if fp8 else "bf16" if Q == 1 else f"rows{Q}"),
+                         args.config, "fp8" if fp8 else "bf16" if Q == 1 else
+                         f"rows{Q}" + ("_tcgen05" if attention_tc else "")),
                      "kernel": ("pa_attention" if Q > 1 else "pa_decode_fp8" if fp8 else "pa_decode")
                                + " (partition kernel"
                                + (" + LSE merge)" if split else ")"),

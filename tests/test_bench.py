@@ -36,7 +36,7 @@ def test_algorithmic_bytes_count_shared_blocks_once():
 
 
 def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
-    for kind in ("bf16", "fp8", "rows4"):
+    for kind in ("bf16", "fp8", "rows4", "rows16_tcgen05"):
         t = bench.profiled_traffic("chat", kind)
         assert isinstance(t, int) and t > 0, kind
     assert bench.profiled_traffic("long", "bf16") is None  # captured on chat only
