@@ -361,7 +361,10 @@ __device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &r
 // gridDim.x, ...  Tiles, S buffers and P buffers are counted across units
 // (T), so the producer streams the next unit's q tile and K/V tiles while
 // the current unit's softmax and epilogue finish.
-template <int G>
+//
+// kZeroScale: the caller's scale is 0, so every visible token weighs 1 and a
+// masked one 0; the scaled-score form below would give 0 * inf there.
+template <int G, bool kZeroScale>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_q, const AttendParams ap) {
@@ -670,7 +673,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     // scaled, or with a negative scale the min of x
                     float m8[8];
                     float mt;
-                    if (pos) {
+                    if (kZeroScale) {
+                        mt = jcount > 0 ? 0.f : -INFINITY;
+                    } else if (pos) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             m8[i] = max8(&x[8 * i]);
@@ -730,7 +735,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         float e[8];
 #pragma unroll
                         for (int v = 0; v < 8; ++v)
-                            e[v] = exp2_approx(fmaf(x[8 * kq + v], sl2, neg));
+                            e[v] = kZeroScale ? (8 * kq + v < jcount ? 1.f : 0.f)
+                                              : exp2_approx(fmaf(x[8 * kq + v], sl2, neg));
                         lsum += ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
                         pw[4 * kq + 0] = pack_bf16x2(e[0], e[1]);
                         pw[4 * kq + 1] = pack_bf16x2(e[2], e[3]);

@@ -406,11 +406,11 @@ int encode_q_map(CUtensorMap *tm, const void *q, int32_t num_tokens, int32_t num
 
 // The tensor-memory variant (attend_tc.cuh): 128 columns per work unit, a
 // persistent grid of one CTA per SM walking the units.
-template <int G>
+template <int G, bool kZeroScale>
 int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const void *q, pa::AttendParams ap,
                        int32_t num_kv_heads, cudaStream_t stream) {
     static CtxDone done = {};
-    int rc = prepare_kernel(pa::attend_tc_kernel<G>, pa::kAttendTcSmemBytes, done);
+    int rc = prepare_kernel(pa::attend_tc_kernel<G, kZeroScale>, pa::kAttendTcSmemBytes, done);
     if (rc)
         return rc;
     CUtensorMap tq;
@@ -422,7 +422,7 @@ int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const void 
     ap.num_kv_heads = num_kv_heads;
     ap.num_units = static_cast<int32_t>(units);
     const dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, sm_count())));
-    cudaError_t e = launch_pdl(pa::attend_tc_kernel<G>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
+    cudaError_t e = launch_pdl(pa::attend_tc_kernel<G, kZeroScale>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
                                stream, tk, tv, tq, ap);
     if (e != cudaSuccess)
         return cuda_fail(e, "attend_tc_kernel launch");
@@ -918,11 +918,20 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     ap.chunks = a.chunks;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (a.tcgen05) {
+        const int nk = cache->num_kv_heads;
+        if (scale == 0.f) {
+            switch (G) {
+            case 1: return launch_attend_tc_g<1, true>(tk, tv, q, ap, nk, st);
+            case 2: return launch_attend_tc_g<2, true>(tk, tv, q, ap, nk, st);
+            case 4: return launch_attend_tc_g<4, true>(tk, tv, q, ap, nk, st);
+            default: return launch_attend_tc_g<8, true>(tk, tv, q, ap, nk, st);
+            }
+        }
         switch (G) {
-        case 1: return launch_attend_tc_g<1>(tk, tv, q, ap, cache->num_kv_heads, st);
-        case 2: return launch_attend_tc_g<2>(tk, tv, q, ap, cache->num_kv_heads, st);
-        case 4: return launch_attend_tc_g<4>(tk, tv, q, ap, cache->num_kv_heads, st);
-        default: return launch_attend_tc_g<8>(tk, tv, q, ap, cache->num_kv_heads, st);
+        case 1: return launch_attend_tc_g<1, false>(tk, tv, q, ap, nk, st);
+        case 2: return launch_attend_tc_g<2, false>(tk, tv, q, ap, nk, st);
+        case 4: return launch_attend_tc_g<4, false>(tk, tv, q, ap, nk, st);
+        default: return launch_attend_tc_g<8, false>(tk, tv, q, ap, nk, st);
         }
     }
     const bool w2 = a.warps == 2;

@@ -3,8 +3,8 @@ the oracle: within the decode tolerance on every output element, for
 speculative-decode-sized and prefill-chunk-sized queries, every group size
 and block size, split-K, requests without rows, and unused storage poisoned
 with NaN.  Every case runs on both attention kernels: the mma.sync kernel
-(8 (row, head) columns per warp) and the tcgen05 kernel (128 columns per CTA,
-S and O in tensor memory)."""
+(8 (row, head) columns per warp) and the tcgen05 kernel (128 columns per work
+unit, S, P and O in tensor memory)."""
 import numpy as np
 import pytest
 
@@ -114,17 +114,40 @@ def test_attention_split_k(pa, part):
     assert pa.pa_get_device_error(clear=True) == 0
 
 
-@pytest.mark.parametrize("scale", [-SCALE, 2 * SCALE])
+@pytest.mark.parametrize("scale", [-SCALE, 2 * SCALE, 0.0])
 def test_attention_negative_and_large_scale(pa, scale):
     """Any finite scale is the caller's: a negative one flips which keys
-    dominate (the tcgen05 kernel folds its sign into q), a large one sharpens
-    the softmax; split into partitions so the merge sees the same domain."""
+    dominate (the tcgen05 kernel takes the tile minimum of the raw scores), a
+    large one sharpens the softmax, zero makes it the mean of the visible V
+    rows (masked tokens still weigh 0); split into partitions so the merge
+    sees the same domain."""
     lens = [5, 70, 300, 1000]
     q, kc, vc, bt, qsl, n = _case(83, lens, [5, 9, 40, 100], 16, 32, 8)
     ref = oracle.attention(q, kc, vc, bt, qsl, n, scale)
     prev = pa.pa_decode_set_partition_tokens(256)
     try:
         _check(_run(pa, q, kc, vc, bt, qsl, n, scale=scale), ref, f"scale={scale}")
+    finally:
+        pa.pa_decode_set_partition_tokens(prev)
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("scale", [SCALE, -SCALE, 0.0])
+@pytest.mark.parametrize("part", [0, 128])
+def test_attention_up_to_64_columns(pa, G, scale, part):
+    """At most 64 (row, head) columns per request (the bench's many-row case
+    has 64): requests of one tile and of many, whole or split into 128-token
+    partitions (work units of one or two tiles back to back), positive,
+    negative and zero scale."""
+    rmax = 64 // G
+    lens = [1, 3, 64, 65, 100, 129, 700, 5, 2000, 64, 20, 190]
+    q_lens = [min(n, r) for n, r in zip(lens, [1, 3, rmax, rmax, rmax - 1, rmax, rmax, 5, rmax // 2, 0, rmax, 2])]
+    q, kc, vc, bt, qsl, n = _case(900 + 10 * G + part, lens, q_lens, 16, 2 * G, 2)
+    ref = oracle.attention(q, kc, vc, bt, qsl, n, scale)
+    prev = pa.pa_decode_set_partition_tokens(part)
+    try:
+        _check(_run(pa, q, kc, vc, bt, qsl, n, scale=scale), ref, f"G={G} scale={scale} part={part}")
     finally:
         pa.pa_decode_set_partition_tokens(prev)
     assert pa.pa_get_device_error(clear=True) == 0
@@ -164,6 +187,21 @@ def test_attention_spec_decode_full_size(pa):
     ref = oracle.attention(q, kc, vc, bt, qsl, n, SCALE)
     _check(got, ref, "spec decode 64 x 4")
     assert pa.pa_get_device_error(clear=True) == 0
+
+
+def test_attention_chunk16_full_size(pa):
+    """Chat-sized batch (64 requests, 512..612 tokens, Llama-3-8B heads) with
+    16 query rows each: 64 columns per request, the bench's many-row case.
+    Eight requests are checked against the oracle row by row."""
+    gen = synth.make_rng(84)
+    lens = gen.integers(512, 613, size=64).tolist()
+    q, kc, vc, bt, qsl, n = _case(85, lens, [16] * 64, 16, 32, 8)
+    got = _run(pa, q, kc, vc, bt, qsl, n)
+    assert pa.pa_get_device_error(clear=True) == 0
+    for r in gen.choice(64, size=8, replace=False).tolist():
+        rows = slice(int(qsl[r]), int(qsl[r + 1]))
+        ref = oracle.attention(q[rows], kc, vc, bt[r:r + 1], np.array([0, 16], np.int32), n[r:r + 1], SCALE)
+        _check(got[rows], ref, f"request {r}")
 
 
 def test_attention_rejects_bad_query_start_loc(pa):
