@@ -183,39 +183,43 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- ncu traffic
-PROFILE_FOR = {"bf16": "decode_mma_chat_full.md", "fp8": "decode_fp8_chat_full.md",
-               "rows4": "attention_q4_chat_full.md", "rows16_tcgen05": "attention_tc_q16_chat_full.md"}
+PROFILE_FOR = {"bf16": ("decode_mma_chat_full.md",),
+               "fp8": ("decode_fp8_chat_full.md", "decode_fp8_sweep_b1_full.md"),
+               "rows4": ("attention_q4_chat_full.md",), "rows16_tcgen05": ("attention_tc_q16_chat_full.md",)}
 
 
 def profiled_traffic(config: str, kind: str = "bf16"):
     """DRAM bytes (read + write) per launch of the timed kernel from the
     committed ncu capture of that kernel (kind: "bf16" decode, "fp8" decode,
     "rows4" = pa_attention with 4 rows per sequence on the mma.sync kernel,
-    "rows16_tcgen05" = 16 rows on the tcgen05 kernel), if that capture was of
-    this workload and of the kernel sources as they are now; otherwise None."""
+    "rows16_tcgen05" = 16 rows on the tcgen05 kernel), if a capture of that
+    kind was of this workload and of the kernel sources as they are now;
+    otherwise None."""
     import hashlib
-    if kind not in PROFILE_FOR:
-        return None
-    prof = os.path.join(ROOT, "profiles", PROFILE_FOR[kind])
-    try:
-        text = open(prof).read()
-    except OSError:
-        return None
-    fields = {}
-    for line in text.splitlines():
-        line = line.strip()
-        if ":" in line and line.split(":")[0] in ("kernel_sources_sha256_16", "workload", "traffic_bytes_per_launch"):
-            k, v = line.split(":", 1)
-            fields[k.strip()] = v.strip()
-    if fields.get("workload") != config or "traffic_bytes_per_launch" not in fields:
-        return None
-    csrc = os.path.join(ROOT, "paged_kv_cache_333_b200", "csrc")
-    for item in fields.get("kernel_sources_sha256_16", "").split():
-        name, digest = item.split("=")
-        with open(os.path.join(csrc, name), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
-                return None
-    return int(fields["traffic_bytes_per_launch"])
+    for name in PROFILE_FOR.get(kind, ()):
+        try:
+            text = open(os.path.join(ROOT, "profiles", name)).read()
+        except OSError:
+            continue
+        fields = {}
+        for line in text.splitlines():
+            line = line.strip()
+            if ":" in line and line.split(":")[0] in ("kernel_sources_sha256_16", "workload",
+                                                       "traffic_bytes_per_launch"):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+        if fields.get("workload") != config or "traffic_bytes_per_launch" not in fields:
+            continue
+        csrc = os.path.join(ROOT, "paged_kv_cache_333_b200", "csrc")
+        current = True
+        for item in fields.get("kernel_sources_sha256_16", "").split():
+            fname, digest = item.split("=")
+            with open(os.path.join(csrc, fname), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest()[:16] != digest:
+                    current = False
+        if current:
+            return int(fields["traffic_bytes_per_launch"])
+    return None
 
 
 # --------------------------------------------------------------------------- bytes

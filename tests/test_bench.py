@@ -41,6 +41,7 @@ def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
         assert isinstance(t, int) and t > 0, kind
     assert bench.profiled_traffic("long", "bf16") is None  # captured on chat only
     assert bench.profiled_traffic("chat", "rows8") is None
+    assert bench.profiled_traffic("sweep_b1", "fp8") > 0  # a second capture of the same kind
     # a copy of the tree with one kernel source edited: no traffic reported
     root = tmp_path / "tree"
     shutil.copytree(os.path.join(bench.ROOT, "profiles"), root / "profiles")
