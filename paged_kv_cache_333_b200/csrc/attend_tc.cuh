@@ -27,21 +27,26 @@
 // loads in flight for about a third of its life (set-up, first load,
 // epilogue).
 //
-// Roles (192 threads):
+// Roles (320 threads):
 //   warps 0-3  softmax: thread t owns column t of the unit, which is tensor-
 //              memory lane t (a warp may only read lanes 32 * (warp % 4) ..
 //              + 31).  Per tile: read its S row (64 fp32), mask, online
 //              softmax with a lazily moved reference max, write its P row
-//              (bf16 pairs) to tensor memory; per unit: read its O row and
-//              write the output (or the split-K partials), then free O;
+//              (bf16 pairs) to tensor memory; per unit: leave (m_ref, l) in
+//              tensor memory for the epilogue warps and go on to the next;
 //   warp 4     producer: per unit, the block-table slice into shared memory,
 //              the q tile by TMA (two buffers), and the 64-token K/V tiles
 //              into a 5-stage ring, by TMA for whole tiles of blocks >= 8
 //              tokens, else by a cp.async gather that zero-fills the rows past
 //              the range;
-//   warp 5     allocates tensor memory; one thread issues the MMAs.
+//   warp 5     allocates tensor memory; one thread issues the MMAs;
+//   warps 6-9  epilogue: warp w reads lane quarter w % 4 of a finished
+//              unit's O buffer and (m_ref, l), and writes the output rows (or
+//              the split-K partials), while the softmax warps already work on
+//              the next unit.
 // Tensor memory (512 columns): S double-buffered in [0, 64) and [64, 128),
-// O in [128, 256), P double-buffered in [256, 288) and [288, 320).
+// O double-buffered by unit in [128, 256) and [256, 384), P double-buffered
+// in [384, 416) and [416, 448), (m_ref, l) of unit k at 448 + 2 (k % 2).
 //
 // Lazy rescaling.  A column keeps a reference max m_ref (log2 domain) and
 // moves it only when a tile's max exceeds it by more than 8; the weights
@@ -61,7 +66,10 @@
 //   s_free[b]   softmax (4 warps) -> MMA  S buffer b read
 //   p_full[b]   softmax (4 warps) -> MMA  P buffer b written, O rescaled
 //   pv_done[b]  MMA commit -> softmax  P V of tile t done: P buffer b free, O current
-//   o_free      softmax (4 warps) -> MMA  unit k's O read: the next unit may overwrite it
+//   o_full[b]   MMA commit -> epilogue  unit k's last P V done: O buffer b = k % 2 final
+//   ml_full[b]  softmax (4 warps) -> epilogue  unit k's (m_ref, l) in tensor memory
+//   o_free[b]   epilogue (4 warps) -> MMA, softmax  unit k's O and (m_ref, l) read:
+//               unit k + 2 may overwrite them
 // The MMA thread issues S(t + 1) before P V(t), so the tensor pipe computes
 // the next scores while the softmax warps work on the current tile.  No
 // waiter can fall two phases behind a barrier: each phase it waits for is
@@ -76,11 +84,16 @@ constexpr int kTokTc = 64;      // tokens per tile
 constexpr int kStagesTc = 5;    // K/V ring depth
 constexpr int kMaxPartBlocksTc = 256;  // block-table entries one work unit may cover
 constexpr int kColsTc = 128;    // columns per CTA (= MMA M = tensor-memory lanes)
-constexpr int kTmemColsTc = 512;  // S 2x64, O 128, P 2x32 (bf16 pairs)
-constexpr int kTcThreads = 192;
+constexpr int kTmemColsTc = 512;  // S 2x64, O 2x128, P 2x32 (bf16 pairs), (m_ref, l) 2x2
+constexpr int kTmemOTc = 2 * kTokTc;             // O of unit k in [128 + 128 (k % 2), ...)
+constexpr int kTmemPTc = kTmemOTc + 2 * kD;      // P of tile t in [384 + 32 (t % 2), ...)
+constexpr int kTmemMlTc = kTmemPTc + 2 * 32;     // (m_ref, l) of unit k at 448 + 2 (k % 2)
+static_assert(kTmemMlTc + 4 <= kTmemColsTc, "tensor memory columns");
+constexpr int kTcThreads = 320;
 constexpr int kTcSoftmaxThreads = 128;
 constexpr int kTcProducerWarp = 4;
 constexpr int kTcMmaWarp = 5;
+constexpr int kTcEpilogueWarp0 = 6;  // warps 6-9: lane quarters 2, 3, 0, 1
 constexpr float kLazyRescaleLog2 = 8.f;
 
 // ---------------------------------------------------------------- descriptors
@@ -242,6 +255,45 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, uint32_t &a, uint32_t &b) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(a), "=r"(b)
+        : "r"(taddr)
+        : "memory");
+}
+// 64 consecutive fp32 columns of this thread's lane, one load and one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+}
+
+// mbar_wait for warps off the critical path: sleeps between polls so that
+// its spinning takes few issue slots from the warps it shares a scheduler
+// with; the same time limit.
+__device__ __forceinline__ bool mbar_wait_idle(uint64_t *bar, uint32_t parity) {
+    const uint32_t addr = smem_addr(bar);
+    if (mbar_try_wait(addr, parity))
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (;;) {
+        __nanosleep(200);
+        if (mbar_try_wait(addr, parity))
+            return true;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            flag_error(PA_DEVERR_TIMEOUT);
+            return false;
+        }
+    }
+}
 
 // max(a, b, c) in one instruction (the three-input form of max.f32, sm_100).
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
@@ -277,7 +329,9 @@ struct AttendTcSmem {
     uint64_t pv_done[2];
     uint64_t q_full[2];
     uint64_t q_empty[2];
-    uint64_t o_free;
+    uint64_t o_full[2];
+    uint64_t o_free[2];
+    uint64_t ml_full[2];
     uint64_t mma_done;
     uint32_t tmem_base;
     int32_t blocks[kMaxPartBlocksTc];
@@ -392,7 +446,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_init(&sm.q_full[b], 1);
             mbar_init(&sm.q_empty[b], 1);
         }
-        mbar_init(&sm.o_free, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.o_full[b], 1);
+            mbar_init(&sm.o_free[b], 4);
+            mbar_init(&sm.ml_full[b], 4);
+        }
         mbar_init(&sm.mma_done, 1);
         mbar_init_fence();
     }
@@ -411,8 +469,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tmem_o = tmem + 2 * kTokTc;
-    const uint32_t tmem_p = tmem + 2 * kTokTc + kD;  // two P buffers of 32 columns
+    const uint32_t tmem_o = tmem + kTmemOTc;
+    const uint32_t tmem_p = tmem + kTmemPTc;
     grid_dependency_wait();
 
     if (warp == kTcProducerWarp) {
@@ -533,29 +591,33 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     } else if (warp == kTcMmaWarp) {
         // ============================================================ MMA issue
         if (lane == 0) {
-            // P V of tile pt (the first of its unit when first; unit index pk):
-            // O is overwritten by the first one, after the previous unit's
-            // epilogue has read it
-            auto pv = [&](int pt, bool first, int pk) -> bool {
+            // P V of tile pt (the first / last of its unit when first / last;
+            // unit index pk) into the O buffer of its unit: the first one
+            // overwrites it, after the epilogue warps have read unit pk - 2's O
+            // from it; the last one's completion hands it to the epilogue warps
+            auto pv = [&](int pt, bool first, bool last, int pk) -> bool {
+                const int ob = pk & 1;
                 if (!mbar_wait(&sm.p_full[pt & 1], (pt >> 1) & 1))
                     return false;
-                if (first && pk >= 1 && !mbar_wait(&sm.o_free, (pk - 1) & 1))
+                if (first && pk >= 2 && !mbar_wait(&sm.o_free[ob], ((pk >> 1) - 1) & 1))
                     return false;
                 tc_fence_after();
                 const uint32_t v_base = smem_addr(&sm.kv[pt % kStagesTc][2][0]);
 #pragma unroll
                 for (int kk = 0; kk < kTokTc / 16; ++kk)
-                    umma_bf16_ts(tmem_o, tmem_p + (pt & 1) * 32 + kk * 8,
+                    umma_bf16_ts(tmem_o + ob * kD, tmem_p + (pt & 1) * 32 + kk * 8,
                                  umma_sdesc_sw128(v_base + v_step(kk), kLboV, kSbo), kIdescPV,
                                  (!first || kk > 0) ? 1u : 0u);
                 umma_commit(&sm.pv_done[pt & 1]);
                 umma_commit(&sm.empty[pt % kStagesTc]);
+                if (last)
+                    umma_commit(&sm.o_full[ob]);
                 return true;
             };
             bool ok = true;
             int T = 0, k = 0;
             int prev_t = -1, prev_k = 0;
-            bool prev_first = false;
+            bool prev_first = false, prev_last = false;
             TcRaw raw = tc_raw(ap, blockIdx.x);
             for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
                 const TcUnit w = tc_unit<G>(ap, raw);
@@ -585,20 +647,93 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     if (t == w.num_tiles - 1)
                         umma_commit(&sm.q_empty[qb]);  // the unit's last S read of this q buffer
                     if (prev_t >= 0)
-                        ok = pv(prev_t, prev_first, prev_k);
+                        ok = pv(prev_t, prev_first, prev_last, prev_k);
                     prev_t = T;
                     prev_first = t == 0;
+                    prev_last = t == w.num_tiles - 1;
                     prev_k = k;
                 }
                 ++k;
             }
             if (ok && prev_t >= 0)
-                pv(prev_t, prev_first, prev_k);
+                pv(prev_t, prev_first, prev_last, prev_k);
             // everything issued above has completed before the allocation is freed
             umma_commit(&sm.mma_done);
             mbar_wait(&sm.mma_done, 0);
         }
         __syncwarp();
+    } else if (warp >= kTcEpilogueWarp0) {
+        // ============================================================ epilogue
+        // Warp 6 + i reads lane quarter (6 + i) % 4 of unit k's O buffer once
+        // the unit's last P V has completed and the softmax warps have left
+        // (m_ref, l), writes the output rows (or the split-K partials), and
+        // frees the buffer; the softmax warps meanwhile work on unit k + 1.
+        const int quarter = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        bool ok = true;
+        int k = 0;
+        TcRaw raw = tc_raw(ap, blockIdx.x);
+        for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
+            const TcUnit w = tc_unit<G>(ap, raw);
+            raw = tc_raw(ap, u + gridDim.x);
+            if (!w.work)
+                continue;
+            const int ob = k & 1;
+            if (lane == 0) {
+                ok = mbar_wait_idle(&sm.o_full[ob], (k >> 1) & 1);
+                if (ok)
+                    ok = mbar_wait_idle(&sm.ml_full[ob], (k >> 1) & 1);
+            }
+            ok = __shfl_sync(FULL, ok, 0);
+            if (!ok)
+                break;
+            tc_fence_after();
+            const int c = w.col0 + quarter * 32 + lane;
+            const int lim = c <= w.last_col ? w.first_visible + c / G : -1;
+            const bool warp_live = __any_sync(FULL, lim >= w.t_begin);
+            if (warp_live) {
+                uint32_t mr, lr;
+                tmem_ld2(tmem + kTmemMlTc + 2 * ob + lane_base, mr, lr);
+                const float m_ref = __uint_as_float(mr), l = __uint_as_float(lr);
+                const bool valid = c <= w.last_col;
+                const int64_t qrow = valid ? w.q0 + c / G : 0;
+                const int j = w.h * G + c % G;
+#pragma unroll 1
+                for (int cc = 0; cc < kD / 32; ++cc) {
+                    uint32_t o[32];
+                    __syncwarp();  // the load is warp-collective
+                    tmem_ld32(tmem_o + ob * kD + lane_base + cc * 32, o);
+                    if (!valid) {
+                    } else if (p.num_parts == 1) {
+                        const float inv = l > 0.f ? 1.f / l : 0.f;
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qrow * p.num_q_heads + j) * kD + cc * 32);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 v;
+                            v.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
+                            v.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
+                            v.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
+                            v.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
+                            dst[q4] = v;
+                        }
+                    } else {
+                        const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + w.part;
+                        float4 *dst = reinterpret_cast<float4 *>(p.part_acc + idx * kD + cc * 32);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
+                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
+                        if (cc == 0)
+                            p.part_ml[idx] = make_float2(m_ref, l);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sm.o_free[ob]);
+            ++k;
+        }
     } else {
         // ============================================================ softmax
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
@@ -635,26 +770,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 // raw scores; tokens column c does not see get `masked`
                 float x[kTokTc];
                 if (warp_live) {
-                    uint32_t s[32];
-                    tmem_ld32(tmem + lane_base + (T & 1) * kTokTc, s);
+                    uint32_t s[64];
+                    tmem_ld64(tmem + lane_base + (T & 1) * kTokTc, s);
                     if (jcount == kTokTc) {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
+                        for (int j = 0; j < 64; ++j)
                             x[j] = __uint_as_float(s[j]);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 32; ++j)
+                        for (int j = 0; j < 64; ++j)
                             x[j] = j < jcount ? __uint_as_float(s[j]) : masked;
-                    }
-                    tmem_ld32(tmem + lane_base + (T & 1) * kTokTc + 32, s);
-                    if (jcount == kTokTc) {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            x[32 + j] = __uint_as_float(s[j]);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            x[32 + j] = 32 + j < jcount ? __uint_as_float(s[j]) : masked;
                     }
                 }
                 tc_fence_before();
@@ -716,11 +841,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
 #pragma unroll 1
                         for (int cc = 0; cc < kD / 32; ++cc) {
                             uint32_t o[32];
-                            tmem_ld32(tmem_o + lane_base + cc * 32, o);
+                            tmem_ld32(tmem_o + (k & 1) * kD + lane_base + cc * 32, o);
 #pragma unroll
                             for (int j = 0; j < 32; ++j)
                                 o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-                            tmem_st32(tmem_o + lane_base + cc * 32, o);
+                            tmem_st32(tmem_o + (k & 1) * kD + lane_base + cc * 32, o);
                         }
                         tmem_st_wait();
                     }
@@ -752,49 +877,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if (lane == 0)
                     mbar_arrive(&sm.p_full[T & 1]);
             }
-            // ---- epilogue: this column's O row, then O is free for the next unit
-            if (ok && lane == 0)
-                ok = mbar_wait(&sm.pv_done[(T - 1) & 1], ((T - 1) >> 1) & 1);
+            // ---- end of unit: hand this column's (m_ref, l) to the epilogue
+            // warps through tensor memory (its slot of unit k - 2 read first)
+            const int ob = k & 1;
+            if (ok && k >= 2 && lane == 0)
+                ok = mbar_wait(&sm.o_free[ob], ((k >> 1) - 1) & 1);
             ok = __shfl_sync(FULL, ok, 0);
-            if (ok && warp_live) {
-                tc_fence_after();
-                const bool valid = c <= w.last_col;
-                const int64_t qrow = valid ? w.q0 + c / G : 0;
-                const int j = w.h * G + c % G;
-#pragma unroll 1
-                for (int cc = 0; cc < kD / 32; ++cc) {
-                    uint32_t o[32];
-                    __syncwarp();  // the load is warp-collective
-                    tmem_ld32(tmem_o + lane_base + cc * 32, o);
-                    if (!valid) {
-                    } else if (p.num_parts == 1) {
-                        const float inv = l > 0.f ? 1.f / l : 0.f;
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (qrow * p.num_q_heads + j) * kD + cc * 32);
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 v;
-                            v.x = pack_bf16x2(__uint_as_float(o[8 * q4 + 0]) * inv, __uint_as_float(o[8 * q4 + 1]) * inv);
-                            v.y = pack_bf16x2(__uint_as_float(o[8 * q4 + 2]) * inv, __uint_as_float(o[8 * q4 + 3]) * inv);
-                            v.z = pack_bf16x2(__uint_as_float(o[8 * q4 + 4]) * inv, __uint_as_float(o[8 * q4 + 5]) * inv);
-                            v.w = pack_bf16x2(__uint_as_float(o[8 * q4 + 6]) * inv, __uint_as_float(o[8 * q4 + 7]) * inv);
-                            dst[q4] = v;
-                        }
-                    } else {
-                        const int64_t idx = (qrow * p.num_q_heads + j) * p.num_parts + w.part;
-                        float4 *dst = reinterpret_cast<float4 *>(p.part_acc + idx * kD + cc * 32);
-#pragma unroll
-                        for (int q4 = 0; q4 < 8; ++q4)
-                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]), __uint_as_float(o[4 * q4 + 1]),
-                                                  __uint_as_float(o[4 * q4 + 2]), __uint_as_float(o[4 * q4 + 3]));
-                        if (cc == 0)
-                            p.part_ml[idx] = make_float2(m_ref, l);
-                    }
-                }
-            }
+            if (!ok)
+                break;
+            tc_fence_after();
+            tmem_st2(tmem + kTmemMlTc + 2 * ob + lane_base, __float_as_uint(m_ref), __float_as_uint(l));
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&sm.o_free);
+                mbar_arrive(&sm.ml_full[ob]);
             ++k;
         }
         if (threadIdx.x == 0)
