@@ -278,16 +278,20 @@ PA_API int32_t pa_decode_set_kernel(int32_t kind);
  *   PA_ATTENTION_KERNEL_MMA     warps of 8 (row, head) columns on
  *                               mma.m16n8k16, 16-token K/V tiles: for a few
  *                               rows per request (speculative decoding);
- *   PA_ATTENTION_KERNEL_TCGEN05 128 columns per CTA on tcgen05.mma with the
- *                               S and O accumulators in tensor memory, 64-token
- *                               K/V tiles: for requests with many rows
- *                               (prefill chunks);
+ *   PA_ATTENTION_KERNEL_TCGEN05 work units of 128 (row, head) columns (two KV
+ *                               heads of up to 64 columns each, when the KV
+ *                               head count is even) on tcgen05.mma with S, P
+ *                               and O in tensor memory, 64-row K/V tiles: for
+ *                               requests with many rows (prefill chunks);
  *   PA_ATTENTION_KERNEL_AUTO    (default) per call: the tcgen05 kernel when
  *                               max_query_len x (num_q_heads / num_kv_heads)
- *                               is at least PA_ATTENTION_TCGEN05_MIN_COLUMNS,
- *                               else the mma.sync kernel. */
+ *                               is at least PA_ATTENTION_TCGEN05_MIN_COLUMNS
+ *                               (above 16 columns the mma.sync kernel moves to
+ *                               its wider CTA shape, and the tcgen05 kernel is
+ *                               faster from there on B200), else the mma.sync
+ *                               kernel. */
 enum { PA_ATTENTION_KERNEL_MMA = 0, PA_ATTENTION_KERNEL_TCGEN05 = 1, PA_ATTENTION_KERNEL_AUTO = 2 };
-#define PA_ATTENTION_TCGEN05_MIN_COLUMNS 64
+#define PA_ATTENTION_TCGEN05_MIN_COLUMNS 17
 PA_API int32_t pa_attention_set_kernel(int32_t kind);
 
 /* Tokens per split-K partition used by pa_decode: 0 = automatic (the

@@ -31,7 +31,7 @@ EXPORTED = ("pa_write_kv", "pa_compute_slot_mapping", "pa_write_kv_positions", "
             "pa_last_cuda_error", "pa_status_str")
 PA_DECODE_KERNEL_MMA, PA_DECODE_KERNEL_SIMT = 0, 1
 PA_ATTENTION_KERNEL_MMA, PA_ATTENTION_KERNEL_TCGEN05, PA_ATTENTION_KERNEL_AUTO = 0, 1, 2
-PA_ATTENTION_TCGEN05_MIN_COLUMNS = 64  # include/pa.h
+PA_ATTENTION_TCGEN05_MIN_COLUMNS = 17  # include/pa.h
 
 
 class PaCache(ctypes.Structure):

@@ -86,7 +86,8 @@ struct AttendParams {
     int32_t max_query_len;
     int32_t chunks;                  // column chunks per request
     int32_t num_kv_heads;            // tcgen05 kernel: the KV heads (its grid is 1-D)
-    int32_t num_units;               // tcgen05 kernel: partitions x KV heads x requests x chunks
+    int32_t head_groups;             // tcgen05 kernel: KV heads / heads per work unit
+    int32_t num_units;               // tcgen05 kernel: partitions x head groups x requests x chunks
 };
 
 template <int W>

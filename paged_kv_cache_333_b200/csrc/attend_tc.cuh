@@ -82,18 +82,19 @@ namespace pa {
 
 constexpr int kTokTc = 64;      // tokens per tile
 constexpr int kStagesTc = 5;    // K/V ring depth
-constexpr int kMaxPartBlocksTc = 256;  // block-table entries one work unit may cover
+constexpr int kMaxPartBlocksTc = 192;  // block-table entries one work unit may cover
 constexpr int kColsTc = 128;    // columns per CTA (= MMA M = tensor-memory lanes)
 constexpr int kTmemColsTc = 512;  // S 2x64, O 2x128, P 2x32 (bf16 pairs), (m_ref, l) 2x2
 constexpr int kTmemOTc = 2 * kTokTc;             // O of unit k in [128 + 128 (k % 2), ...)
 constexpr int kTmemPTc = kTmemOTc + 2 * kD;      // P of tile t in [384 + 32 (t % 2), ...)
 constexpr int kTmemMlTc = kTmemPTc + 2 * 32;     // (m_ref, l) of unit k at 448 + 2 (k % 2)
 static_assert(kTmemMlTc + 4 <= kTmemColsTc, "tensor memory columns");
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 352;
 constexpr int kTcSoftmaxThreads = 128;
 constexpr int kTcProducerWarp = 4;
 constexpr int kTcMmaWarp = 5;
 constexpr int kTcEpilogueWarp0 = 6;  // warps 6-9: lane quarters 2, 3, 0, 1
+constexpr int kTcProducer2Warp = 10;  // the second producer
 constexpr float kLazyRescaleLog2 = 8.f;
 
 // ---------------------------------------------------------------- descriptors
@@ -254,6 +255,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st2(uint32_t taddr, uint32_t a, uint32_t b) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(a), "r"(b) : "memory");
@@ -334,18 +343,18 @@ struct AttendTcSmem {
     uint64_t ml_full[2];
     uint64_t mma_done;
     uint32_t tmem_base;
-    int32_t blocks[kMaxPartBlocksTc];
+    int32_t blocks[2][kMaxPartBlocksTc];  // each producer's copy of the unit's table slice
 };
 constexpr size_t kAttendTcSmemBytes = sizeof(AttendTcSmem) + 1024;
 static_assert(kAttendTcSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(offsetof(AttendTcSmem, q) % 1024 == 0, "swizzle atoms start on 1024-byte boundaries");
 
-// One work unit: (split-K partition, KV head, request, 128-column chunk),
-// numbered as part + P * (head + Hkv * (request * chunks + chunk)).  Every
-// role derives the same fields from global memory, so all agree on which
-// units have work and on their tile counts.
+// One work unit: (split-K partition, group of HP KV heads, request, chunk of
+// 128 / HP columns), numbered as part + P * (group + (Hkv / HP) * (request *
+// chunks + chunk)).  Every role derives the same fields from global memory,
+// so all agree on which units have work and on their tile counts.
 struct TcUnit {
-    int part, h, r, chunk;
+    int part, h, r, chunk;  // h: the head group (KV heads h * HP .. h * HP + HP - 1)
     int q0, n, col0, last_col, first_visible, t_begin, t_end, num_tiles;
     bool bad;   // query_start_loc / seq_lens inconsistent for this request
     bool work;  // at least one tile
@@ -359,7 +368,7 @@ struct TcRaw {
 __device__ __forceinline__ TcRaw tc_raw(const AttendParams &ap, int u) {
     TcRaw raw{u, 0, 0, 0};
     if (u < ap.num_units) {
-        const int r = (u / ap.d.num_parts / ap.num_kv_heads) / ap.chunks;
+        const int r = (u / ap.d.num_parts / ap.head_groups) / ap.chunks;
         raw.q0 = ap.query_start_loc[r];
         raw.q1 = ap.query_start_loc[r + 1];
         raw.n = ap.d.seq_lens[r];
@@ -367,15 +376,15 @@ __device__ __forceinline__ TcRaw tc_raw(const AttendParams &ap, int u) {
     return raw;
 }
 
-template <int G>
+template <int G, int HP>
 __device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &raw) {
     const DecodeParams &p = ap.d;
     TcUnit w{};
     const int u = raw.u;
     w.part = u % p.num_parts;
     int rest = u / p.num_parts;
-    w.h = rest % ap.num_kv_heads;
-    rest /= ap.num_kv_heads;
+    w.h = rest % ap.head_groups;
+    rest /= ap.head_groups;
     w.r = rest / ap.chunks;
     w.chunk = rest % ap.chunks;
     int n = raw.n;  // clamped as clamp_seq_len does
@@ -396,17 +405,17 @@ __device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &r
     if (w.bad)
         return w;
     const int cols = q_len * G;
-    w.col0 = w.chunk * kColsTc;
+    w.col0 = w.chunk * (kColsTc / HP);
     if (w.col0 >= cols)
         return w;
-    w.last_col = min(cols, w.col0 + kColsTc) - 1;
+    w.last_col = min(cols, w.col0 + kColsTc / HP) - 1;
     w.first_visible = n - q_len;  // row i sees positions <= first_visible + i
     const int lim_max = w.first_visible + w.last_col / G;
     w.t_begin = w.part * p.part_tokens;
     if (w.t_begin > lim_max)
         return w;
     w.t_end = min(lim_max + 1, w.t_begin + p.part_tokens);
-    w.num_tiles = (w.t_end - w.t_begin + kTokTc - 1) / kTokTc;
+    w.num_tiles = (w.t_end - w.t_begin + kTokTc / HP - 1) / (kTokTc / HP);
     w.work = true;
     return w;
 }
@@ -418,11 +427,24 @@ __device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &r
 //
 // kZeroScale: the caller's scale is 0, so every visible token weighs 1 and a
 // masked one 0; the scaled-score form below would give 0 * inf there.
-template <int G, bool kZeroScale>
+//
+// HP (1 or 2): KV heads per work unit.  With HP = 2 (at most 64 columns per
+// head) a tile is 32 tokens of both heads: stage rows 0-31 hold head 2g's K
+// (V) rows, rows 32-63 head 2g + 1's, and the q tile holds head 2g's columns
+// in MMA rows 0-63 and head 2g + 1's in rows 64-127.  The MMAs are those of
+// HP = 1; S's two off-diagonal 64 x 32 blocks (one head's q against the
+// other's K) are not read, and each softmax warp writes zeros into the P
+// columns of the other head's tokens, so P V adds only a head's own tokens
+// into its O rows.  All four softmax warps then have live columns, and a
+// 32 KiB stage still feeds one tile, so the ring keeps its depth.
+template <int G, bool kZeroScale, int HP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_q, const AttendParams ap) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+    static_assert(HP == 1 || HP == 2, "heads per work unit");
+    constexpr int kTokH = kTokTc / HP;   // tokens of one head per tile
+    constexpr int kColsH = kColsTc / HP;  // columns of one head per unit
     constexpr unsigned FULL = 0xffffffffu;
     const DecodeParams &p = ap.d;
     extern __shared__ uint8_t smem_raw[];
@@ -473,14 +495,20 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     const uint32_t tmem_p = tmem + kTmemPTc;
     grid_dependency_wait();
 
-    if (warp == kTcProducerWarp) {
-        // ============================================================ producer
+    if (warp == kTcProducerWarp || warp == kTcProducer2Warp) {
+        // ============================================================ producers
+        // Producer p fills the ring slots s with s % 2 == p, so each slot has
+        // one owner that waits for every phase of it; producer 0 also loads
+        // the q tiles.  One warp issuing all 16 boxes of every tile could not
+        // keep the stream at the rate two-head tiles are consumed.
+        const int pidx = warp == kTcProducer2Warp;
+        int32_t *const blocks = sm.blocks[pidx];
         const uint64_t pol = l2_evict_first_policy();
         int T = 0, k = 0;
         bool dead = false;
         TcRaw raw = tc_raw(ap, blockIdx.x);
         for (int u = blockIdx.x; u < ap.num_units && !dead; u += gridDim.x) {
-            const TcUnit w = tc_unit<G>(ap, raw);
+            const TcUnit w = tc_unit<G, HP>(ap, raw);
             raw = tc_raw(ap, u + gridDim.x);
             if (w.bad && w.part == 0 && w.h == 0 && w.chunk == 0 && lane == 0)
                 flag_error(PA_DEVERR_QUERY_LOC);
@@ -498,15 +526,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         flag_error(PA_DEVERR_BLOCK_ID);
                         b = 0;
                     }
-                    sm.blocks[i] = b;
+                    blocks[i] = b;
                 }
             }
             __syncwarp();
-            // the unit's q tile: rows q0 + col0/G .., heads hG .. hG+G-1, both
-            // 64-dim halves; rows past the request hold other rows or zeros
-            // (their columns are masked)
+            // the unit's q tile, both 64-dim halves, as two boxes of 64 columns
+            // each: MMA rows 0-63 and 64-127 are columns col0 .. and col0 + 64 ..
+            // of the unit's head (HP = 1) or columns col0 .. of its first and
+            // second head (HP = 2); column c of head h is q row q0 + c / G, head
+            // h G + c % G.  Rows past the request hold other rows or zeros
+            // (their columns are masked).
             const int qb = k & 1;
-            if (k >= 2) {
+            if (pidx == 0 && k >= 2) {
                 bool ok = true;
                 if (lane == 0)
                     ok = mbar_wait(&sm.q_empty[qb], ((k >> 1) - 1) & 1);
@@ -515,13 +546,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     break;
                 }
             }
-            if (lane == 0) {
+            if (pidx == 0 && lane == 0) {
                 mbar_arrive_expect_tx(&sm.q_full[qb], static_cast<uint32_t>(2 * kColsTc * 128));
-                tma_load_3d(&sm.q[qb][0][0], &tm_q, 0, w.h * G, w.q0 + w.col0 / G, &sm.q_full[qb], pol);
-                tma_load_3d(&sm.q[qb][1][0], &tm_q, 64, w.h * G, w.q0 + w.col0 / G, &sm.q_full[qb], pol);
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+#pragma unroll
+                    for (int rb = 0; rb < 2; ++rb) {
+                        const int head = w.h * HP + (HP == 2 ? rb : 0);
+                        const int qrow = w.q0 + (w.col0 + (HP == 1 ? rb * 64 : 0)) / G;
+                        tma_load_3d(&sm.q[qb][d][rb * 64 * 64], &tm_q, d * 64, head * G, qrow, &sm.q_full[qb], pol);
+                    }
             }
             for (int it = 0; it < w.num_tiles; ++it, ++T) {
                 const int slot = T % kStagesTc;
+                if ((slot & 1) != pidx)
+                    continue;
                 if (T >= kStagesTc) {
                     bool ok = true;
                     if (lane == 0)
@@ -531,40 +570,45 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         break;
                     }
                 }
-                const int t0 = w.t_begin + it * kTokTc;
-                const int ntok = min(kTokTc, w.t_end - t0);
-                if (B >= 8 && ntok == kTokTc) {
-                    // whole tile by TMA: boxes of min(B, 16) rows, 4 quarters each
+                // stage row hh * kTokH + i holds token t0 + i of head w.h * HP + hh
+                const int t0 = w.t_begin + it * kTokH;
+                const int ntok = min(kTokH, w.t_end - t0);
+                if (B >= 8 && ntok == kTokH) {
+                    // whole tile by TMA: boxes of min(B, 16) rows, 4 quarters each,
+                    // per head
                     const int rows = B < kTile ? B : kTile;
-                    const int nbox = kTokTc / rows;  // 4 or 8
+                    const int nbox = kTokH / rows;  // HP * nbox * 4 <= 32 lanes
                     if (lane == 0)
                         mbar_arrive_expect_tx(&sm.full[slot], static_cast<uint32_t>(kTokTc * 128 * 4));
                     __syncwarp();
-                    const int j = lane >> 2, qd = lane & 3;  // box j of quarter qd (K lo, K hi, V lo, V hi)
-                    if (j < nbox) {
+                    // box j of head hh of quarter qd (K lo, K hi, V lo, V hi)
+                    const int qd = lane & 3, j = (lane >> 2) % nbox, hh = (lane >> 2) / nbox;
+                    if (hh < HP) {
                         const int t = t0 + j * rows;
-                        const int32_t rr = sm.blocks[t / B - first_blk] * B + (t % B);
-                        tma_load_3d(&sm.kv[slot][qd][j * rows * 64], (qd < 2) ? &tm_k : &tm_v, (qd & 1) * 64, w.h,
-                                    rr, &sm.full[slot], pol);
+                        const int32_t rr = blocks[t / B - first_blk] * B + (t % B);
+                        tma_load_3d(&sm.kv[slot][qd][(hh * kTokH + j * rows) * 64], (qd < 2) ? &tm_k : &tm_v,
+                                    (qd & 1) * 64, w.h * HP + hh, rr, &sm.full[slot], pol);
                     }
                 } else {
                     // gather: lane = (quarter, 16-byte chunk); rows past the range
                     // are zero-filled so that 0-weight V rows stay finite
                     const int qd = lane >> 3, ch = lane & 7;
                     const uint16_t *cache = static_cast<const uint16_t *>(qd < 2 ? p.k_cache : p.v_cache);
-                    int64_t row_lo = 0, row_hi = 0;
+                    int64_t slot_lo = 0, slot_hi = 0;  // cache slots of tokens t0 + lane, t0 + lane + 32
                     if (lane < ntok) {
                         const int t = t0 + lane;
-                        row_lo = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + w.h;
+                        slot_lo = static_cast<int64_t>(blocks[t / B - first_blk]) * B + (t % B);
                     }
                     if (lane + 32 < ntok) {
                         const int t = t0 + lane + 32;
-                        row_hi = (static_cast<int64_t>(sm.blocks[t / B - first_blk]) * B + (t % B)) * Hkv + w.h;
+                        slot_hi = static_cast<int64_t>(blocks[t / B - first_blk]) * B + (t % B);
                     }
                     const uint32_t base = smem_addr(&sm.kv[slot][qd][0]);
                     for (int i = 0; i < kTokTc; ++i) {
-                        const int64_t rr = __shfl_sync(FULL, i < 32 ? row_lo : row_hi, i & 31);
-                        const bool in = i < ntok;
+                        const int hh = i / kTokH, tt = i % kTokH;
+                        const int64_t sl = __shfl_sync(FULL, tt < 32 ? slot_lo : slot_hi, tt & 31);
+                        const bool in = tt < ntok;
+                        const int64_t rr = sl * Hkv + w.h * HP + hh;
                         cp_async16_zfill(base + swz(i, ch), cache + (in ? rr * kD + (qd & 1) * 64 + ch * 8 : 0),
                                          in ? 16u : 0u);
                     }
@@ -579,11 +623,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         // nothing may still be copying into shared memory when the CTA ends
         asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0) {
-            for (int sl = 0; sl < kStagesTc && sl < T; ++sl) {
+            for (int sl = pidx; sl < kStagesTc && sl < T; sl += 2) {
                 const int last = sl + ((T - 1 - sl) / kStagesTc) * kStagesTc;
                 mbar_wait(&sm.full[sl], (last / kStagesTc) & 1);
             }
-            for (int b = 0; b < 2 && b < k; ++b) {
+            for (int b = 0; b < 2 && b < k && pidx == 0; ++b) {
                 const int last = b + ((k - 1 - b) / 2) * 2;
                 mbar_wait(&sm.q_full[b], (last >> 1) & 1);
             }
@@ -620,7 +664,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             bool prev_first = false, prev_last = false;
             TcRaw raw = tc_raw(ap, blockIdx.x);
             for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
-                const TcUnit w = tc_unit<G>(ap, raw);
+                const TcUnit w = tc_unit<G, HP>(ap, raw);
                 raw = tc_raw(ap, u + gridDim.x);
                 if (!w.work)
                     continue;
@@ -662,7 +706,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             mbar_wait(&sm.mma_done, 0);
         }
         __syncwarp();
-    } else if (warp >= kTcEpilogueWarp0) {
+    } else if (warp >= kTcEpilogueWarp0 && warp < kTcEpilogueWarp0 + 4) {
         // ============================================================ epilogue
         // Warp 6 + i reads lane quarter (6 + i) % 4 of unit k's O buffer once
         // the unit's last P V has completed and the softmax warps have left
@@ -674,7 +718,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int k = 0;
         TcRaw raw = tc_raw(ap, blockIdx.x);
         for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
-            const TcUnit w = tc_unit<G>(ap, raw);
+            const TcUnit w = tc_unit<G, HP>(ap, raw);
             raw = tc_raw(ap, u + gridDim.x);
             if (!w.work)
                 continue;
@@ -688,7 +732,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             if (!ok)
                 break;
             tc_fence_after();
-            const int c = w.col0 + quarter * 32 + lane;
+            const int hh = (quarter * 32) / kColsH;  // the unit's head of these rows
+            const int c = w.col0 + (quarter * 32 + lane) % kColsH;
             const int lim = c <= w.last_col ? w.first_visible + c / G : -1;
             const bool warp_live = __any_sync(FULL, lim >= w.t_begin);
             if (warp_live) {
@@ -697,7 +742,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 const float m_ref = __uint_as_float(mr), l = __uint_as_float(lr);
                 const bool valid = c <= w.last_col;
                 const int64_t qrow = valid ? w.q0 + c / G : 0;
-                const int j = w.h * G + c % G;
+                const int j = (w.h * HP + hh) * G + c % G;
 #pragma unroll 1
                 for (int cc = 0; cc < kD / 32; ++cc) {
                     uint32_t o[32];
@@ -737,6 +782,17 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     } else {
         // ============================================================ softmax
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const int hh = (warp * 32) / kColsH;  // the unit's head of this warp's columns
+        if constexpr (HP == 2) {
+            // the P columns of the other head's tokens stay zero in these lanes
+            uint32_t z[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                z[j] = 0u;
+            tmem_st16(tmem_p + lane_base + (1 - hh) * 16, z);
+            tmem_st16(tmem_p + lane_base + 32 + (1 - hh) * 16, z);
+            tmem_st_wait();
+        }
         // score multiplier (log2 domain) with the scale's sign; masked tokens
         // are set to the value that the multiplier sends to -inf
         const float sl2 = p.scale_log2;
@@ -746,11 +802,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         int T = 0, k = 0;
         TcRaw raw = tc_raw(ap, blockIdx.x);
         for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
-            const TcUnit w = tc_unit<G>(ap, raw);
+            const TcUnit w = tc_unit<G, HP>(ap, raw);
             raw = tc_raw(ap, u + gridDim.x);
             if (!w.work)
                 continue;
-            const int c = w.col0 + threadIdx.x;
+            const int c = w.col0 + threadIdx.x % kColsH;
             const int lim = c <= w.last_col ? w.first_visible + c / G : -1;  // last position column c sees
             const bool warp_live = __any_sync(FULL, lim >= w.t_begin);
             if (p.num_parts > 1 && w.part == 0 && w.h == 0 && warp == 0) {
@@ -764,21 +820,25 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if (!__shfl_sync(FULL, ok, 0))
                     break;
                 tc_fence_after();
-                const int t0 = w.t_begin + t * kTokTc;
-                const int ntok = min(kTokTc, w.t_end - t0);
+                const int t0 = w.t_begin + t * kTokH;
+                const int ntok = min(kTokH, w.t_end - t0);
                 const int jcount = max(0, min(ntok, lim - t0 + 1));  // tokens of this tile column c sees
-                // raw scores; tokens column c does not see get `masked`
-                float x[kTokTc];
+                // raw scores of this head's tokens (S columns hh * kTokH ..);
+                // tokens column c does not see get `masked`
+                float x[kTokH];
                 if (warp_live) {
-                    uint32_t s[64];
-                    tmem_ld64(tmem + lane_base + (T & 1) * kTokTc, s);
-                    if (jcount == kTokTc) {
+                    uint32_t s[kTokH];
+                    if constexpr (HP == 1)
+                        tmem_ld64(tmem + lane_base + (T & 1) * kTokTc, s);
+                    else
+                        tmem_ld32(tmem + lane_base + (T & 1) * kTokTc + hh * kTokH, s);
+                    if (jcount == kTokH) {
 #pragma unroll
-                        for (int j = 0; j < 64; ++j)
+                        for (int j = 0; j < kTokH; ++j)
                             x[j] = __uint_as_float(s[j]);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < 64; ++j)
+                        for (int j = 0; j < kTokH; ++j)
                             x[j] = j < jcount ? __uint_as_float(s[j]) : masked;
                     }
                 }
@@ -796,19 +856,23 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                 if (warp_live) {
                     // the tile's max of sl2 * x in the log2 domain: the max of x
                     // scaled, or with a negative scale the min of x
-                    float m8[8];
+                    constexpr int NG = kTokH / 8;
+                    float m8[NG];
                     float mt;
                     if (kZeroScale) {
                         mt = jcount > 0 ? 0.f : -INFINITY;
                     } else if (pos) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
+                        for (int i = 0; i < NG; ++i)
                             m8[i] = max8(&x[8 * i]);
-                        mt = sl2 * fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
-                                          fmaxf(m8[6], m8[7]));
+                        if constexpr (NG == 8)
+                            mt = sl2 * fmax3f(fmax3f(m8[0], m8[1], m8[2]), fmax3f(m8[3], m8[4], m8[5]),
+                                              fmaxf(m8[6], m8[7]));
+                        else
+                            mt = sl2 * fmax3f(m8[0], m8[1], fmaxf(m8[2], m8[3]));
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
+                        for (int i = 0; i < NG; ++i) {
                             float v = x[8 * i];
 #pragma unroll
                             for (int j = 1; j < 8; ++j)
@@ -817,7 +881,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         }
                         float v = m8[0];
 #pragma unroll
-                        for (int i = 1; i < 8; ++i)
+                        for (int i = 1; i < NG; ++i)
                             v = fminf(v, m8[i]);
                         mt = sl2 * v;
                     }
@@ -853,10 +917,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                     // 0 where masked.  While the column has seen nothing,
                     // m_ref is -inf: the offset 0 keeps the FMA at -inf.
                     const float neg = m_ref != -INFINITY ? -m_ref : 0.f;
-                    uint32_t pw[32];
+                    uint32_t pw[kTokH / 2];  // this head's tokens as bf16 pairs
                     float lsum = 0.f;
 #pragma unroll
-                    for (int kq = 0; kq < 8; ++kq) {
+                    for (int kq = 0; kq < kTokH / 8; ++kq) {
                         float e[8];
 #pragma unroll
                         for (int v = 0; v < 8; ++v)
@@ -868,7 +932,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                         pw[4 * kq + 2] = pack_bf16x2(e[4], e[5]);
                         pw[4 * kq + 3] = pack_bf16x2(e[6], e[7]);
                     }
-                    tmem_st32(tmem_p + lane_base + (T & 1) * 32, pw);
+                    if constexpr (HP == 1)
+                        tmem_st32(tmem_p + lane_base + (T & 1) * 32, pw);
+                    else
+                        tmem_st16(tmem_p + lane_base + (T & 1) * 32 + hh * 16, pw);
                     tmem_st_wait();
                     l += lsum;
                 }

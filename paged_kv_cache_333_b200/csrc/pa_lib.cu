@@ -318,7 +318,8 @@ namespace {
 // (m, l), acc and per-row length arrays when there is more than one
 // partition.
 struct AttendLayout {
-    bool tcgen05;  // attend_tc_kernel (128 columns per CTA), else attend_partition_kernel
+    bool tcgen05;  // attend_tc_kernel, else attend_partition_kernel
+    int32_t heads_per_unit;  // attend_tc_kernel: 2 KV heads per work unit when each has <= 64 columns
     int32_t warps, chunks, part_tokens, num_parts;
     size_t acc_offset, len_offset, total;
 };
@@ -329,8 +330,9 @@ AttendLayout attend_layout(int32_t num_reqs, int32_t num_tokens, int32_t max_que
     a.tcgen05 = tcgen05;
     const int64_t G = num_q_heads / num_kv_heads;
     const int64_t cols = static_cast<int64_t>(max_query_len) * G;
+    a.heads_per_unit = tcgen05 && cols <= pa::kColsTc / 2 && num_kv_heads % 2 == 0 ? 2 : 1;
     a.warps = cols <= 16 ? 2 : 4;  // CTA shape: 16 columns x 4 CTAs/SM, or 32 columns x 2 CTAs/SM
-    const int64_t per_cta = tcgen05 ? pa::kColsTc : 8 * a.warps;
+    const int64_t per_cta = tcgen05 ? pa::kColsTc / a.heads_per_unit : 8 * a.warps;
     a.chunks = static_cast<int32_t>(std::max<int64_t>(1, (cols + per_cta - 1) / per_cta));
     const int64_t units = std::min<int64_t>(INT32_MAX, static_cast<int64_t>(num_reqs) * a.chunks);
     a.part_tokens = choose_part_tokens(static_cast<int32_t>(units), num_kv_heads, max_seq_len, block_size, true);
@@ -379,8 +381,8 @@ int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Atte
 
 // The tensor-memory variant (attend_tc.cuh): 128 columns per CTA, one CTA per SM.
 // The q rows as a 3-D tensor (dim, head, row) for the tcgen05 kernel's TMA
-// loads of its q tiles: boxes of (64 dims, G heads, 128 / G rows), the
-// 128-byte swizzle, rows past num_tokens read as zeros.
+// loads of its q tiles: boxes of (64 dims, G heads, 64 / G rows), i.e. 64
+// columns, the 128-byte swizzle, rows past num_tokens read as zeros.
 int encode_q_map(CUtensorMap *tm, const void *q, int32_t num_tokens, int32_t num_q_heads, int32_t G) {
     auto fn = encode_fn();
     if (!fn) {
@@ -391,7 +393,7 @@ int encode_q_map(CUtensorMap *tm, const void *q, int32_t num_tokens, int32_t num
                                 static_cast<cuuint64_t>(num_tokens)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(pa::kD) * 2,
                                    static_cast<cuuint64_t>(num_q_heads) * pa::kD * 2};
-    const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(pa::kColsTc / G)};
+    const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(pa::kColsTc / 2 / G)};
     const cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -406,27 +408,48 @@ int encode_q_map(CUtensorMap *tm, const void *q, int32_t num_tokens, int32_t num
 
 // The tensor-memory variant (attend_tc.cuh): 128 columns per work unit, a
 // persistent grid of one CTA per SM walking the units.
-template <int G, bool kZeroScale>
+template <int G, bool kZeroScale, int HP>
 int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const void *q, pa::AttendParams ap,
                        int32_t num_kv_heads, cudaStream_t stream) {
     static CtxDone done = {};
-    int rc = prepare_kernel(pa::attend_tc_kernel<G, kZeroScale>, pa::kAttendTcSmemBytes, done);
+    int rc = prepare_kernel(pa::attend_tc_kernel<G, kZeroScale, HP>, pa::kAttendTcSmemBytes, done);
     if (rc)
         return rc;
     CUtensorMap tq;
     if ((rc = encode_q_map(&tq, q, ap.num_tokens, ap.d.num_q_heads, G)) != PA_OK)
         return rc;
-    const int64_t units = static_cast<int64_t>(ap.d.num_parts) * num_kv_heads * ap.d.num_seqs * ap.chunks;
+    const int64_t units = static_cast<int64_t>(ap.d.num_parts) * (num_kv_heads / HP) * ap.d.num_seqs * ap.chunks;
     if (units > INT32_MAX)
         return PA_EUNSUPPORTED;
     ap.num_kv_heads = num_kv_heads;
+    ap.head_groups = num_kv_heads / HP;
     ap.num_units = static_cast<int32_t>(units);
     const dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, sm_count())));
-    cudaError_t e = launch_pdl(pa::attend_tc_kernel<G, kZeroScale>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
+    cudaError_t e = launch_pdl(pa::attend_tc_kernel<G, kZeroScale, HP>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
                                stream, tk, tv, tq, ap);
     if (e != cudaSuccess)
         return cuda_fail(e, "attend_tc_kernel launch");
     return launch_row_merge(ap, stream);
+}
+
+template <bool kZeroScale, int HP>
+int launch_attend_tc_hp(int32_t G, const CUtensorMap &tk, const CUtensorMap &tv, const void *q,
+                        const pa::AttendParams &ap, int32_t nk, cudaStream_t st) {
+    switch (G) {
+    case 1: return launch_attend_tc_g<1, kZeroScale, HP>(tk, tv, q, ap, nk, st);
+    case 2: return launch_attend_tc_g<2, kZeroScale, HP>(tk, tv, q, ap, nk, st);
+    case 4: return launch_attend_tc_g<4, kZeroScale, HP>(tk, tv, q, ap, nk, st);
+    default: return launch_attend_tc_g<8, kZeroScale, HP>(tk, tv, q, ap, nk, st);
+    }
+}
+// The instantiation for a call: group size, zero scale, KV heads per unit.
+int launch_attend_tc(int32_t G, bool zero_scale, int32_t heads_per_unit, const CUtensorMap &tk,
+                     const CUtensorMap &tv, const void *q, const pa::AttendParams &ap, int32_t nk, cudaStream_t st) {
+    if (heads_per_unit == 2)
+        return zero_scale ? launch_attend_tc_hp<true, 2>(G, tk, tv, q, ap, nk, st)
+                          : launch_attend_tc_hp<false, 2>(G, tk, tv, q, ap, nk, st);
+    return zero_scale ? launch_attend_tc_hp<true, 1>(G, tk, tv, q, ap, nk, st)
+                      : launch_attend_tc_hp<false, 1>(G, tk, tv, q, ap, nk, st);
 }
 
 pa_cache_t as_cache(const pa_cache_fp8_t *c) {
@@ -918,21 +941,7 @@ int pa_attention(const void *q, int32_t num_tokens, const int32_t *query_start_l
     ap.chunks = a.chunks;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (a.tcgen05) {
-        const int nk = cache->num_kv_heads;
-        if (scale == 0.f) {
-            switch (G) {
-            case 1: return launch_attend_tc_g<1, true>(tk, tv, q, ap, nk, st);
-            case 2: return launch_attend_tc_g<2, true>(tk, tv, q, ap, nk, st);
-            case 4: return launch_attend_tc_g<4, true>(tk, tv, q, ap, nk, st);
-            default: return launch_attend_tc_g<8, true>(tk, tv, q, ap, nk, st);
-            }
-        }
-        switch (G) {
-        case 1: return launch_attend_tc_g<1, false>(tk, tv, q, ap, nk, st);
-        case 2: return launch_attend_tc_g<2, false>(tk, tv, q, ap, nk, st);
-        case 4: return launch_attend_tc_g<4, false>(tk, tv, q, ap, nk, st);
-        default: return launch_attend_tc_g<8, false>(tk, tv, q, ap, nk, st);
-        }
+        return launch_attend_tc(G, scale == 0.f, a.heads_per_unit, tk, tv, q, ap, cache->num_kv_heads, st);
     }
     const bool w2 = a.warps == 2;
     switch (G) {

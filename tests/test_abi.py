@@ -74,9 +74,16 @@ def test_host_side_validation_of_the_widened_entry_points():
     assert attn(Hq=24) == PA_EUNSUPPORTED                 # group size 3
     assert attn(q=18) == PA_EUNSUPPORTED                  # q not 16-byte aligned
     assert attn(scale=float("nan")) == PA_EINVAL
-    # requests x column chunks > 65535: 40000 x 2 chunks of 32 columns (48 per request) on the mma.sync kernel, and
-    # 70000 x 1 chunk of 128 on the tcgen05 one (which the automatic choice takes from 64 columns)
-    assert attn(R=40000, T=40000, maxq=12) == PA_EUNSUPPORTED
+    # requests x column chunks > 65535: 40000 x 2 chunks of 32 columns (48 per request) on the mma.sync
+    # kernel (chosen by the knob), 70000 x 1 chunk of 16 columns on it (the automatic choice below 17
+    # columns), and 70000 x 1 unit of two heads' 64 columns on the tcgen05 kernel
+    from paged_kv_cache_333_b200._abi import PA_ATTENTION_KERNEL_MMA
+    prev = lib.pa_attention_set_kernel(PA_ATTENTION_KERNEL_MMA)
+    try:
+        assert attn(R=40000, T=40000, maxq=12) == PA_EUNSUPPORTED
+    finally:
+        lib.pa_attention_set_kernel(prev)
+    assert attn(R=70000, T=70000, maxq=4) == PA_EUNSUPPORTED
     assert attn(R=70000, T=70000, maxq=16) == PA_EUNSUPPORTED
     assert attn(maxlen=32768) == PA_EWORKSPACE            # split-K needs scratch, none given
     assert lib.pa_attention_workspace_bytes(64, 256, 4, 32, 600, c) == 0

@@ -153,6 +153,16 @@ def test_attention_up_to_64_columns(pa, G, scale, part):
     assert pa.pa_get_device_error(clear=True) == 0
 
 
+def test_attention_odd_kv_heads(pa):
+    """Three KV heads (group size 2) and at most 64 columns per request: the
+    tcgen05 kernel cannot pair the heads and keeps one head per work unit."""
+    lens = [1, 40, 300, 77, 129]
+    q, kc, vc, bt, qsl, n = _case(95, lens, [1, 12, 32, 5, 32], 16, 6, 3)
+    ref = oracle.attention(q, kc, vc, bt, qsl, n, SCALE)
+    _check(_run(pa, q, kc, vc, bt, qsl, n), ref, "3 KV heads")
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
 def test_attention_whole_prefill(pa):
     """q_len = n: the first rows see a handful of tokens, the last all."""
     lens = [1, 16, 31, 160]
