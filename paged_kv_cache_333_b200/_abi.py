@@ -418,8 +418,9 @@ _ATTENTION_KERNELS = {"mma": PA_ATTENTION_KERNEL_MMA, "tcgen05": PA_ATTENTION_KE
 def pa_attention_set_kernel(kind: str) -> str:
     """Select the pa_attention kernel: "auto" (default: "tcgen05" from
     PA_ATTENTION_TCGEN05_MIN_COLUMNS (row, head) columns per request, else
-    "mma"), "mma" (8 columns per warp on mma.sync) or "tcgen05" (128 columns
-    per CTA, accumulators in tensor memory); returns the previous setting."""
+    "mma"), "mma" (8 columns per warp on mma.sync) or "tcgen05" (persistent,
+    work units of 128 MMA rows, S, P and O in tensor memory); returns the
+    previous setting.  The setting is process-wide."""
     prev = lib.pa_attention_set_kernel(_ATTENTION_KERNELS[kind])
     return {v: k for k, v in _ATTENTION_KERNELS.items()}[prev]
 

@@ -379,7 +379,6 @@ int launch_attend_g(const CUtensorMap &tk, const CUtensorMap &tv, const pa::Atte
     return launch_row_merge(ap, stream);
 }
 
-// The tensor-memory variant (attend_tc.cuh): 128 columns per CTA, one CTA per SM.
 // The q rows as a 3-D tensor (dim, head, row) for the tcgen05 kernel's TMA
 // loads of its q tiles: boxes of (64 dims, G heads, 64 / G rows), i.e. 64
 // columns, the 128-byte swizzle, rows past num_tokens read as zeros.
