@@ -17,13 +17,16 @@ attention.  Inputs are resident in HBM when the timed region starts.
 --impl reference times the CPU oracle (its (sequence, head) pairs split over
 the host's cores) on a bounded sample of the same workload.  The default run
 also reports the oracle in cpu_baseline, with a one-thread timing beside it,
-and times the 32K long-context decode under per_config.  With torchrun
+and times, under per_config, the 32K long-context decode and two variants of
+the chat step: the FP8 cache's decode and 16 query rows per sequence through
+pa_attention.  With torchrun
 (N > 1) every rank runs its own replica (the path does not shard; no
 collective is needed) and the time is the max over ranks.
 """
 from __future__ import annotations
 
 import argparse
+import copy
 import datetime
 import json
 import os
@@ -86,6 +89,10 @@ def parse_args():
                     help="comma-separated workloads whose bf16 decode is also timed in this run and reported "
                          "under per_config (auto = the 32K long-context one when the main run is the chat "
                          "decode; none = no extra)")
+    ap.add_argument("--related", default="auto",
+                    help="comma-separated variants of the main workload also timed in this run and reported "
+                         "under per_config: fp8 (the FP8 cache's decode), rows16 (16 query rows per sequence "
+                         "through pa_attention); auto = both when the main run is the chat bf16 decode; none")
     args = ap.parse_args()
     if args.queries > 1 and args.kv_dtype == "fp8":
         ap.error("--queries > 1 runs pa_attention, which reads a bf16 cache: use --kv-dtype bf16")
@@ -609,6 +616,44 @@ def extra_configs(args) -> list:
     return [n for n in names if n != args.config]
 
 
+def related_runs(args) -> list:
+    """Variants of the main workload timed after it: by default the FP8
+    cache's decode and 16 query rows per sequence (pa_attention), when the
+    main run is the bf16 chat decode."""
+    if args.related == "auto":
+        default = args.config == "chat" and args.queries == 1 and args.kv_dtype == "bf16" and not args.part_tokens
+        return ["fp8", "rows16"] if default else []
+    if args.related in ("", "none"):
+        return []
+    return [n.strip() for n in args.related.split(",") if n.strip() in ("fp8", "rows16")]
+
+
+def time_related(name, args, world, rank, local) -> dict:
+    """The main workload with the FP8 cache (name "fp8") or with 16 query
+    rows per sequence (name "rows16"), staged and timed as the main run is,
+    without its end-to-end, per-op and CPU legs.  Returns the per_config
+    record."""
+    sub = copy.copy(args)
+    sub.no_e2e, sub.no_per_op, sub.no_cpu_baseline = True, True, True
+    sub.extra_configs, sub.related = "none", "none"
+    if name == "fp8":
+        sub.kv_dtype = "fp8"
+    else:
+        sub.queries = 16
+    r, _ = run_ours(sub, world, rank, local)
+    rec = {"workload": r["config"]["workload"]}
+    for key in ("value", "unit", "ms_per_step", "dtype", "decode_tokens_per_s_per_layer", "roofline",
+                "gpu_launches", "clocks"):
+        if key in r:
+            rec[key] = r[key]
+    if "attention" in r.get("per_op", {}):
+        rec["attention"] = r["per_op"]["attention"]
+    rec["attention_kernel"] = r["config"].get("attention_kernel")
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
 def time_decode_config(name, args, world, local) -> dict:
     """The bf16 decode step of workload `name`, staged and timed like the main
     one: --layers distinct layer caches, a CUDA graph of the whole step
@@ -812,6 +857,9 @@ def main():
             for name in extra_configs(args):
                 torch.cuda.empty_cache()
                 result.setdefault("per_config", {})[name] = time_decode_config(name, args, world, local)
+            for name in related_runs(args):
+                torch.cuda.empty_cache()
+                result.setdefault("per_config", {})[name] = time_related(name, args, world, rank, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline and args.queries == 1:
                 result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
             if rank == 0:

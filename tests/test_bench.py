@@ -145,6 +145,15 @@ def test_split_oracle_layer_computes_every_pair_once(monkeypatch):
     assert len(pairs) == len(expect) and {tuple(p) for p in pairs} == expect
 
 
+def test_related_runs_default_to_fp8_and_sixteen_rows():
+    args = bench.argparse.Namespace(related="auto", config="chat", queries=1, kv_dtype="bf16", part_tokens=0)
+    assert bench.related_runs(args) == ["fp8", "rows16"]
+    for change in ({"config": "long"}, {"queries": 4}, {"kv_dtype": "fp8"}, {"part_tokens": 640}):
+        assert bench.related_runs(bench.argparse.Namespace(**{**vars(args), **change})) == []
+    assert bench.related_runs(bench.argparse.Namespace(**{**vars(args), "related": "none"})) == []
+    assert bench.related_runs(bench.argparse.Namespace(**{**vars(args), "related": "rows16,other"})) == ["rows16"]
+
+
 def test_extra_configs_default_to_the_long_context_decode():
     args = bench.argparse.Namespace(extra_configs="auto", config="chat", queries=1, kv_dtype="bf16", part_tokens=0)
     assert bench.extra_configs(args) == ["long"]
