@@ -8,10 +8,13 @@
 //
 // Work decomposition.  A column is one (query row, query head of the KV group)
 // pair, c = i * G + g, as in attend.cuh.  A work unit is one (split-K
-// partition, KV head, request, chunk of 128 columns); its token range is
-// streamed in 64-token tiles:
-//   S = Q K^T    M = 128 columns, N = 64 tokens, K = 128 dims: 8 MMAs of K = 16
-//   O += P V     M = 128 columns, N = 128 dims, K = 64 tokens: 4 MMAs of K = 16
+// partition, KV head, request, chunk of 128 columns), or, when every request
+// has at most 64 columns and the KV head count is even, one (partition, pair
+// of KV heads, request) with each head's columns in 64 of the 128 MMA rows
+// (HP = 2, described at the kernel).  Its token range is streamed in tiles
+// of 64 rows (64 tokens of the head, or 32 tokens of each of the two):
+//   S = Q K^T    M = 128 columns, N = 64 rows, K = 128 dims: 8 MMAs of K = 16
+//   O += P V     M = 128 columns, N = 128 dims, K = 64 rows: 4 MMAs of K = 16
 // (tcgen05.mma.cta_group::1.kind::f16, bf16 operands, fp32 accumulators in
 // tensor memory).  Q and K are K-major and V is MN-major in shared memory, in
 // the 128-byte swizzled layout the TMA loads write: rows of 128 bytes, 16-byte
@@ -27,16 +30,17 @@
 // loads in flight for about a third of its life (set-up, first load,
 // epilogue).
 //
-// Roles (320 threads):
+// Roles (352 threads):
 //   warps 0-3  softmax: thread t owns column t of the unit, which is tensor-
 //              memory lane t (a warp may only read lanes 32 * (warp % 4) ..
 //              + 31).  Per tile: read its S row (64 fp32), mask, online
 //              softmax with a lazily moved reference max, write its P row
 //              (bf16 pairs) to tensor memory; per unit: leave (m_ref, l) in
 //              tensor memory for the epilogue warps and go on to the next;
-//   warp 4     producer: per unit, the block-table slice into shared memory,
-//              the q tile by TMA (two buffers), and the 64-token K/V tiles
-//              into a 5-stage ring, by TMA for whole tiles of blocks >= 8
+//   warps 4, 10 producers: per unit, the block-table slice into shared memory
+//              (each its own copy), the q tile by TMA (two buffers; warp 4),
+//              and the K/V tiles into a 5-stage ring (warp 4 the even slots,
+//              warp 10 the odd ones), by TMA for whole tiles of blocks >= 8
 //              tokens, else by a cp.async gather that zero-fills the rows past
 //              the range;
 //   warp 5     allocates tensor memory; one thread issues the MMAs;
@@ -90,7 +94,6 @@ constexpr int kTmemPTc = kTmemOTc + 2 * kD;      // P of tile t in [384 + 32 (t 
 constexpr int kTmemMlTc = kTmemPTc + 2 * 32;     // (m_ref, l) of unit k at 448 + 2 (k % 2)
 static_assert(kTmemMlTc + 4 <= kTmemColsTc, "tensor memory columns");
 constexpr int kTcThreads = 352;
-constexpr int kTcSoftmaxThreads = 128;
 constexpr int kTcProducerWarp = 4;
 constexpr int kTcMmaWarp = 5;
 constexpr int kTcEpilogueWarp0 = 6;  // warps 6-9: lane quarters 2, 3, 0, 1
