@@ -363,15 +363,41 @@ struct TcUnit {
     bool work;  // at least one tile
 };
 
+// n / d for 0 <= n < 2^31 by a multiply-high, an add and a shift, the
+// divisor's constants set on the host (the round-up method of Granlund and
+// Montgomery, "Division by invariant integers using multiplication", 1994):
+// with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1, which fits in
+// 32 bits, n / d = (umulhi(m, n) + n) >> s.  Every role decodes each work
+// unit at its start; the GPU has no integer divide instruction, and the
+// emulated division by a runtime divisor is a long dependent chain on the
+// path from one unit's last tile to the next unit's first.
+struct FastDiv {
+    uint32_t d, m, s;
+};
+inline FastDiv make_fast_div(uint32_t d) {
+    uint32_t s = 0;
+    while ((uint64_t(1) << s) < d)
+        ++s;
+    const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << s) - d)) / d + 1;
+    return FastDiv{d, static_cast<uint32_t>(m), s};
+}
+__device__ __forceinline__ int fast_div(int n, const FastDiv &f) {
+    return static_cast<int>((__umulhi(static_cast<uint32_t>(n), f.m) + static_cast<uint32_t>(n)) >> f.s);
+}
+// The divisors of the unit number: partitions, head groups, column chunks.
+struct TcDivs {
+    FastDiv parts, groups, chunks;
+};
+
 // The unit's raw metadata, loaded one unit ahead so that its latency
 // overlaps the current unit's tiles; tc_unit() derives the rest.
 struct TcRaw {
     int u, q0, q1, n;
 };
-__device__ __forceinline__ TcRaw tc_raw(const AttendParams &ap, int u) {
+__device__ __forceinline__ TcRaw tc_raw(const AttendParams &ap, const TcDivs &dv, int u) {
     TcRaw raw{u, 0, 0, 0};
     if (u < ap.num_units) {
-        const int r = (u / ap.d.num_parts / ap.head_groups) / ap.chunks;
+        const int r = fast_div(fast_div(fast_div(u, dv.parts), dv.groups), dv.chunks);
         raw.q0 = ap.query_start_loc[r];
         raw.q1 = ap.query_start_loc[r + 1];
         raw.n = ap.d.seq_lens[r];
@@ -380,16 +406,16 @@ __device__ __forceinline__ TcRaw tc_raw(const AttendParams &ap, int u) {
 }
 
 template <int G, int HP>
-__device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &raw) {
+__device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcDivs &dv, const TcRaw &raw) {
     const DecodeParams &p = ap.d;
     TcUnit w{};
     const int u = raw.u;
-    w.part = u % p.num_parts;
-    int rest = u / p.num_parts;
-    w.h = rest % ap.head_groups;
-    rest /= ap.head_groups;
-    w.r = rest / ap.chunks;
-    w.chunk = rest % ap.chunks;
+    int rest = fast_div(u, dv.parts);
+    w.part = u - rest * p.num_parts;
+    int next = fast_div(rest, dv.groups);
+    w.h = rest - next * ap.head_groups;
+    w.r = fast_div(next, dv.chunks);
+    w.chunk = next - w.r * ap.chunks;
     int n = raw.n;  // clamped as clamp_seq_len does
     {
         const int64_t cap64 = static_cast<int64_t>(p.max_blocks_per_seq) * p.block_size;
@@ -443,7 +469,7 @@ __device__ __forceinline__ TcUnit tc_unit(const AttendParams &ap, const TcRaw &r
 template <int G, bool kZeroScale, int HP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_q, const AttendParams ap) {
+                 const __grid_constant__ CUtensorMap tm_q, const AttendParams ap, const TcDivs dv) {
     static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
     static_assert(HP == 1 || HP == 2, "heads per work unit");
     constexpr int kTokH = kTokTc / HP;   // tokens of one head per tile
@@ -509,10 +535,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const uint64_t pol = l2_evict_first_policy();
         int T = 0, k = 0;
         bool dead = false;
-        TcRaw raw = tc_raw(ap, blockIdx.x);
+        TcRaw raw = tc_raw(ap, dv, blockIdx.x);
         for (int u = blockIdx.x; u < ap.num_units && !dead; u += gridDim.x) {
-            const TcUnit w = tc_unit<G, HP>(ap, raw);
-            raw = tc_raw(ap, u + gridDim.x);
+            const TcUnit w = tc_unit<G, HP>(ap, dv, raw);
+            raw = tc_raw(ap, dv, u + gridDim.x);
             if (w.bad && w.part == 0 && w.h == 0 && w.chunk == 0 && lane == 0)
                 flag_error(PA_DEVERR_QUERY_LOC);
             if (!w.work)
@@ -665,10 +691,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
             int T = 0, k = 0;
             int prev_t = -1, prev_k = 0;
             bool prev_first = false, prev_last = false;
-            TcRaw raw = tc_raw(ap, blockIdx.x);
+            TcRaw raw = tc_raw(ap, dv, blockIdx.x);
             for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
-                const TcUnit w = tc_unit<G, HP>(ap, raw);
-                raw = tc_raw(ap, u + gridDim.x);
+                const TcUnit w = tc_unit<G, HP>(ap, dv, raw);
+                raw = tc_raw(ap, dv, u + gridDim.x);
                 if (!w.work)
                     continue;
                 const int qb = k & 1;
@@ -719,10 +745,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         bool ok = true;
         int k = 0;
-        TcRaw raw = tc_raw(ap, blockIdx.x);
+        TcRaw raw = tc_raw(ap, dv, blockIdx.x);
         for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
-            const TcUnit w = tc_unit<G, HP>(ap, raw);
-            raw = tc_raw(ap, u + gridDim.x);
+            const TcUnit w = tc_unit<G, HP>(ap, dv, raw);
+            raw = tc_raw(ap, dv, u + gridDim.x);
             if (!w.work)
                 continue;
             const int ob = k & 1;
@@ -803,10 +829,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const float masked = pos ? -INFINITY : INFINITY;
         bool ok = true;
         int T = 0, k = 0;
-        TcRaw raw = tc_raw(ap, blockIdx.x);
+        TcRaw raw = tc_raw(ap, dv, blockIdx.x);
         for (int u = blockIdx.x; u < ap.num_units && ok; u += gridDim.x) {
-            const TcUnit w = tc_unit<G, HP>(ap, raw);
-            raw = tc_raw(ap, u + gridDim.x);
+            const TcUnit w = tc_unit<G, HP>(ap, dv, raw);
+            raw = tc_raw(ap, dv, u + gridDim.x);
             if (!w.work)
                 continue;
             const int c = w.col0 + threadIdx.x % kColsH;

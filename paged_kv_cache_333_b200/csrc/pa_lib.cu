@@ -424,8 +424,11 @@ int launch_attend_tc_g(const CUtensorMap &tk, const CUtensorMap &tv, const void 
     ap.head_groups = num_kv_heads / HP;
     ap.num_units = static_cast<int32_t>(units);
     const dim3 grid(static_cast<unsigned>(std::min<int64_t>(units, sm_count())));
+    const pa::TcDivs dv = {pa::make_fast_div(static_cast<uint32_t>(ap.d.num_parts)),
+                           pa::make_fast_div(static_cast<uint32_t>(ap.head_groups)),
+                           pa::make_fast_div(static_cast<uint32_t>(ap.chunks))};
     cudaError_t e = launch_pdl(pa::attend_tc_kernel<G, kZeroScale, HP>, grid, dim3(pa::kTcThreads), pa::kAttendTcSmemBytes,
-                               stream, tk, tv, tq, ap);
+                               stream, tk, tv, tq, ap, dv);
     if (e != cudaSuccess)
         return cuda_fail(e, "attend_tc_kernel launch");
     return launch_row_merge(ap, stream);
