@@ -163,6 +163,22 @@ def test_attention_odd_kv_heads(pa):
     assert pa.pa_get_device_error(clear=True) == 0
 
 
+@pytest.mark.parametrize("B,part", [(16, 3072), (8, 1536)])
+def test_attention_partition_fills_the_table_slice(pa, B, part):
+    """Partitions of exactly 192 blocks, the most a tcgen05 CTA stages: a
+    request that fills one partition exactly, one that spills a single token
+    into a second, and longer ones, 16 rows each."""
+    lens = [part, part + 1, part + part // 2, 2 * part]
+    q, kc, vc, bt, qsl, n = _case(79 + B, lens, [16] * 4, B, 32, 8)
+    ref = oracle.attention(q, kc, vc, bt, qsl, n, SCALE)
+    prev = pa.pa_decode_set_partition_tokens(part)
+    try:
+        _check(_run(pa, q, kc, vc, bt, qsl, n), ref, f"B={B} part={part}")
+    finally:
+        pa.pa_decode_set_partition_tokens(prev)
+    assert pa.pa_get_device_error(clear=True) == 0
+
+
 def test_attention_whole_prefill(pa):
     """q_len = n: the first rows see a handful of tokens, the last all."""
     lens = [1, 16, 31, 160]
